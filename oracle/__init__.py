@@ -1,0 +1,125 @@
+"""CPU oracle of the Graph Machine sparse layer (SER, SEA forward, SEA backward).
+
+TEST INFRASTRUCTURE. Only the tests, the package smoke check and the benchmark's CPU-baseline
+leg import this module. It wraps the plain C library built from gm_oracle.c (compiled on
+first use if missing or stale); the CUDA library shares no code with it.
+
+Every function takes CPU tensors or numpy arrays in the library's layouts (features
+[B, n, H, d] fp32 or bf16, edges [B, n, k, s] int32 + fp32) and returns numpy arrays.
+Features are widened exactly to fp32 before the call; SEA and its backward compute in fp64.
+The definitions, the citations and the readings of the pages are in gm_oracle.c's header.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(_build.build())
+        i32p = np.ctypeslib.ndpointer(np.int32, flags="C_CONTIGUOUS")
+        f32p = np.ctypeslib.ndpointer(np.float32, flags="C_CONTIGUOUS")
+        f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
+        ci = ctypes.c_int
+        lib.oracle_num_threads.restype = ci
+        lib.oracle_ser.restype = ctypes.c_int64
+        lib.oracle_ser.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci, ci, ci, ci]
+        lib.oracle_sea_forward.restype = ctypes.c_int64
+        lib.oracle_sea_forward.argtypes = [f32p, f32p, f32p, i32p, f32p, ci, ci, ci, ci, ci, ci,
+                                           ctypes.c_double, ctypes.c_void_p, ctypes.c_int64,
+                                           f64p, f64p]
+        lib.oracle_sea_backward.restype = ctypes.c_int64
+        lib.oracle_sea_backward.argtypes = [f32p, f32p, f32p, f32p, i32p, f32p, ci, ci, ci, ci,
+                                            ci, ci, ctypes.c_double, f64p, f64p, f64p, f64p]
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """Threads the oracle's parallel loops use (OMP_NUM_THREADS or all cores)."""
+    return int(_load().oracle_num_threads())
+
+
+def _np(x, dtype):
+    """CPU tensor / array -> contiguous numpy array of `dtype` (bf16 widened exactly)."""
+    if hasattr(x, "detach"):
+        x = x.detach().cpu()
+        if dtype == np.float32:
+            x = x.float()
+        x = x.numpy()
+    return np.ascontiguousarray(np.asarray(x), dtype=dtype)
+
+
+def ser(a1_idx, a1_w, a2_idx, a2_w, s1: int):
+    """A' = Sparsify_s1(A1 A2) per (b, i, h). Returns (idx int32, w fp32, bad_refs)."""
+    i1, w1 = _np(a1_idx, np.int32), _np(a1_w, np.float32)
+    i2, w2 = _np(a2_idx, np.int32), _np(a2_w, np.float32)
+    B, n, k, s2 = i1.shape
+    s3 = i2.shape[3]
+    assert i2.shape[:3] == (B, n, k) and w1.shape == i1.shape and w2.shape == i2.shape
+    out_i = np.zeros((B, n, k, s1), np.int32)
+    out_w = np.zeros((B, n, k, s1), np.float32)
+    bad = _load().oracle_ser(i1, w1, s2, i2, w2, s3, out_i, out_w, s1, B, n, k)
+    if bad < 0:
+        raise ValueError("s2*s3 exceeds the oracle's candidate buffer")
+    return out_i, out_w, int(bad)
+
+
+def sea_forward(q, k, v, idx, w, scale: float | None = None, rows=None):
+    """SEA forward in fp64. Returns (o [R,hq,d], lse [R,hq], bad_refs).
+
+    R = B*n rows in order, or len(rows) for the flat positions b*n+i listed in `rows`.
+    """
+    qa, ka, va = _np(q, np.float32), _np(k, np.float32), _np(v, np.float32)
+    ia, wa = _np(idx, np.int32), _np(w, np.float32)
+    B, n, hq, d = qa.shape
+    hkv, s = ia.shape[2], ia.shape[3]
+    assert ka.shape == (B, n, hkv, d) and va.shape == ka.shape and wa.shape == ia.shape
+    assert hq % hkv == 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if rows is None:
+        R, rp, keep = B * n, None, None
+    else:
+        keep = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        R, rp = len(keep), keep.ctypes.data_as(ctypes.c_void_p)
+    o = np.zeros((R, hq, d), np.float64)
+    lse = np.zeros((R, hq), np.float64)
+    bad = _load().oracle_sea_forward(qa, ka, va, ia, wa, s, B, n, hq, hkv, d, float(scale),
+                                     rp, R, o, lse)
+    return o, lse, int(bad)
+
+
+def sea_backward(q, k, v, dout, idx, w, scale: float | None = None):
+    """SEA backward in fp64. Returns (dq, dk, dv, dlogw, bad_refs) in the input layouts."""
+    qa, ka, va = _np(q, np.float32), _np(k, np.float32), _np(v, np.float32)
+    ga = _np(dout, np.float32)
+    ia, wa = _np(idx, np.int32), _np(w, np.float32)
+    B, n, hq, d = qa.shape
+    hkv, s = ia.shape[2], ia.shape[3]
+    assert ga.shape == qa.shape and ka.shape == (B, n, hkv, d) and va.shape == ka.shape
+    assert hq % hkv == 0
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = np.zeros(qa.shape, np.float64)
+    dk = np.zeros(ka.shape, np.float64)
+    dv = np.zeros(va.shape, np.float64)
+    dlw = np.zeros(ia.shape, np.float64)
+    bad = _load().oracle_sea_backward(qa, ka, va, ga, ia, wa, s, B, n, hq, hkv, d,
+                                      float(scale), dq, dk, dv, dlw)
+    return dq, dk, dv, dlw, int(bad)
+
+
+def ser_sea_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, s1: int, scale=None, rows=None):
+    """SER followed by SEA on its output. Returns (idx, w, o, lse, bad_refs)."""
+    oi, ow, bad1 = ser(a1_idx, a1_w, a2_idx, a2_w, s1)
+    o, lse, bad2 = sea_forward(q, k, v, oi, ow, scale, rows)
+    return oi, ow, o, lse, bad1 + bad2
