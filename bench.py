@@ -1,0 +1,518 @@
+#!/usr/bin/env python
+"""Benchmark of the Graph Machine sparse-layer hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+  1. gm_ser_sea_forward  - SER (two-hop referral, merge, top-s1) fused with SEA forward,
+  2. gm_sea_backward     - zero-fill of dK/dV, then the SEA backward (dq, dK/dV scatter-add,
+                           d ln w) on the refreshed edges with upstream gradient dO.
+Metric: tokens/s per sparse layer (B*n tokens per step / step time), summed over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier +
+torch.cuda.synchronize() on both sides, timed with CUDA events on the launching stream, max
+over ranks. The inputs (q, k, v, dO, edges: 0.55 GB per step at the default workload) are
+larger than the 126 MB L2, so no flush runs between steps. Per-call CUDA events inside the
+timed region give each call's average duration, which with the compulsory bytes counted
+from the actual index tensors gives the HBM roofline fraction. SM clocks and throttle
+reasons are sampled through NVML during the timed region.
+
+`--impl reference` times the CPU oracle (the plain C restatement used by the tests) on the
+host cores on a bounded sample of the same workload, in the same units.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from sparse_dynamic_routing_b200 import inputs as I  # noqa: E402
+
+DEFAULT_WORKLOAD = "layer_b8_n4096_s4_local"
+METRIC = "SER+SEA tokens/s per sparse layer (1xB200) and achieved HBM GB/s vs ~8 TB/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(I.WORKLOADS))
+    p.add_argument("--e2e-steps", type=int, default=5)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle sample")
+    return p.parse_args(argv)
+
+
+# ---- distributed plumbing ------------------------------------------------------------------
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def shard_seed(wl: I.Workload, rank: int) -> I.Workload:
+    """Weak scaling: every rank runs the full per-GPU workload on its own independent draw."""
+    return wl if rank == 0 else wl.with_(seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, local: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[local])
+
+
+# ---- clocks ----------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Polls SM clock, power and clock-event reasons through NVML (read-only)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            phys = device_index
+            if vis:
+                ids = [v.strip() for v in vis.split(",") if v.strip()]
+                if device_index < len(ids) and ids[device_index].isdigit():
+                    phys = int(ids[device_index])
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(phys)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+        self.thread = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                t = time.perf_counter()
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                pw = nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+                self.samples.append((t, mhz, rs, pw))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.thread.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.thread.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed_region"
+        if len(inside) < 3:  # a short timed region: widen to the samples around it
+            pad = 0.25
+            inside = [s for s in self.samples if t0 - pad <= s[0] <= t1 + pad]
+            window = "timed_region+-250ms"
+        if not inside:
+            return {"error": "no samples"}
+        reasons = 0
+        for s in inside:
+            reasons |= s[2]
+        names = sorted(k for k, v in self.REASONS.items() if reasons & v and k != "gpu_idle")
+        return {
+            "sm_mhz": statistics.median(s[1] for s in inside),
+            "sm_max_mhz": self.max_mhz,
+            "reasons": names,
+            "power_w_max": max(s[3] for s in inside),
+            "samples": len(inside),
+            "window": window,
+            "source": "nvml",
+        }
+
+
+# ---- byte accounting --------------------------------------------------------------------------
+
+def distinct_rows(idx: np.ndarray, w: np.ndarray, n: int) -> int:
+    """Distinct (b, t, h) rows referenced by the active slots of an edge tensor [B,n,H,s]."""
+    B, _, H, s = idx.shape
+    act = w > 0
+    b = np.broadcast_to(np.arange(B)[:, None, None, None], idx.shape)
+    h = np.broadcast_to(np.arange(H)[None, None, :, None], idx.shape)
+    keys = (b[act].astype(np.int64) * n + idx[act]) * H + h[act]
+    return int(np.unique(keys).size)
+
+
+def compulsory_bytes(wl: I.Workload, a1_idx, a1_w, ap_idx, ap_w) -> dict:
+    """Minimum DRAM bytes of each call: every input byte read once, every output written once,
+    gathered rows counted once per distinct row actually referenced."""
+    es = 2 if wl.dtype == "bf16" else 4
+    B, n, hq, hkv, d = wl.B, wl.n, wl.hq, wl.hkv, wl.d
+    tok = B * n
+    feat_q = tok * hq * d * es
+    kv_row = d * es
+    a2_rows = distinct_rows(a1_idx, a1_w, n)
+    kv_rows = distinct_rows(ap_idx, ap_w, n)
+    fwd = {
+        "q": feat_q, "o": feat_q, "lse": tok * hq * 4,
+        "a1": tok * hkv * wl.s2 * 8, "a2_rows": a2_rows * wl.s3 * 8,
+        "a_prime": tok * hkv * wl.s1 * 8, "kv_rows": kv_rows * kv_row * 2,
+    }
+    zero = {"dk_dv": 2 * tok * hkv * d * 4}
+    bwd = {
+        "q_dout": 2 * feat_q, "edges": tok * hkv * wl.s1 * 8, "kv_rows": kv_rows * kv_row * 2,
+        "dq": tok * hq * d * 4, "dlogw": tok * hkv * wl.s1 * 4,
+        "dk_dv_rows": kv_rows * d * 4 * 2,
+    }
+    logical_fwd = (2 * hq * d * es + hq * 4
+                   + hkv * (wl.s2 * 8 + wl.s2 * wl.s3 * 8 + wl.s1 * 8 + wl.s1 * 2 * kv_row)) * tok
+    return {
+        "fused_forward": sum(fwd.values()), "zero_fill": sum(zero.values()),
+        "backward": sum(bwd.values()), "fused_forward_logical": logical_fwd,
+        "kv_rows_touched": kv_rows, "kv_rows_total": tok * hkv, "a2_rows_touched": a2_rows,
+        "detail": {"fused_forward": fwd, "zero_fill": zero, "backward": bwd},
+    }
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    cdir = os.path.join(ROOT, "sparse_dynamic_routing_b200", "csrc")
+    for name in sorted(os.listdir(cdir)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(cdir, name), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    cur = source_hash()
+    for line in open(path):
+        if line.startswith("#") or not line.strip():
+            continue
+        f = dict(kv.split("=", 1) for kv in line.split())
+        if f.get("kernel") == kernel and f.get("workload") == workload:
+            if f.get("source") != cur:
+                return None
+            return float(f["dram_bytes_per_launch"])
+    return None
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---- CPU oracle (baseline / reference arm) -------------------------------------------------------
+
+def oracle_sample_step(wl: I.Workload, x: dict) -> None:
+    import oracle
+    oi, ow, _ = oracle.ser(x["a1_idx"], x["a1_w"], x["a2_idx"], x["a2_w"], wl.s1)
+    oracle.sea_forward(x["q"], x["k"], x["v"], oi, ow, wl.scale)
+    oracle.sea_backward(x["q"], x["k"], x["v"], x["dout"], oi, ow, wl.scale)
+
+
+def cpu_baseline(wl: I.Workload, seconds: float) -> dict:
+    """Oracle (SER + SEA forward + SEA backward) on one sequence of the workload, repeated."""
+    import oracle
+    sample = wl.with_(B=1)
+    x = I.make(sample, grad=True)
+    x = {k: (v.float().numpy() if v.dtype == torch.bfloat16 else v.numpy()) for k, v in x.items()}
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_sample_step(sample, x)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 50:
+            break
+    tokens = reps * sample.n
+    return {
+        "value": tokens / el, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+        "sample": f"1 of {wl.B} sequences ({sample.n} tokens, same recipe) x {reps} passes of "
+                  f"SER + SEA fwd + SEA bwd in the C oracle ({el:.1f} s wall)",
+    }
+
+
+# ---- our arm -------------------------------------------------------------------------------------
+
+def run_ours(args):
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    import sparse_dynamic_routing_b200 as gm
+    gm.load_library()
+
+    wl = shard_seed(I.WORKLOADS[args.workload], rank)
+    assert wl.kind == "ser_sea", "the bench step is SER->SEA forward + SEA backward"
+    x = I.make(wl, grad=True)
+    g = {k: v.to(dev) for k, v in x.items()}
+    B, n, hq, hkv, d = wl.B, wl.n, wl.hq, wl.hkv, wl.d
+    f32 = torch.float32
+    ap_i = torch.empty((B, n, hkv, wl.s1), dtype=torch.int32, device=dev)
+    ap_w = torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev)
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, n, hq), dtype=f32, device=dev)
+    dq = torch.empty((B, n, hq, d), dtype=f32, device=dev)
+    dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev)
+    dv = torch.empty_like(dk)
+    dlw = torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        gm.gm_ser_sea_forward(g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], g["a2_idx"],
+                              g["a2_w"], wl.s1, wl.scale, out_idx=ap_i, out_w=ap_w, o=o, lse=lse,
+                              stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], ap_i, ap_w, wl.scale, dq=dq, dk=dk,
+                           dv=dv, dlogw=dlw, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    launches_per_step = 3  # fused forward, zero-fill, backward
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    gm.gm_check_device_errors(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world, local)
+    torch.cuda.synchronize(dev)
+    w0 = time.perf_counter()
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.perf_counter()
+    barrier(world, local)
+    sampler.stop()
+    clocks = sampler.summary(w0, w1)
+    gm.gm_check_device_errors(stream)
+
+    ms_local = t_start.elapsed_time(t_end)
+    ms = max_over_ranks(ms_local, world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    tokens = B * n * world
+    value = tokens * args.steps / (ms / 1e3)
+
+    # byte accounting from the actual edge tensors (outside the timed region)
+    cb = compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ap_i.cpu().numpy(),
+                          ap_w.cpu().numpy())
+    peak, peak_kind = peak_hbm()
+    calls = {
+        "fused_forward": {"kernel": "ser_sea_fwd_kernel", "us": fwd_ms * 1e3,
+                          "bytes": cb["fused_forward"]},
+        "backward": {"kernel": "zero2_kernel+sea_bwd_kernel", "us": bwd_ms * 1e3,
+                     "bytes": cb["backward"] + cb["zero_fill"]},
+    }
+    for c in calls.values():
+        c["GBps"] = c["bytes"] / (c["us"] * 1e-6) / 1e9
+        c["frac"] = c["GBps"] / peak
+    calls["fused_forward"]["logical_bytes"] = cb["fused_forward_logical"]
+    calls["fused_forward"]["logical_GBps"] = (cb["fused_forward_logical"]
+                                              / (fwd_ms * 1e-3) / 1e9)
+    dom_name = max(calls, key=lambda k: calls[k]["us"])
+    dom = calls[dom_name]
+    roofline = {
+        "bound": "hbm", "kernel": dom["kernel"], "call": dom_name,
+        "achieved": round(dom["GBps"], 1), "peak": peak, "unit": "GB/s",
+        "frac": round(dom["frac"], 4), "peak_kind": peak_kind,
+        "traffic": ncu_traffic(dom["kernel"], wl.name),
+        "bytes_per_launch": dom["bytes"], "bytes_kind": "compulsory",
+    }
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(gm, wl, x, dev, stream, args.e2e_steps, world)
+
+    result = None
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_baseline(wl, args.cpu_seconds)
+        result = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+            if wl.dtype == "bf16" else "f32", "data": "synthetic",
+            "config": {
+                "workload": wl.name, "B_per_gpu": B, "n": n, "hq": hq, "hkv": hkv, "d": d,
+                "s1": wl.s1, "s2": wl.s2, "s3": wl.s3, "alpha": wl.alpha,
+                "local_frac": wl.local_frac, "step": "ser_sea_forward + sea_backward",
+                "global_batch": B * world, "seq_len": n, "parallelism": f"dp{world}",
+                "l2": "no flush; inputs larger than L2 "
+                      f"({(cb['detail']['backward']['q_dout'] + 2 * g['k'].numel() * g['k'].element_size()) / 1e6:.0f} MB read per step)",
+            },
+            "roofline": roofline,
+            "calls": {k: {kk: (round(vv, 3) if isinstance(vv, float) else vv)
+                          for kk, vv in c.items()} for k, c in calls.items()},
+            "kv_rows_touched_frac": cb["kv_rows_touched"] / cb["kv_rows_total"],
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks, "source_hash": source_hash(),
+        }
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return result
+
+
+def measure_e2e(gm, wl, x, dev, stream, steps, world):
+    """Same step through the public API with host buffers: pinned H2D of every input, the two
+    calls, D2H of every output, all inside the timed region."""
+    pin_in = {k: v.contiguous().pin_memory() for k, v in x.items()}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in x.items()}
+    B, n, hq, hkv, d = wl.B, wl.n, wl.hq, wl.hkv, wl.d
+    f32 = torch.float32
+    outs_dev = {
+        "ap_i": torch.empty((B, n, hkv, wl.s1), dtype=torch.int32, device=dev),
+        "ap_w": torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev),
+        "o": torch.empty_like(dev_in["q"]),
+        "lse": torch.empty((B, n, hq), dtype=f32, device=dev),
+        "dq": torch.empty((B, n, hq, d), dtype=f32, device=dev),
+        "dk": torch.empty((B, n, hkv, d), dtype=f32, device=dev),
+        "dv": torch.empty((B, n, hkv, d), dtype=f32, device=dev),
+        "dlw": torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev),
+    }
+    outs_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs_dev.items()}
+    h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
+    d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
+
+    def one():
+        for k, v in pin_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        od = outs_dev
+        gm.gm_ser_sea_forward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["a1_idx"],
+                              dev_in["a1_w"], dev_in["a2_idx"], dev_in["a2_w"], wl.s1, wl.scale,
+                              out_idx=od["ap_i"], out_w=od["ap_w"], o=od["o"], lse=od["lse"],
+                              stream=stream)
+        gm.gm_sea_backward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dout"], od["ap_i"],
+                           od["ap_w"], wl.scale, dq=od["dq"], dk=od["dk"], dv=od["dv"],
+                           dlogw=od["dlw"], stream=stream)
+        for k, v in od.items():
+            outs_host[k].copy_(v, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    return {"value": round(B * n * world * steps / (ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+# ---- reference arm: the CPU oracle --------------------------------------------------------------
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    wl = I.WORKLOADS[args.workload]
+    sample = wl.with_(B=1)
+    x = I.make(sample, grad=True)
+    x = {k: (v.float().numpy() if v.dtype == torch.bfloat16 else v.numpy()) for k, v in x.items()}
+    for _ in range(max(args.warmup, 0)):
+        oracle_sample_step(sample, x)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(sample, x)
+    el = time.perf_counter() - t0
+    value = sample.n * args.steps / el
+    cores = oracle.num_threads()
+    return {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "impl": "reference",
+        "config": {"workload": wl.name, "B_per_gpu": wl.B, "n": wl.n, "hq": wl.hq,
+                   "hkv": wl.hkv, "d": wl.d, "s1": wl.s1, "s2": wl.s2, "s3": wl.s3,
+                   "step": "ser_sea_forward + sea_backward", "global_batch": wl.B,
+                   "seq_len": wl.n, "parallelism": "host cores"},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": cores,
+                         "kind": "oracle",
+                         "sample": f"each step: 1 of {wl.B} sequences ({sample.n} tokens, same "
+                                   "recipe), SER + SEA fwd + SEA bwd in the C oracle"},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        res = run_reference(args)
+    else:
+        res = run_ours(args)
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

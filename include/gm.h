@@ -1,0 +1,182 @@
+/*
+ * gm.h - C ABI of the Graph Machine sparse-layer library for NVIDIA B200 (sm_100a).
+ *
+ * The library computes the data-parallel hot path of one Graph Machine sparse layer, as
+ * described in "Graph Machine: Towards Better Pretraining via Edges" (arXiv 2609.02881;
+ * ai.info summary, "Key Contributions" items 2-3 and "Methodology in Plain English"):
+ *
+ *   - sparse edge referral (SER): A' = Sparsify_s1(A1 A2), two-hop composition of each
+ *     position's edges, duplicate targets merged by summation, top-s1 kept;
+ *   - sparse edge attention (SEA): K/V gathered at each position's edge indices per KV head,
+ *     shared by the query heads of the GQA group, score = scale * q.k + ln w, softmax over
+ *     the entries, weighted sum of V;
+ *   - the SEA backward pass.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout. All tensors are dense, contiguous, row-major device arrays:
+ *   features  q, o, dout, dq  [B, n, hq,  d]
+ *             k, v, dk, dv    [B, n, hkv, d]
+ *   edges     idx (int32), w (fp32), dlogw (fp32)   [B, n, k, s]   (k edge channels)
+ *   lse       fp32 [B, n, hq]
+ * In SEA the edge channel h drives KV head h (k = hkv), and query head hq reads KV head
+ * hq / (hq_count / hkv) (contiguous GQA groups).
+ *
+ * Edge semantics. A slot (index, weight) is active iff weight > 0. Inactive slots are never
+ * dereferenced. An active slot whose index lies outside [0, n) is treated as inactive and
+ * raises the device error flag (see gm_check_device_errors); kernels never trap. Weights are
+ * expected finite and >= 0; indices are expected causal (<= the row's own position) but
+ * this is not checked. Position 0 of each sequence is the padding token: SER pads missing
+ * output slots with (index 0, weight 0.0f).
+ *
+ * Ownership and synchrony. The caller allocates and owns every buffer. Entry points allocate
+ * no device memory, enqueue their kernels on `stream` (0 = the legacy default stream) and
+ * return without synchronising; only gm_check_device_errors synchronises.
+ *
+ * Errors. Argument checks are synchronous and happen before any launch:
+ *   GM_ERR_INVALID_ARG  null pointer, negative size, hq % hkv != 0, non-finite scale,
+ *                       misaligned feature pointer (16 bytes required), s out of [1, 32];
+ *   GM_ERR_UNSUPPORTED  a valid shape this build has no kernel for (see each function);
+ *   GM_ERR_CUDA         the launch failed (cudaGetLastError after the launch);
+ *   GM_ERR_INDEX_RANGE  returned by gm_check_device_errors only.
+ * B == 0 or n == 0 is an empty problem: GM_OK, nothing launched.
+ */
+#ifndef GM_H
+#define GM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *cudaStream_t;
+
+typedef enum gm_status {
+    GM_OK = 0,
+    GM_ERR_INVALID_ARG = 1,
+    GM_ERR_UNSUPPORTED = 2,
+    GM_ERR_CUDA = 3,
+    GM_ERR_INDEX_RANGE = 4
+} gm_status;
+
+/* Element type of q, k, v, o and dout. */
+typedef enum gm_dtype {
+    GM_F32 = 0,
+    GM_BF16 = 1
+} gm_dtype;
+
+/*
+ * gm_ser_forward - sparse edge referral, A' = Sparsify_s1(A1 A2).
+ * Source: ai.info summary, "Key Contributions" item 3 (A' = Sparsify_s1(A1 A2), up to s2*s3
+ * candidates cut back to s1) and "Methodology in Plain English", referral paragraph (the
+ * first leg's indices fetch the second leg's indices and weights; hard top-s selection).
+ *
+ * For each (b, i, h): candidate c = a*s3 + e (a < s2, e < s3) is the path
+ * i -> j = a1_idx[b,i,h,a] -> t = a2_idx[b,j,h,e] with weight fl32(a1_w[..a] * a2_w[..e])
+ * (one fp32 rounding, no FMA). Zero-weight candidates are dropped; candidates that reach the
+ * same t are summed in fp32, in ascending c, each add rounded to nearest. The s1 heaviest
+ * targets are written to out_idx/out_w[b,i,h,0..s1) in order of weight descending, then
+ * index ascending; missing slots are (0, 0.0f). No renormalisation.
+ *
+ *   a1_idx, a1_w   device, [B, n, k, s2]        first leg
+ *   a2_idx, a2_w   device, [B, n, k, s3]        second leg (channel h reads channel h)
+ *   out_idx, out_w device, [B, n, k, s1]        written; must not alias the inputs
+ *   limits         1 <= s2*s3 <= 32, 1 <= s1 <= 32, k >= 1
+ * Result is deterministic and bit-identical to the plain definition above.
+ */
+gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                         const int32_t *a2_idx, const float *a2_w, int s3,
+                         int32_t *out_idx, float *out_w, int s1,
+                         int B, int n, int k, cudaStream_t stream);
+
+/*
+ * gm_sea_forward - sparse edge attention.
+ * Source: ai.info summary, "Key Contributions" item 3 (SEA: edge indices select the K/V
+ * positions; node factor = scaled q.k, edge factor = log edge weight, combined as a product
+ * of experts) and "Methodology in Plain English", SEA paragraph (no RoPE inside SEA).
+ *
+ * For each (b, i, hq) with h = hq / (hq_count / hkv), over the active slots j of
+ * idx/w[b,i,h,:]:  z_j = scale * <q[b,i,hq], k[b,t_j,h]> + ln w_j,  p = softmax(z),
+ * o[b,i,hq] = sum_j p_j v[b,t_j,h],  lse[b,i,hq] = ln sum_j exp(z_j).  A row with no active
+ * slot gives o = 0 and lse = -inf. Duplicate indices in a row count as separate slots.
+ * Arithmetic is fp32 (bf16 inputs widened); o is rounded to `dtype` (nearest even).
+ *
+ *   q, k, v   device, `dtype`, 16-byte aligned, layouts above
+ *   idx, w    device, [B, n, hkv, s], 1 <= s <= 32
+ *   o         device, `dtype`, [B, n, hq, d], written
+ *   lse       device fp32 [B, n, hq], written; may be NULL
+ *   scale     any finite float (1/sqrt(d) for the standard score)
+ *   limits    hq/hkv in {1, 2, 4, 8}; d in {32, 64, 128, 256} for GM_BF16 and
+ *             {32, 64, 128} for GM_F32 (else GM_ERR_UNSUPPORTED)
+ */
+gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype dtype,
+                         const int32_t *idx, const float *w, int s,
+                         int B, int n, int hq, int hkv, int d, float scale,
+                         void *o, float *lse, cudaStream_t stream);
+
+/*
+ * gm_ser_sea_forward - SER followed by SEA on its output, in one kernel.
+ * Same definitions as gm_ser_forward (with k = hkv) and gm_sea_forward (with s = s1, idx/w =
+ * the referral output). The refreshed edges stay in registers between the two steps; they
+ * are written to out_idx/out_w once, for the next layer, and never read back. out_idx and
+ * out_w may both be NULL when the caller does not need them.
+ * Results equal gm_ser_forward then gm_sea_forward bit for bit.
+ */
+gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                             const int32_t *a2_idx, const float *a2_w, int s3,
+                             int32_t *out_idx, float *out_w, int s1,
+                             const void *q, const void *k, const void *v, gm_dtype dtype,
+                             int B, int n, int hq, int hkv, int d, float scale,
+                             void *o, float *lse, cudaStream_t stream);
+
+/*
+ * gm_sea_backward - gradients of gm_sea_forward.
+ * Source: the derivative of the SEA definition above; ai.info summary, "Methodology in
+ * Plain English": indices get no gradient, the soft edge weights carry the learning signal.
+ *
+ * With p, z as in the forward (recomputed here from q, k, v, idx, w; no forward state is
+ * needed) and dp_j = <dout, v[t_j]>, dz_j = p_j (dp_j - sum_l p_l dp_l):
+ *   dq[b,i,hq]      = scale * sum_j dz_j k[b,t_j,h]
+ *   dk[b,t_j,h]    += scale * dz_j q[b,i,hq]          (scatter-add over all rows)
+ *   dv[b,t_j,h]    += p_j dout[b,i,hq]                (scatter-add over all rows)
+ *   dlogw[b,i,h,j]  = sum over the group's query heads of dz_j   (gradient w.r.t. ln w_j)
+ * Inactive slots get 0 in dlogw and contribute nothing. All arithmetic is fp32; the
+ * scatter-adds use fp32 atomics, so dk/dv summation order (not the set of terms) varies run
+ * to run.
+ *
+ *   q, k, v, dout       device, `dtype`, 16-byte aligned
+ *   idx, w              device, [B, n, hkv, s]
+ *   dq                  device fp32 [B, n, hq, d], 16-byte aligned
+ *   dk, dv              device fp32 [B, n, hkv, d], 16-byte aligned
+ *   dlogw               device fp32 [B, n, hkv, s]
+ *   accumulate          0: all four outputs are overwritten (dk/dv are zeroed first by a
+ *                       library kernel on `stream`); 1: results are added to their contents
+ *   limits              as gm_sea_forward
+ */
+gm_status gm_sea_backward(const void *q, const void *k, const void *v, const void *dout,
+                          gm_dtype dtype, const int32_t *idx, const float *w, int s,
+                          int B, int n, int hq, int hkv, int d, float scale,
+                          float *dq, float *dk, float *dv, float *dlogw,
+                          int accumulate, cudaStream_t stream);
+
+/*
+ * gm_check_device_errors - synchronise `stream`, then read and clear this device's error
+ * flag. Returns GM_ERR_INDEX_RANGE if any kernel of this library on the current device met
+ * an active slot whose index lay outside [0, n) since the last check, GM_ERR_CUDA if the
+ * synchronisation failed, else GM_OK.
+ */
+gm_status gm_check_device_errors(cudaStream_t stream);
+
+/* Static, human-readable name of a status code. Never NULL. */
+const char *gm_status_string(gm_status status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int gm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GM_H */

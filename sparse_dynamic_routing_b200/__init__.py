@@ -1,1 +1,25 @@
-"""Graph Machine sparse layer (SER + SEA) for B200 (sm_100a)."""
+"""Graph Machine sparse layer (SER + SEA) for NVIDIA B200 (sm_100a).
+
+The compute lives in the CUDA library libgm_b200.so (C ABI: include/gm.h); this package is
+its Python binding plus the seeded synthetic-input generators (`inputs`).
+
+    gm_ser_forward      sparse edge referral, A' = Sparsify_s1(A1 A2)
+    gm_sea_forward      sparse edge attention
+    gm_ser_sea_forward  both in one kernel
+    gm_sea_backward     gradients of sparse edge attention
+"""
+from ._binding import (  # noqa: F401
+    GM_BF16,
+    GM_F32,
+    GMError,
+    GMIndexRangeError,
+    LIB_PATH,
+    gm_check_device_errors,
+    gm_sea_backward,
+    gm_sea_forward,
+    gm_ser_forward,
+    gm_ser_sea_forward,
+    gm_version,
+    load_library,
+    status_string,
+)

@@ -1,0 +1,223 @@
+"""Python binding of the C ABI in include/gm.h (ctypes).
+
+Argument marshalling only: every step of SER, SEA and the SEA backward runs in the CUDA
+library libgm_b200.so. PyTorch supplies device memory (outputs are allocated with
+torch.empty when not given) and the stream (the current torch stream unless one is passed).
+There is no fallback: if the library is missing, or a tensor is not on a CUDA device, the
+call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgm_b200.so")
+
+GM_OK, GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED, GM_ERR_CUDA, GM_ERR_INDEX_RANGE = range(5)
+GM_F32, GM_BF16 = 0, 1
+
+# Entry points of include/gm.h with their ctypes signatures.
+_vp, _ci, _cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "gm_ser_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
+    "gm_sea_forward": [_vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp,
+                       _vp],
+    "gm_ser_sea_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _vp, _ci, _ci,
+                           _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp],
+    "gm_sea_backward": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf,
+                        _vp, _vp, _vp, _vp, _ci, _vp],
+    "gm_check_device_errors": [_vp],
+    "gm_status_string": [_ci],
+    "gm_version": [],
+}
+
+
+class GMError(RuntimeError):
+    """A library call returned a status other than GM_OK."""
+
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+class GMIndexRangeError(GMError):
+    """A kernel met an active edge slot whose index was outside [0, n)."""
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libgm_b200.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m sparse_dynamic_routing_b200.build`")
+        lib = ctypes.CDLL(path)
+        for name, args in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = ctypes.c_char_p if name == "gm_status_string" else ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load_library().gm_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != GM_OK:
+        cls = GMIndexRangeError if status == GM_ERR_INDEX_RANGE else GMError
+        raise cls(status, f"{what}: {status_string(status)}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _ptr(t: torch.Tensor | None, dtype=None, name="tensor") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _fdtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return GM_BF16
+    if t.dtype == torch.float32:
+        return GM_F32
+    raise ValueError(f"features must be bfloat16 or float32, got {t.dtype}")
+
+
+def _scale(scale, d):
+    return float(1.0 / math.sqrt(d)) if scale is None else float(scale)
+
+
+def gm_ser_forward(a1_idx, a1_w, a2_idx, a2_w, s1: int, out_idx=None, out_w=None, stream=None):
+    """Sparse edge referral A' = Sparsify_s1(A1 A2). Returns (out_idx, out_w) [B,n,k,s1]."""
+    B, n, k, s2 = a1_idx.shape
+    s3 = a2_idx.shape[3]
+    if a2_idx.shape[:3] != (B, n, k) or a1_w.shape != a1_idx.shape or a2_w.shape != a2_idx.shape:
+        raise ValueError("edge tensor shapes disagree")
+    dev = a1_idx.device
+    if out_idx is None:
+        out_idx = torch.empty((B, n, k, s1), dtype=torch.int32, device=dev)
+    if out_w is None:
+        out_w = torch.empty((B, n, k, s1), dtype=torch.float32, device=dev)
+    lib = load_library()
+    st = lib.gm_ser_forward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, torch.float32, "a1_w"), s2,
+        _ptr(a2_idx, torch.int32, "a2_idx"), _ptr(a2_w, torch.float32, "a2_w"), s3,
+        _ptr(out_idx, torch.int32, "out_idx"), _ptr(out_w, torch.float32, "out_w"), s1,
+        B, n, k, _stream(stream))
+    _check(st, "gm_ser_forward")
+    return out_idx, out_w
+
+
+def gm_sea_forward(q, k, v, idx, w, scale=None, o=None, lse=None, want_lse=True, stream=None):
+    """Sparse edge attention. Returns (o [B,n,hq,d] in q's dtype, lse fp32 [B,n,hq] or None)."""
+    B, n, hq, d = q.shape
+    hkv, s = idx.shape[2], idx.shape[3]
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape or w.shape != idx.shape:
+        raise ValueError("tensor shapes disagree")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share a dtype")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n, hq), dtype=torch.float32, device=q.device)
+    lib = load_library()
+    st = lib.gm_sea_forward(
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _fdtype(q),
+        _ptr(idx, torch.int32, "idx"), _ptr(w, torch.float32, "w"), s,
+        B, n, hq, hkv, d, _scale(scale, d), _ptr(o, q.dtype, "o"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(st, "gm_sea_forward")
+    return o, lse
+
+
+def gm_ser_sea_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, s1: int, scale=None,
+                       out_idx=None, out_w=None, o=None, lse=None, want_edges=True,
+                       want_lse=True, stream=None):
+    """Fused SER -> SEA forward. Returns (out_idx, out_w, o, lse); edges/lse None if not wanted."""
+    B, n, hq, d = q.shape
+    hkv = k.shape[2]
+    s2, s3 = a1_idx.shape[3], a2_idx.shape[3]
+    if a1_idx.shape[:3] != (B, n, hkv) or a2_idx.shape[:3] != (B, n, hkv):
+        raise ValueError("edge tensors must be [B, n, hkv, s]")
+    if a1_w.shape != a1_idx.shape or a2_w.shape != a2_idx.shape:
+        raise ValueError("edge weight shapes disagree with their indices")
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape:
+        raise ValueError("k/v shapes disagree with q")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share a dtype")
+    dev = q.device
+    if want_edges:
+        if out_idx is None:
+            out_idx = torch.empty((B, n, hkv, s1), dtype=torch.int32, device=dev)
+        if out_w is None:
+            out_w = torch.empty((B, n, hkv, s1), dtype=torch.float32, device=dev)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, n, hq), dtype=torch.float32, device=dev)
+    lib = load_library()
+    st = lib.gm_ser_sea_forward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, torch.float32, "a1_w"), s2,
+        _ptr(a2_idx, torch.int32, "a2_idx"), _ptr(a2_w, torch.float32, "a2_w"), s3,
+        _ptr(out_idx, torch.int32, "out_idx"), _ptr(out_w, torch.float32, "out_w"), s1,
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _fdtype(q),
+        B, n, hq, hkv, d, _scale(scale, d), _ptr(o, q.dtype, "o"),
+        _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(st, "gm_ser_sea_forward")
+    return out_idx, out_w, o, lse
+
+
+def gm_sea_backward(q, k, v, dout, idx, w, scale=None, dq=None, dk=None, dv=None, dlogw=None,
+                    accumulate=False, stream=None):
+    """SEA backward. Returns (dq, dk, dv, dlogw), all fp32."""
+    B, n, hq, d = q.shape
+    hkv, s = idx.shape[2], idx.shape[3]
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape or w.shape != idx.shape:
+        raise ValueError("tensor shapes disagree")
+    if dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError("dout must match q")
+    dev = q.device
+    f32 = torch.float32
+    dq = torch.empty((B, n, hq, d), dtype=f32, device=dev) if dq is None else dq
+    dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dk is None else dk
+    dv = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dv is None else dv
+    dlogw = torch.empty((B, n, hkv, s), dtype=f32, device=dev) if dlogw is None else dlogw
+    lib = load_library()
+    st = lib.gm_sea_backward(
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _ptr(dout, name="dout"),
+        _fdtype(q), _ptr(idx, torch.int32, "idx"), _ptr(w, f32, "w"), s,
+        B, n, hq, hkv, d, _scale(scale, d), _ptr(dq, f32, "dq"), _ptr(dk, f32, "dk"),
+        _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_sea_backward")
+    return dq, dk, dv, dlogw
+
+
+def gm_check_device_errors(stream=None):
+    """Synchronise the stream and raise GMIndexRangeError if a kernel met a bad index."""
+    _check(load_library().gm_check_device_errors(_stream(stream)), "gm_check_device_errors")
+
+
+def gm_version() -> int:
+    return int(load_library().gm_version())

@@ -1,0 +1,216 @@
+// gm_api.cu - host side of the C ABI declared in include/gm.h: argument checks, dispatch to
+// the kernel instantiation for (dtype, head_dim, GQA group), launch on the caller's stream.
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/gm.h"
+#include "gm_common.cuh"
+#include "gm_sea.cuh"
+#include "gm_sea_bwd.cuh"
+#include "gm_ser.cuh"
+
+namespace {
+
+using gm::SeaArgs;
+using gm::SeaBwdArgs;
+using gm::SerArgs;
+
+constexpr int WPB_SER = 8;   // warps (edge rows) per block
+constexpr int WPB_SEA = 8;
+constexpr int WPB_BWD = 8;
+constexpr int MAX_SLOTS = 32;
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline gm_status launched()
+{
+    return cudaGetLastError() == cudaSuccess ? GM_OK : GM_ERR_CUDA;
+}
+
+inline unsigned blocks_for(int64_t rows, int wpb) { return (unsigned)((rows + wpb - 1) / wpb); }
+
+gm_status check_ser(const int32_t *a1_idx, const float *a1_w, int s2, const int32_t *a2_idx,
+                    const float *a2_w, int s3, int s1, int B, int n, int k)
+{
+    if (B < 0 || n < 0 || k < 1) return GM_ERR_INVALID_ARG;
+    if (s1 < 1 || s2 < 1 || s3 < 1 || s1 > MAX_SLOTS || s2 * s3 > MAX_SLOTS) return GM_ERR_INVALID_ARG;
+    if ((int64_t)B * n == 0) return GM_OK;
+    if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
+    return GM_OK;
+}
+
+// Shapes shared by SEA forward and backward. Returns GM_OK, or the error to report.
+gm_status check_sea(const void *q, const void *k, const void *v, gm_dtype dtype,
+                    const int32_t *idx, const float *w, int s, int B, int n, int hq, int hkv,
+                    int d, float scale)
+{
+    if (B < 0 || n < 0 || hq < 1 || hkv < 1 || d < 1) return GM_ERR_INVALID_ARG;
+    if (hq % hkv != 0 || s < 1 || s > MAX_SLOTS || !std::isfinite(scale)) return GM_ERR_INVALID_ARG;
+    if (dtype != GM_F32 && dtype != GM_BF16) return GM_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return GM_ERR_UNSUPPORTED;
+    if (d != 32 && d != 64 && d != 128 && d != 256) return GM_ERR_UNSUPPORTED;
+    if (dtype == GM_F32 && d > 128) return GM_ERR_UNSUPPORTED;
+    if ((int64_t)B * n == 0) return GM_OK;
+    if (!q || !k || !v || !idx || !w) return GM_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GM_ERR_INVALID_ARG;
+    return GM_OK;
+}
+
+// ---- dispatch over (dtype, d, G) ----------------------------------------------------------
+
+template <template <typename, int, int> class F, typename... Args>
+gm_status dispatch(gm_dtype dtype, int d, int G, Args &&...args)
+{
+#define GM_CASE_G(T, D)                                               \
+    switch (G) {                                                      \
+    case 1: return F<T, D, 1>::run(args...);                          \
+    case 2: return F<T, D, 2>::run(args...);                          \
+    case 4: return F<T, D, 4>::run(args...);                          \
+    case 8: return F<T, D, 8>::run(args...);                          \
+    default: return GM_ERR_UNSUPPORTED;                               \
+    }
+    if (dtype == GM_BF16) {
+        switch (d) {
+        case 32: GM_CASE_G(__nv_bfloat16, 32)
+        case 64: GM_CASE_G(__nv_bfloat16, 64)
+        case 128: GM_CASE_G(__nv_bfloat16, 128)
+        case 256: GM_CASE_G(__nv_bfloat16, 256)
+        default: return GM_ERR_UNSUPPORTED;
+        }
+    } else {
+        switch (d) {
+        case 32: GM_CASE_G(float, 32)
+        case 64: GM_CASE_G(float, 64)
+        case 128: GM_CASE_G(float, 128)
+        default: return GM_ERR_UNSUPPORTED;
+        }
+    }
+#undef GM_CASE_G
+}
+
+template <typename T, int D, int G> struct SeaFwd {
+    static gm_status run(const SeaArgs &a, cudaStream_t st)
+    {
+        gm::sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(a);
+        return launched();
+    }
+};
+
+template <typename T, int D, int G> struct SerSeaFwd {
+    static gm_status run(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
+    {
+        gm::ser_sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(sa, a);
+        return launched();
+    }
+};
+
+template <typename T, int D, int G> struct SeaBwd {
+    static gm_status run(const SeaBwdArgs &a, cudaStream_t st)
+    {
+        gm::sea_bwd_kernel<T, D, G, WPB_BWD><<<blocks_for(a.rows, WPB_BWD), WPB_BWD * 32, 0, st>>>(a);
+        return launched();
+    }
+};
+
+}  // namespace
+
+extern "C" {
+
+int gm_version(void) { return 100; }
+
+const char *gm_status_string(gm_status status)
+{
+    switch (status) {
+    case GM_OK: return "GM_OK";
+    case GM_ERR_INVALID_ARG: return "GM_ERR_INVALID_ARG: invalid argument";
+    case GM_ERR_UNSUPPORTED: return "GM_ERR_UNSUPPORTED: shape not supported by this build";
+    case GM_ERR_CUDA: return "GM_ERR_CUDA: CUDA launch or synchronisation failed";
+    case GM_ERR_INDEX_RANGE: return "GM_ERR_INDEX_RANGE: an active edge index was outside [0, n)";
+    default: return "unknown gm_status";
+    }
+}
+
+gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                         const int32_t *a2_idx, const float *a2_w, int s3,
+                         int32_t *out_idx, float *out_w, int s1,
+                         int B, int n, int k, cudaStream_t stream)
+{
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, k);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
+    SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k, (int64_t)B * n * k};
+    gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
+    return launched();
+}
+
+gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype dtype,
+                         const int32_t *idx, const float *w, int s,
+                         int B, int n, int hq, int hkv, int d, float scale,
+                         void *o, float *lse, cudaStream_t stream)
+{
+    gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    SeaArgs a{q, k, v, idx, w, o, lse, s, n, hkv, scale, (int64_t)B * n * hkv};
+    return dispatch<SeaFwd>(dtype, d, hq / hkv, a, stream);
+}
+
+gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                             const int32_t *a2_idx, const float *a2_w, int s3,
+                             int32_t *out_idx, float *out_w, int s1,
+                             const void *q, const void *k, const void *v, gm_dtype dtype,
+                             int B, int n, int hq, int hkv, int d, float scale,
+                             void *o, float *lse, cudaStream_t stream)
+{
+    if ((out_idx == nullptr) != (out_w == nullptr)) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, hkv);
+    if (st != GM_OK) return st;
+    // the referral output is the attention's edge set: validate SEA with a stand-in pointer
+    const int32_t dummy_idx = 0;
+    const float dummy_w = 0.0f;
+    st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * n * hkv;
+    SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows};
+    SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows};
+    return dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
+}
+
+gm_status gm_sea_backward(const void *q, const void *k, const void *v, const void *dout,
+                          gm_dtype dtype, const int32_t *idx, const float *w, int s,
+                          int B, int n, int hq, int hkv, int d, float scale,
+                          float *dq, float *dk, float *dv, float *dlogw,
+                          int accumulate, cudaStream_t stream)
+{
+    if (accumulate != 0 && accumulate != 1) return GM_ERR_INVALID_ARG;
+    gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!dout || !dq || !dk || !dv || !dlogw) return GM_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * n * hkv;
+    if (!accumulate) {
+        const int64_t count4 = rows * d / 4;
+        const int64_t want = (count4 + 255) / 256;
+        const unsigned grid = (unsigned)(want < 148 * 16 ? want : 148 * 16);
+        gm::zero2_kernel<<<grid, 256, 0, stream>>>(reinterpret_cast<float4 *>(dk),
+                                                    reinterpret_cast<float4 *>(dv), count4);
+        if (launched() != GM_OK) return GM_ERR_CUDA;
+    }
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, s, n, hkv, scale, accumulate, rows};
+    return dispatch<SeaBwd>(dtype, d, hq / hkv, a, stream);
+}
+
+gm_status gm_check_device_errors(cudaStream_t stream)
+{
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return GM_ERR_CUDA;
+    unsigned flag = 0;
+    if (cudaMemcpyFromSymbol(&flag, gm::g_error_flag, sizeof(flag)) != cudaSuccess) return GM_ERR_CUDA;
+    if (flag == 0) return GM_OK;
+    const unsigned zero = 0;
+    if (cudaMemcpyToSymbol(gm::g_error_flag, &zero, sizeof(zero)) != cudaSuccess) return GM_ERR_CUDA;
+    return GM_ERR_INDEX_RANGE;
+}
+
+}  // extern "C"

@@ -1,0 +1,120 @@
+"""The C ABI without a GPU: the library builds, loads, exports every symbol include/gm.h
+declares, and rejects bad arguments on the host before any CUDA call.
+
+Only argument combinations that fail validation are passed here, so no kernel is ever
+launched (and no pointer below is ever dereferenced).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_dynamic_routing_b200 import _binding as bnd
+from sparse_dynamic_routing_b200 import build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "gm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return bnd.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"gm_ser_forward", "gm_sea_forward", "gm_ser_sea_forward", "gm_sea_backward",
+            "gm_check_device_errors"} <= set(names)
+    for name in names:
+        assert hasattr(lib, name), name
+        assert name in bnd.SIGNATURES, f"{name} has no binding"
+
+
+def test_status_strings(lib):
+    for st in range(5):
+        assert bnd.status_string(st).startswith("GM_")
+    assert "unknown" in bnd.status_string(99)
+    assert lib.gm_version() >= 100
+
+
+NULL = None
+FAKE = 0x1000  # never dereferenced: every call below fails validation first
+
+
+def test_ser_argument_checks(lib):
+    f = lib.gm_ser_forward
+    ok_empty = f(NULL, NULL, 2, NULL, NULL, 2, NULL, NULL, 2, 0, 128, 1, NULL)
+    assert ok_empty == bnd.GM_OK  # B = 0: nothing to do
+    assert f(NULL, NULL, 2, NULL, NULL, 2, NULL, NULL, 2, 4, 0, 1, NULL) == bnd.GM_OK  # n = 0
+    assert f(NULL, NULL, 2, NULL, NULL, 2, NULL, NULL, 2, 1, 8, 1, NULL) == bnd.GM_ERR_INVALID_ARG
+    bad = [
+        dict(s2=8, s3=5),  # 40 candidates > 32
+        dict(s1=33),
+        dict(s1=0),
+        dict(k=0),
+        dict(B=-1),
+    ]
+    for b in bad:
+        a = dict(s2=2, s3=2, s1=2, B=1, n=8, k=1)
+        a.update(b)
+        st = f(FAKE, FAKE, a["s2"], FAKE, FAKE, a["s3"], FAKE, FAKE, a["s1"], a["B"], a["n"],
+               a["k"], NULL)
+        assert st == bnd.GM_ERR_INVALID_ARG, b
+    # null outputs
+    assert f(FAKE, FAKE, 2, FAKE, FAKE, 2, NULL, FAKE, 2, 1, 8, 1, NULL) == bnd.GM_ERR_INVALID_ARG
+
+
+def sea_call(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, dt=bnd.GM_BF16, idx=FAKE, w=FAKE, s=4, B=1, n=8, hq=4,
+             hkv=2, d=128, scale=0.1, o=FAKE + 1, lse=NULL)  # o misaligned: never launches
+    a.update(kw)
+    return lib.gm_sea_forward(a["q"], a["k"], a["v"], a["dt"], a["idx"], a["w"], a["s"], a["B"],
+                              a["n"], a["hq"], a["hkv"], a["d"], a["scale"], a["o"], a["lse"],
+                              NULL)
+
+
+def test_sea_argument_checks(lib):
+    assert sea_call(lib) == bnd.GM_ERR_INVALID_ARG  # misaligned o
+    assert sea_call(lib, B=0) == bnd.GM_OK
+    assert sea_call(lib, hq=3) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, s=0) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, s=33) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, scale=float("nan")) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, scale=float("inf")) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, dt=7) == bnd.GM_ERR_INVALID_ARG
+    assert sea_call(lib, d=96) == bnd.GM_ERR_UNSUPPORTED
+    assert sea_call(lib, dt=bnd.GM_F32, d=256) == bnd.GM_ERR_UNSUPPORTED
+    assert sea_call(lib, hq=32, hkv=2) == bnd.GM_ERR_UNSUPPORTED  # group of 16
+    assert sea_call(lib, q=FAKE + 8) == bnd.GM_ERR_INVALID_ARG  # misaligned q
+    assert sea_call(lib, k=NULL) == bnd.GM_ERR_INVALID_ARG
+
+
+def test_backward_and_fused_argument_checks(lib):
+    f = lib.gm_sea_backward
+    # dout misaligned in every case: a call that got past the checks under test would still
+    # be rejected before its launch
+    base = [FAKE, FAKE, FAKE, FAKE + 2, bnd.GM_BF16, FAKE, FAKE, 4, 1, 8, 4, 2, 128, 0.1,
+            FAKE, FAKE, FAKE, FAKE, 0, NULL]
+    a = list(base)
+    a[18] = 2  # accumulate must be 0 or 1
+    assert f(*a) == bnd.GM_ERR_INVALID_ARG
+    a = list(base)
+    a[14] = FAKE + 4  # misaligned dq
+    assert f(*a) == bnd.GM_ERR_INVALID_ARG
+    a = list(base)
+    a[17] = NULL  # no dlogw
+    assert f(*a) == bnd.GM_ERR_INVALID_ARG
+    g = lib.gm_ser_sea_forward
+    fb = [FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, NULL, 4, FAKE, FAKE, FAKE, bnd.GM_BF16, 1, 8, 4,
+          2, 128, 0.1, FAKE + 1, NULL, NULL]  # o misaligned: never launches
+    assert g(*fb) == bnd.GM_ERR_INVALID_ARG  # out_idx given without out_w
+    fb2 = list(fb)
+    fb2[2], fb2[5] = 8, 8  # 64 candidates
+    assert g(*fb2) == bnd.GM_ERR_INVALID_ARG
