@@ -27,9 +27,7 @@ import argparse
 import datetime
 import hashlib
 import json
-import math
 import os
-import re
 import statistics
 import sys
 import threading
@@ -55,6 +53,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(I.WORKLOADS))
+    p.add_argument("--batch", type=int, default=None,
+                   help="override the workload's batch size (small cases for profiling)")
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -295,7 +295,10 @@ def run_ours(args):
     import sparse_dynamic_routing_b200 as gm
     gm.load_library()
 
-    wl = shard_seed(I.WORKLOADS[args.workload], rank)
+    wl = I.WORKLOADS[args.workload]
+    if args.batch is not None:
+        wl = wl.with_(B=args.batch)
+    wl = shard_seed(wl, rank)
     assert wl.kind == "ser_sea", "the bench step is SER->SEA forward + SEA backward"
     x = I.make(wl, grad=True)
     g = {k: v.to(dev) for k, v in x.items()}

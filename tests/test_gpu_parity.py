@@ -45,7 +45,8 @@ def assert_ser_equal(gi, gw, oi, ow):
 def assert_close(got, want, tol, what):
     got = host(got).double().numpy().reshape(want.shape)
     both_inf = np.isneginf(got) & np.isneginf(want)
-    diff = np.where(both_inf, 0.0, np.abs(got - want))
+    with np.errstate(invalid="ignore"):
+        diff = np.where(both_inf, 0.0, np.abs(got - want))
     err = float(np.nanmax(diff)) if diff.size else 0.0
     assert not np.isnan(diff).any(), f"{what}: NaN"
     assert err <= tol, f"{what}: max-abs error {err:.3g} > {tol}"
