@@ -16,9 +16,10 @@ using gm::SeaBwdArgs;
 using gm::SerArgs;
 
 constexpr int WPB_SER = 8;   // warps (edge rows) per block
-constexpr int WPB_SEA = 8;
-constexpr int WPB_BWD = 8;
+constexpr int WPB_SEA = GM_WPB_SEA;
+constexpr int WPB_BWD = GM_WPB_BWD;
 constexpr int MAX_SLOTS = 32;
+constexpr int64_t MAX_ROWS = (int64_t)1 << 31;  // edge rows B*n*heads indexed in 32 bits
 
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -29,12 +30,18 @@ inline gm_status launched()
 
 inline unsigned blocks_for(int64_t rows, int wpb) { return (unsigned)((rows + wpb - 1) / wpb); }
 
+inline gm::RowMap row_map(int heads, int n)
+{
+    return gm::RowMap{gm::FastDiv((uint32_t)heads), gm::FastDiv((uint32_t)n)};
+}
+
 gm_status check_ser(const int32_t *a1_idx, const float *a1_w, int s2, const int32_t *a2_idx,
                     const float *a2_w, int s3, int s1, int B, int n, int k)
 {
     if (B < 0 || n < 0 || k < 1) return GM_ERR_INVALID_ARG;
     if (s1 < 1 || s2 < 1 || s3 < 1 || s1 > MAX_SLOTS || s2 * s3 > MAX_SLOTS) return GM_ERR_INVALID_ARG;
     if ((int64_t)B * n == 0) return GM_OK;
+    if ((int64_t)B * n * k >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
     if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
     return GM_OK;
 }
@@ -52,6 +59,7 @@ gm_status check_sea(const void *q, const void *k, const void *v, gm_dtype dtype,
     if (d != 32 && d != 64 && d != 128 && d != 256) return GM_ERR_UNSUPPORTED;
     if (dtype == GM_F32 && d > 128) return GM_ERR_UNSUPPORTED;
     if ((int64_t)B * n == 0) return GM_OK;
+    if ((int64_t)B * n * hkv >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
     if (!q || !k || !v || !idx || !w) return GM_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return GM_ERR_INVALID_ARG;
     return GM_OK;
@@ -139,7 +147,8 @@ gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, k);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
-    SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k, (int64_t)B * n * k};
+    SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k,
+              (uint32_t)((int64_t)B * n * k), row_map(k, n)};
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
     return launched();
 }
@@ -152,7 +161,8 @@ gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype d
     gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
-    SeaArgs a{q, k, v, idx, w, o, lse, s, n, hkv, scale, (int64_t)B * n * hkv};
+    SeaArgs a{q, k, v, idx, w, o, lse, s, n, hkv, scale, (uint32_t)((int64_t)B * n * hkv),
+              row_map(hkv, n)};
     return dispatch<SeaFwd>(dtype, d, hq / hkv, a, stream);
 }
 
@@ -172,9 +182,9 @@ gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
-    const int64_t rows = (int64_t)B * n * hkv;
-    SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows};
-    SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows};
+    const uint32_t rows = (uint32_t)((int64_t)B * n * hkv);
+    SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows, row_map(hkv, n)};
+    SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows, row_map(hkv, n)};
     return dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
 }
 
@@ -198,7 +208,8 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
                                                     reinterpret_cast<float4 *>(dv), count4);
         if (launched() != GM_OK) return GM_ERR_CUDA;
     }
-    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, s, n, hkv, scale, accumulate, rows};
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, s, n, hkv, scale, accumulate,
+                 (uint32_t)rows, row_map(hkv, n)};
     return dispatch<SeaBwd>(dtype, d, hq / hkv, a, stream);
 }
 

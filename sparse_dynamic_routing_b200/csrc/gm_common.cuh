@@ -12,6 +12,21 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+// Launch shape: warps (edge rows) per block and minimum resident blocks per SM of the
+// attention kernels (the latter caps registers per thread at 65536 / (32 * WPB * MINB)).
+#ifndef GM_WPB_SEA
+#define GM_WPB_SEA 4
+#endif
+#ifndef GM_WPB_BWD
+#define GM_WPB_BWD 4
+#endif
+#ifndef GM_FWD_MINB
+#define GM_FWD_MINB 8
+#endif
+#ifndef GM_BWD_MINB
+#define GM_BWD_MINB 6
+#endif
+
 namespace gm {
 
 constexpr unsigned FULL = 0xffffffffu;
@@ -25,7 +40,61 @@ constexpr unsigned ERR_INDEX_RANGE = 1u;
 
 __device__ __forceinline__ void raise_index_error() { atomicOr(&g_error_flag, ERR_INDEX_RANGE); }
 
+// ---- integer division by a launch-invariant divisor ---------------------------------------
+//
+// Row decomposition (row -> b, i, h) divides by n and by the head count on every warp; a
+// hardware integer divide is a long instruction sequence, so the host precomputes a
+// multiplier and shift (Granlund & Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, section 4) and the device divides with one multiply-high,
+// a subtract, an add and two shifts. Exact for every 32-bit unsigned dividend.
+struct FastDiv {
+    uint32_t d;      // divisor (>= 1)
+    uint32_t mul;    // magic multiplier
+    uint32_t s1, s2; // shifts
+
+    FastDiv() = default;
+    __host__ explicit FastDiv(uint32_t divisor) : d(divisor)
+    {
+        uint32_t l = 0;
+        while (l < 32 && (uint64_t(1) << l) < divisor) ++l;  // l = ceil(log2 d)
+        // mul = floor(2^32 * (2^l - d) / d) + 1
+        mul = (uint32_t)(((uint64_t(1) << 32) * ((uint64_t(1) << l) - divisor)) / divisor + 1);
+        s1 = l > 0 ? 1 : 0;
+        s2 = l > 0 ? l - 1 : 0;
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t x) const
+    {
+        const uint32_t t = __umulhi(x, mul);
+        return (t + ((x - t) >> s1)) >> s2;
+    }
+};
+
+// Edge row -> (sequence start b*n, head h), for row = (b*n + i)*heads + h < 2^31.
+struct RowMap {
+    FastDiv heads, n;
+    __device__ __forceinline__ void split(uint32_t row, uint32_t &seq_base, uint32_t &h) const
+    {
+        const uint32_t bi = heads.div(row);
+        h = row - bi * heads.d;
+        seq_base = n.div(bi) * n.d;  // b * n
+    }
+};
+
 // ---- 16-byte chunks of feature rows -------------------------------------------------------
+
+// Fast base-2 exponential / logarithm (MUFU; relative error ~2^-22, subnormals kept).
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float lg2(float x)
+{
+    float y;
+    asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 template <typename T> struct Vec;
 template <> struct Vec<float> { static constexpr int N = 4; };

@@ -9,11 +9,16 @@
 // e_j = exp(z_j - m), l = sum e_j and dp_j = <dO, V[t_j]>:
 //   D   = sum_j p_j dp_j                    = (sum_j e_j dp_j) / l
 //   dq  = scale * sum_j p_j (dp_j - D) K_j  = scale / l * (sum_j e_j dp_j K_j - D sum_j e_j K_j)
-// so one streaming pass over the slots (pass A, online max as in the forward) yields dq; the
-// per-slot scores z_j and dp_j go to shared memory, and pass B turns them into
-// dz_j = p_j (dp_j - D) for the scatter-adds dK[t_j] += scale dz_j q and dV[t_j] += p_j dO
-// (16-byte vector fp32 atomics, summed over the query-head group first) and for
-// dlogw_j = sum over the group of dz_j.
+// so one streaming pass over the slots (pass A, batches of four with an online max as in
+// the forward) yields dq; the per-slot scores z_j and dp_j go to shared memory, and pass B
+// turns them into dz_j = p_j (dp_j - D) for the scatter-adds dK[t_j] += scale dz_j q and
+// dV[t_j] += p_j dO (16-byte vector fp32 atomics, summed over the query-head group first)
+// and for dlogw_j = sum over the group of dz_j.
+//
+// When the group's rows exactly fill the warp in two segments (G = 2, C = 16: bf16
+// head_dim 128), the segments split the scatter: segment 0 adds dK, segment 1 adds dV, and
+// each fetches the other segment's q (resp. dO) chunk once per row, so a slot costs two
+// shuffles instead of a cross-segment reduction of every element.
 #pragma once
 
 #include "gm_common.cuh"
@@ -28,7 +33,8 @@ struct SeaBwdArgs {
     int s, n, hkv;
     float scale;
     int accumulate;
-    int64_t rows;  // B * n * hkv
+    uint32_t rows;  // B * n * hkv
+    RowMap map;     // heads = hkv
 };
 
 __device__ __forceinline__ void red_add4(float *p, float a, float b, float c, float d)
@@ -37,45 +43,50 @@ __device__ __forceinline__ void red_add4(float *p, float a, float b, float c, fl
 }
 
 template <typename T, int D, int G, int WPB>
-__global__ void __launch_bounds__(WPB * 32) sea_bwd_kernel(SeaBwdArgs a)
+__global__ void __launch_bounds__(WPB * 32, GM_BWD_MINB) sea_bwd_kernel(SeaBwdArgs a)
 {
     using Gm = Geom<T, D, G>;
     constexpr int VEC = Gm::VEC, NI = Gm::NI, C = Gm::C, RPI = Gm::RPI;
+    constexpr bool PAIR = (G == 2 && RPI == 2 && NI == 1);  // the two-segment split
     __shared__ float sh_z[WPB][G][32];
     __shared__ float sh_dp[WPB][G][32];
 
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int64_t row = (int64_t)blockIdx.x * WPB + wid;
+    const uint32_t row = blockIdx.x * WPB + wid;
     if (row >= a.rows) return;  // warp-uniform
     const int c = lane % C, seg = lane / C;
-    const int h = (int)(row % a.hkv);
-    const int64_t seq_base = (row / a.hkv) / a.n * a.n;
     const T *Q = static_cast<const T *>(a.q);
     const T *K = static_cast<const T *>(a.k);
     const T *V = static_cast<const T *>(a.v);
     const T *GO = static_cast<const T *>(a.dout);
     const float sl2 = a.scale * LOG2E;
 
-    float qf[NI][VEC], gf[NI][VEC];
+    uint4 qr[NI], gr[NI];
 #pragma unroll
     for (int it = 0; it < NI; ++it) {
         const int g = it * RPI + seg;
-        uint4 qr = make_uint4(0, 0, 0, 0), gr = make_uint4(0, 0, 0, 0);
+        qr[it] = gr[it] = make_uint4(0, 0, 0, 0);
         if (g < G) {
-            qr = ld16_stream(Q + (row * G + g) * D + c * VEC);
-            gr = ld16_stream(GO + (row * G + g) * D + c * VEC);
+            qr[it] = ld16_stream(Q + ((size_t)row * G + g) * D + c * VEC);
+            gr[it] = ld16_stream(GO + ((size_t)row * G + g) * D + c * VEC);
         }
-        unpack<T>(qr, qf[it]);
-        unpack<T>(gr, gf[it]);
     }
     int32_t t_l = 0;
     float w_l = 0.0f;
     if (lane < a.s) {
-        t_l = __ldg(a.idx + row * a.s + lane);
-        w_l = __ldg(a.w + row * a.s + lane);
+        t_l = __ldg(a.idx + (size_t)row * a.s + lane);
+        w_l = __ldg(a.w + (size_t)row * a.s + lane);
+    }
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    float qf[NI][VEC], gf[NI][VEC];
+#pragma unroll
+    for (int it = 0; it < NI; ++it) {
+        unpack<T>(qr[it], qf[it]);
+        unpack<T>(gr[it], gf[it]);
     }
 
-    // ---- pass A: scores, online softmax statistics and the two dq accumulators ----------
+    // ---- pass A: scores, softmax statistics and the two dq accumulators ------------------
     float m[NI], l[NI], sdp[NI], Ak[NI][VEC], Bk[NI][VEC];
 #pragma unroll
     for (int it = 0; it < NI; ++it) {
@@ -89,6 +100,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_kernel(SeaBwdArgs a)
         bool on[4];
         float lw2[4];
         uint4 kr[4], vr[4];
+        bool any = false;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
             const int j = j0 + jj;
@@ -99,48 +111,76 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_kernel(SeaBwdArgs a)
                 if (lane == 0) raise_index_error();
                 on[jj] = false;
             }
-            lw2[jj] = on[jj] ? log2f(w) : 0.0f;
+            lw2[jj] = lg2(w);
             kr[jj] = vr[jj] = make_uint4(0, 0, 0, 0);
             if (on[jj]) {
-                const int64_t off = ((seq_base + t) * a.hkv + h) * D + c * VEC;
+                const size_t off = ((size_t)(seq_base + (uint32_t)t) * a.hkv + h) * D + c * VEC;
                 kr[jj] = ld16(K + off);
                 vr[jj] = ld16(V + off);
                 active |= 1u << j;
             }
+            any |= on[jj];
         }
+        if (!any) continue;  // warp-uniform
+
+        float z[NI][4], dp[NI][4];
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            if (!on[jj]) continue;  // warp-uniform
             float kf[VEC], vf[VEC];
             unpack<T>(kr[jj], kf);
             unpack<T>(vr[jj], vf);
 #pragma unroll
             for (int it = 0; it < NI; ++it) {
-                float dk = 0.0f, dv = 0.0f;
+                float sk = 0.0f, sv = 0.0f;
 #pragma unroll
                 for (int x = 0; x < VEC; ++x) {
-                    dk = fmaf(qf[it][x], kf[x], dk);
-                    dv = fmaf(gf[it][x], vf[x], dv);
+                    sk = fmaf(qf[it][x], kf[x], sk);
+                    sv = fmaf(gf[it][x], vf[x], sv);
                 }
-                const float z = seg_sum<C>(dk) * sl2 + lw2[jj];
-                const float dp = seg_sum<C>(dv);
-                const int g = it * RPI + seg;
-                if (c == 0 && g < G) {
-                    sh_z[wid][g][j0 + jj] = z;
-                    sh_dp[wid][g][j0 + jj] = dp;
+                z[it][jj] = -INFINITY;
+                dp[it][jj] = 0.0f;
+                if (on[jj]) {  // warp-uniform
+                    z[it][jj] = fmaf(seg_sum<C>(sk), sl2, lw2[jj]);
+                    dp[it][jj] = seg_sum<C>(sv);
+                    const int g = it * RPI + seg;
+                    if (c == 0 && g < G) {
+                        sh_z[wid][g][j0 + jj] = z[it][jj];
+                        sh_dp[wid][g][j0 + jj] = dp[it][jj];
+                    }
                 }
-                const float mn = fmaxf(m[it], z);
-                const float alpha = exp2f(m[it] - mn);
-                const float e = exp2f(z - mn);
-                l[it] = l[it] * alpha + e;
-                sdp[it] = sdp[it] * alpha + e * dp;
-                const float edp = e * dp;
+            }
+        }
+#pragma unroll
+        for (int it = 0; it < NI; ++it) {
+            float mb = z[it][0];
+#pragma unroll
+            for (int jj = 1; jj < 4; ++jj) mb = fmaxf(mb, z[it][jj]);
+            const float mn = fmaxf(m[it], mb);
+            if (j0 > 0) {
+                const float alpha = ex2(m[it] - mn);
+                l[it] *= alpha;
+                sdp[it] *= alpha;
 #pragma unroll
                 for (int x = 0; x < VEC; ++x) {
-                    Ak[it][x] = fmaf(edp, kf[x], Ak[it][x] * alpha);
-                    Bk[it][x] = fmaf(e, kf[x], Bk[it][x] * alpha);
+                    Ak[it][x] *= alpha;
+                    Bk[it][x] *= alpha;
                 }
-                m[it] = mn;
+            }
+            m[it] = mn;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                if (!on[jj]) continue;  // warp-uniform
+                float kf[VEC];
+                unpack<T>(kr[jj], kf);
+                const float e = ex2(z[it][jj] - mn);
+                const float edp = e * dp[it][jj];
+                l[it] += e;
+                sdp[it] += edp;
+#pragma unroll
+                for (int x = 0; x < VEC; ++x) {
+                    Ak[it][x] = fmaf(edp, kf[x], Ak[it][x]);
+                    Bk[it][x] = fmaf(e, kf[x], Bk[it][x]);
+                }
             }
         }
     }
@@ -150,18 +190,18 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_kernel(SeaBwdArgs a)
 #pragma unroll
     for (int it = 0; it < NI; ++it) {
         const int g = it * RPI + seg;
-        inv[it] = l[it] > 0.0f ? 1.0f / l[it] : 0.0f;
+        inv[it] = l[it] > 0.0f ? __frcp_rn(l[it]) : 0.0f;
         Dd[it] = sdp[it] * inv[it];
         if (g >= G) continue;
-        float *dqp = a.dq + (row * G + g) * D + c * VEC;
+        float *dqp = a.dq + ((size_t)row * G + g) * D + c * VEC;
         const float f = a.scale * inv[it];
 #pragma unroll
         for (int x = 0; x < VEC; x += 4) {
             float4 r;
-            r.x = f * (Ak[it][x + 0] - Dd[it] * Bk[it][x + 0]);
-            r.y = f * (Ak[it][x + 1] - Dd[it] * Bk[it][x + 1]);
-            r.z = f * (Ak[it][x + 2] - Dd[it] * Bk[it][x + 2]);
-            r.w = f * (Ak[it][x + 3] - Dd[it] * Bk[it][x + 3]);
+            r.x = f * fmaf(-Dd[it], Bk[it][x + 0], Ak[it][x + 0]);
+            r.y = f * fmaf(-Dd[it], Bk[it][x + 1], Ak[it][x + 1]);
+            r.z = f * fmaf(-Dd[it], Bk[it][x + 2], Ak[it][x + 2]);
+            r.w = f * fmaf(-Dd[it], Bk[it][x + 3], Ak[it][x + 3]);
             if (a.accumulate) {
                 const float4 o = *reinterpret_cast<const float4 *>(dqp + x);
                 r.x += o.x; r.y += o.y; r.z += o.z; r.w += o.w;
@@ -173,53 +213,90 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_kernel(SeaBwdArgs a)
 
     // ---- pass B: per-slot gradients, summed over the query-head group, scattered ---------
     float my_dlw = 0.0f;
-    for (int j = 0; j < a.s; ++j) {
-        if (!((active >> j) & 1u)) continue;  // warp-uniform
-        const int32_t t = __shfl_sync(FULL, t_l, j);
-        float pk[VEC], pv[VEC];
+    if constexpr (PAIR) {
+        // segment 0 needs the other head's q, segment 1 the other head's dO
+        float xf[VEC];
+        {
+            const uint4 send = seg == 0 ? gr[0] : qr[0];
+            uint4 recv;
+            recv.x = __shfl_xor_sync(FULL, send.x, C);
+            recv.y = __shfl_xor_sync(FULL, send.y, C);
+            recv.z = __shfl_xor_sync(FULL, send.z, C);
+            recv.w = __shfl_xor_sync(FULL, send.w, C);
+            unpack<T>(recv, xf);
+        }
+        float ownf[VEC];
 #pragma unroll
-        for (int x = 0; x < VEC; ++x) pk[x] = pv[x] = 0.0f;
-        float dzs = 0.0f;
+        for (int x = 0; x < VEC; ++x) ownf[x] = seg == 0 ? qf[0][x] : gf[0][x];
+        for (int j = 0; j < a.s; ++j) {
+            if (!((active >> j) & 1u)) continue;  // warp-uniform
+            const int32_t t = __shfl_sync(FULL, t_l, j);
+            const float p = ex2(sh_z[wid][seg][j] - m[0]) * inv[0];
+            const float dz = p * (sh_dp[wid][seg][j] - Dd[0]);
+            // segment 0 gets the other head's dz, segment 1 the other head's p
+            const float other = __shfl_xor_sync(FULL, seg == 0 ? p : dz, C);
+            const float dz_sum = dz + __shfl_xor_sync(FULL, dz, C);
+            if (lane == j) my_dlw = dz_sum;
+            // seg 0: scale * (dz_own q_own + dz_other q_other); seg 1: p_own dO_own + p_other dO_other
+            const float fo = seg == 0 ? a.scale * dz : p;
+            const float fx = seg == 0 ? a.scale * other : other;
+            float part[VEC];
 #pragma unroll
-        for (int it = 0; it < NI; ++it) {
-            const int g = it * RPI + seg;
-            if (g >= G) continue;
-            const float p = exp2f(sh_z[wid][g][j] - m[it]) * inv[it];
-            const float dz = p * (sh_dp[wid][g][j] - Dd[it]);
-            dzs += dz;
-            const float sdz = a.scale * dz;
+            for (int x = 0; x < VEC; ++x) part[x] = fmaf(fo, ownf[x], fx * xf[x]);
+            float *dst = (seg == 0 ? a.dk : a.dv) +
+                         ((size_t)(seq_base + (uint32_t)t) * a.hkv + h) * D + c * VEC;
+#pragma unroll
+            for (int x = 0; x < VEC; x += 4) red_add4(dst + x, part[x], part[x + 1], part[x + 2], part[x + 3]);
+        }
+    } else {
+        for (int j = 0; j < a.s; ++j) {
+            if (!((active >> j) & 1u)) continue;  // warp-uniform
+            const int32_t t = __shfl_sync(FULL, t_l, j);
+            float pk[VEC], pv[VEC];
+#pragma unroll
+            for (int x = 0; x < VEC; ++x) pk[x] = pv[x] = 0.0f;
+            float dzs = 0.0f;
+#pragma unroll
+            for (int it = 0; it < NI; ++it) {
+                const int g = it * RPI + seg;
+                if (g >= G) continue;
+                const float p = ex2(sh_z[wid][g][j] - m[it]) * inv[it];
+                const float dz = p * (sh_dp[wid][g][j] - Dd[it]);
+                dzs += dz;
+                const float sdz = a.scale * dz;
+#pragma unroll
+                for (int x = 0; x < VEC; ++x) {
+                    pk[x] = fmaf(sdz, qf[it][x], pk[x]);
+                    pv[x] = fmaf(p, gf[it][x], pv[x]);
+                }
+            }
+            // each segment holds a partial over its query heads: combine across segments
 #pragma unroll
             for (int x = 0; x < VEC; ++x) {
-                pk[x] = fmaf(sdz, qf[it][x], pk[x]);
-                pv[x] = fmaf(p, gf[it][x], pv[x]);
+                pk[x] = cross_seg_sum<C>(pk[x]);
+                pv[x] = cross_seg_sum<C>(pv[x]);
             }
-        }
-        // each segment holds a partial over its query heads: combine across segments
+            // dz is uniform inside a segment: count it once per segment (lane c == 0)
+            float part = c == 0 ? dzs : 0.0f;
 #pragma unroll
-        for (int x = 0; x < VEC; ++x) {
-            pk[x] = cross_seg_sum<C>(pk[x]);
-            pv[x] = cross_seg_sum<C>(pv[x]);
-        }
-        // dz is uniform inside a segment: count it once per segment (lane c == 0)
-        float part = c == 0 ? dzs : 0.0f;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(FULL, part, off);
-        if (lane == j) my_dlw = part;
+            for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(FULL, part, off);
+            if (lane == j) my_dlw = part;
 
-        const int64_t off = ((seq_base + t) * a.hkv + h) * D + c * VEC;
-        if (RPI == 1 || seg == 0) {
+            const size_t off = ((size_t)(seq_base + (uint32_t)t) * a.hkv + h) * D + c * VEC;
+            if (RPI == 1 || seg == 0) {
 #pragma unroll
-            for (int x = 0; x < VEC; x += 4)
-                red_add4(a.dk + off + x, pk[x], pk[x + 1], pk[x + 2], pk[x + 3]);
-        }
-        if (RPI == 1 || seg == 1) {
+                for (int x = 0; x < VEC; x += 4)
+                    red_add4(a.dk + off + x, pk[x], pk[x + 1], pk[x + 2], pk[x + 3]);
+            }
+            if (RPI == 1 || seg == 1) {
 #pragma unroll
-            for (int x = 0; x < VEC; x += 4)
-                red_add4(a.dv + off + x, pv[x], pv[x + 1], pv[x + 2], pv[x + 3]);
+                for (int x = 0; x < VEC; x += 4)
+                    red_add4(a.dv + off + x, pv[x], pv[x + 1], pv[x + 2], pv[x + 3]);
+            }
         }
     }
     if (lane < a.s) {
-        float *p = a.dlogw + row * a.s + lane;
+        float *p = a.dlogw + (size_t)row * a.s + lane;
         *p = a.accumulate ? *p + my_dlw : my_dlw;
     }
 }

@@ -25,25 +25,24 @@ struct SerArgs {
     float *out_w;
     int s1, s2, s3;
     int n, k;
-    int64_t rows;  // B * n * k
+    uint32_t rows;  // B * n * k
+    RowMap map;     // heads = k
 };
 
 // Referral of one edge row. On return lane r < s1 holds the r-th kept (t, W); other lanes
-// (and slots beyond the number of distinct targets) hold (0, 0.0f). `row` = (b*n + i)*k + h.
-// Must be called by all 32 lanes of the warp.
-__device__ __forceinline__ void ser_row(const SerArgs &a, int64_t row, int lane, int &t_out,
-                                        float &w_out)
+// (and slots beyond the number of distinct targets) hold (0, 0.0f). Must be called by all
+// 32 lanes of the warp. `seq_base` = b*n and `h` = channel of `row`.
+__device__ __forceinline__ void ser_row(const SerArgs &a, uint32_t row, uint32_t seq_base,
+                                        uint32_t h, int lane, int32_t &t_out, float &w_out)
 {
     const int nc = a.s2 * a.s3;
-    const int h = (int)(row % a.k);
-    const int64_t seq_base = (row / a.k) / a.n * a.n;  // b * n
 
     // first leg: lane a < s2 reads slot a of row i
     int32_t j_l = 0;
     float w1_l = 0.0f;
     if (lane < a.s2) {
-        j_l = __ldg(a.a1_idx + row * a.s2 + lane);
-        w1_l = __ldg(a.a1_w + row * a.s2 + lane);
+        j_l = __ldg(a.a1_idx + (size_t)row * a.s2 + lane);
+        w1_l = __ldg(a.a1_w + (size_t)row * a.s2 + lane);
     }
     const int ca = lane / a.s3;          // first-leg slot of this lane's candidate
     const int ce = lane - ca * a.s3;     // second-leg slot
@@ -55,12 +54,11 @@ __device__ __forceinline__ void ser_row(const SerArgs &a, int64_t row, int lane,
     int32_t t = 0;
     bool act = lane < nc && w1 > 0.0f;
     if (act && (j < 0 || j >= a.n)) {
-        // one report per active first-leg slot, from its e == 0 lane
-        if (ce == 0) raise_index_error();
+        if (ce == 0) raise_index_error();  // once per active first-leg slot
         act = false;
     }
     if (act) {
-        const int64_t r2 = ((seq_base + j) * a.k + h) * a.s3 + ce;
+        const size_t r2 = ((size_t)(seq_base + (uint32_t)j) * a.k + h) * a.s3 + ce;
         const float w2 = __ldg(a.a2_w + r2);
         const int32_t t2 = __ldg(a.a2_idx + r2);
         if (w2 > 0.0f) {
@@ -74,14 +72,18 @@ __device__ __forceinline__ void ser_row(const SerArgs &a, int64_t row, int lane,
     }
     const bool cand = u != 0.0f;
 
-    // merge: equal targets form a group; its lowest lane sums it in ascending lane order
+    // merge: equal targets form a group whose lowest lane (the leader) accumulates the
+    // other members in ascending lane order. Only non-leading members need a shuffle.
     const unsigned cmask = __ballot_sync(FULL, cand);
     const unsigned grp = __match_any_sync(FULL, cand ? t : -1) & cmask;
     const bool leader = cand && (__ffs(grp) - 1 == lane);
     float W = u;
-    for (int src = 0; src < nc; ++src) {
+    unsigned followers = __ballot_sync(FULL, cand && !leader);
+    while (followers) {  // warp-uniform loop, usually empty
+        const int src = __ffs(followers) - 1;
+        followers &= followers - 1;
         const float v = __shfl_sync(FULL, u, src);
-        if (leader && src > lane && ((grp >> src) & 1u)) W = __fadd_rn(W, v);
+        if (leader && ((grp >> src) & 1u)) W = __fadd_rn(W, v);
     }
 
     // top-s1 by (weight desc, index asc)
@@ -105,14 +107,16 @@ template <int WPB>
 __global__ void __launch_bounds__(WPB * 32) ser_kernel(SerArgs a)
 {
     const int lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * WPB + (threadIdx.x >> 5);
+    const uint32_t row = blockIdx.x * WPB + (threadIdx.x >> 5);
     if (row >= a.rows) return;  // warp-uniform
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
     int32_t t;
     float w;
-    ser_row(a, row, lane, t, w);
+    ser_row(a, row, seq_base, h, lane, t, w);
     if (lane < a.s1) {
-        a.out_idx[row * a.s1 + lane] = t;
-        a.out_w[row * a.s1 + lane] = w;
+        a.out_idx[(size_t)row * a.s1 + lane] = t;
+        a.out_w[(size_t)row * a.s1 + lane] = w;
     }
 }
 
