@@ -119,10 +119,11 @@ gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype d
 /*
  * gm_ser_sea_forward - SER followed by SEA on its output, in one kernel.
  * Same definitions as gm_ser_forward (with k = hkv) and gm_sea_forward (with s = s1, idx/w =
- * the referral output). The refreshed edges stay in registers between the two steps; they
- * are written to out_idx/out_w once, for the next layer, and never read back. out_idx and
- * out_w may both be NULL when the caller does not need them.
- * Results equal gm_ser_forward then gm_sea_forward bit for bit.
+ * the referral output). The refreshed edges stay on chip between the two steps; they are
+ * written to out_idx/out_w once, for the next layer, and never read back. out_idx and out_w
+ * may both be NULL when the caller does not need them.
+ * Results equal gm_ser_forward then gm_sea_forward bit for bit (every path computes the
+ * score dot products in the same order).
  */
 gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
                              const int32_t *a2_idx, const float *a2_w, int s3,

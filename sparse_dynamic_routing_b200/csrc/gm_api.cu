@@ -5,6 +5,7 @@
 
 #include "../../include/gm.h"
 #include "gm_common.cuh"
+#include "gm_fused_tile.cuh"
 #include "gm_sea.cuh"
 #include "gm_sea_bwd.cuh"
 #include "gm_ser.cuh"
@@ -97,18 +98,74 @@ gm_status dispatch(gm_dtype dtype, int d, int G, Args &&...args)
 #undef GM_CASE_G
 }
 
-template <typename T, int D, int G> struct SeaFwd {
-    static gm_status run(const SeaArgs &a, cudaStream_t st)
-    {
-        gm::sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(a);
-        return launched();
-    }
+// Persistent grid for a kernel with `smem` bytes of dynamic shared memory per block:
+// as many blocks as fit on the device at once, but no more than the rows need.
+template <typename K>
+unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int rows_per_block)
+{
+    int dev = 0, sms = 148, per_sm = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem);
+    const int64_t need = (rows + rows_per_block - 1) / rows_per_block;
+    const int64_t fit = (int64_t)sms * (per_sm > 0 ? per_sm : 1);
+    return (unsigned)(need < fit ? need : fit);
+}
+
+constexpr int TILE_P = 3;     // passes of copies in flight per warp
+constexpr int WPB_TILE = 4;
+
+// Shapes the tiled forward covers: 2..16 lanes per feature row, at most 16 fp32 values of
+// q per lane for the whole group, head_dim 64 or 128.
+template <typename T, int D, int G> struct TileOK {
+    static constexpr int VEC = gm::Vec<T>::N;
+    static constexpr bool value = (D == 64 || D == 128) && D / VEC >= 2 && D / VEC <= 16 && VEC * G <= 16;
 };
+
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M>
+gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
+{
+    using TG = gm::TileGeom<T, D, G, S1M>;
+    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE>;
+    const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + TILE_P * TG::STAGE);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GM_ERR_CUDA;
+    const int64_t tiles = ((int64_t)a.rows + 31) / 32;
+    const unsigned grid = persistent_blocks(kern, WPB_TILE * 32, smem, tiles, WPB_TILE);
+    kern<<<grid, WPB_TILE * 32, smem, st>>>(sa, a);
+    return launched();
+}
 
 template <typename T, int D, int G> struct SerSeaFwd {
     static gm_status run(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
     {
+        if constexpr (TileOK<T, D, G>::value) {
+            const bool aligned = aligned16(sa.a1_idx) && aligned16(sa.a1_w) && aligned16(sa.a2_idx) &&
+                                 aligned16(sa.a2_w) && aligned16(sa.out_idx) && aligned16(sa.out_w);
+            if (aligned && sa.s2 == 2 && sa.s3 == 2) {
+                if (sa.s1 <= 2) return launch_tile<T, D, G, true, 2, 2, 2>(sa, a, st);
+                if (sa.s1 <= 4) return launch_tile<T, D, G, true, 2, 2, 4>(sa, a, st);
+            }
+            if (aligned && sa.s2 == 4 && sa.s3 == 4) {
+                if (sa.s1 <= 2) return launch_tile<T, D, G, true, 4, 4, 2>(sa, a, st);
+                if (sa.s1 <= 4) return launch_tile<T, D, G, true, 4, 4, 4>(sa, a, st);
+            }
+        }
         gm::ser_sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(sa, a);
+        return launched();
+    }
+};
+
+template <typename T, int D, int G> struct SeaFwd {
+    static gm_status run(const SeaArgs &a, cudaStream_t st)
+    {
+        if constexpr (TileOK<T, D, G>::value) {
+            const SerArgs none{};
+            if (a.s <= 2) return launch_tile<T, D, G, false, 1, 1, 2>(none, a, st);
+            if (a.s <= 4) return launch_tile<T, D, G, false, 1, 1, 4>(none, a, st);
+        }
+        gm::sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(a);
         return launched();
     }
 };

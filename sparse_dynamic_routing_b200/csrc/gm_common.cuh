@@ -147,6 +147,30 @@ template <> __device__ __forceinline__ uint4 pack<__nv_bfloat16>(const float (&f
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// 16-byte asynchronous global -> shared copy (L2 only), its commit and wait (no spin loop:
+// cp.async.wait_group blocks in hardware until this thread's older groups have landed).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_async_wait()
+{
+    asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// Dot product of a 16-byte chunk of q (as fp32 pairs) with a chunk of k: even and odd
+// elements accumulate separately with packed fp32x2 FMAs, then the two halves are added.
+// Every SEA kernel uses this same order, so all paths give identical bits.
+template <int NP> __device__ __forceinline__ float chunk_dot(const float2 (&q2)[NP], const float (&kf)[2 * NP])
+{
+    float2 acc = make_float2(0.0f, 0.0f);
+#pragma unroll
+    for (int x = 0; x < NP; ++x) acc = __ffma2_rn(q2[x], make_float2(kf[2 * x], kf[2 * x + 1]), acc);
+    return acc.x + acc.y;
+}
+
 // Sum over an aligned segment of C lanes (C a power of two <= 32); every lane of the
 // segment gets the total.
 template <int C> __device__ __forceinline__ float seg_sum(float x)

@@ -1,0 +1,352 @@
+// gm_fused_tile.cuh - fused SER -> SEA forward, tiled for small edge budgets.
+//
+// Same arithmetic as ser_row + sea_row (gm_ser.cuh, gm_sea.cuh); a different division of
+// work that spends far fewer warp instructions per edge row when s2, s3, s1 are small
+// ("Graph Machine: Towards Better Pretraining via Edges", ai.info summary, "Main Findings":
+// 2 or 4 positions per KV head).
+//
+// A warp owns tiles of 32 consecutive edge rows (b, i, h).
+//  Phase 1 - referral, one thread per row. Lane L gathers its row's s2 first-leg slots and
+//    the s3 second-leg slots behind each (vector loads), forms the s2*s3 candidates in
+//    registers, merges duplicates in ascending candidate order (the first occurrence
+//    accumulates the later ones with __fadd_rn), and selects the s1 heaviest (weight desc,
+//    index asc) by repeated arg-max. Results: A' to global memory (once, for the next layer)
+//    and to a shared-memory tile with log2 weights for phase 2.
+//  Phase 2 - attention, C lanes (one 16-byte chunk each) per row, 32 / C rows per pass. Each
+//    lane handles its chunk for all G query heads of the group, so a K/V chunk is unpacked
+//    once and used G times, with packed fp32x2 FMAs. The lane stages exactly the q/K/V
+//    chunks it will read with 16-byte cp.async, P passes ahead, so every byte in flight sits
+//    in shared memory, and completion needs no spin-wait (cp.async.wait_group).
+// All shuffles run on all 32 lanes: slots are padded to S1M and inactive ones masked after
+// the reduction, so rows at a ragged tail simply compute on zeros and store nothing.
+#pragma once
+
+#include "gm_common.cuh"
+#include "gm_sea.cuh"
+#include "gm_ser.cuh"
+
+namespace gm {
+
+template <int S> __device__ __forceinline__ void ld_vec(const int32_t *p, int32_t (&o)[S])
+{
+    if constexpr (S == 4) {
+        const int4 v = __ldg(reinterpret_cast<const int4 *>(p));
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else if constexpr (S == 2) {
+        const int2 v = __ldg(reinterpret_cast<const int2 *>(p));
+        o[0] = v.x; o[1] = v.y;
+    } else {
+#pragma unroll
+        for (int x = 0; x < S; ++x) o[x] = __ldg(p + x);
+    }
+}
+template <int S> __device__ __forceinline__ void ld_vec(const float *p, float (&o)[S])
+{
+    if constexpr (S == 4) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        o[0] = v.x; o[1] = v.y; o[2] = v.z; o[3] = v.w;
+    } else if constexpr (S == 2) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
+        o[0] = v.x; o[1] = v.y;
+    } else {
+#pragma unroll
+        for (int x = 0; x < S; ++x) o[x] = __ldg(p + x);
+    }
+}
+
+// Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when both
+// are still nonzero and share a target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
+// group's members are thus added to its first occurrence in ascending candidate order.
+// Unrolled by template recursion so the candidate arrays stay in registers.
+template <int C0, int C2, int NC>
+__device__ __forceinline__ void merge_pairs(const int32_t (&ct)[NC], float (&cu)[NC])
+{
+    if constexpr (C0 < NC - 1) {
+        if constexpr (C2 < NC) {
+            const bool same = cu[C0] != 0.0f && cu[C2] != 0.0f && ct[C2] == ct[C0];
+            cu[C0] = same ? __fadd_rn(cu[C0], cu[C2]) : cu[C0];
+            cu[C2] = same ? 0.0f : cu[C2];
+            merge_pairs<C0, C2 + 1, NC>(ct, cu);
+        } else {
+            merge_pairs<C0 + 1, C0 + 2, NC>(ct, cu);
+        }
+    }
+}
+
+// Referral of one edge row by one thread (exact S2, S3; s1 <= S1M). Slots r >= s1 and slots
+// beyond the number of distinct targets come back as (0, 0.0f).
+template <int S2, int S3, int S1M>
+__device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32_t (&to)[S1M],
+                                           float (&wo)[S1M])
+{
+    constexpr int NC = S2 * S3;
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    int32_t j[S2];
+    float w1[S2];
+    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
+    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
+
+    int32_t ct[NC];
+    float cu[NC];
+#pragma unroll
+    for (int x = 0; x < S2; ++x) {
+        bool act = w1[x] > 0.0f;
+        if (act && (j[x] < 0 || j[x] >= a.n)) {
+            raise_index_error();
+            act = false;
+        }
+        int32_t t2[S3];
+        float w2[S3];
+#pragma unroll
+        for (int e = 0; e < S3; ++e) {
+            t2[e] = 0;
+            w2[e] = 0.0f;
+        }
+        if (act) {
+            const size_t r2 = ((size_t)(seq_base + (uint32_t)j[x]) * a.k + h) * S3;
+            ld_vec<S3>(a.a2_idx + r2, t2);
+            ld_vec<S3>(a.a2_w + r2, w2);
+        }
+#pragma unroll
+        for (int e = 0; e < S3; ++e) {
+            bool v = w2[e] > 0.0f;
+            if (v && (t2[e] < 0 || t2[e] >= a.n)) {
+                raise_index_error();
+                v = false;
+            }
+            ct[x * S3 + e] = t2[e];
+            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+        }
+    }
+    // merge: the first occurrence of a target absorbs the later ones, in ascending order
+    merge_pairs<0, 1, NC>(ct, cu);
+    // top-s1: repeated arg-max by (weight desc, index asc); the winner is then removed by
+    // value (nonzero targets are distinct after the merge, so the match is unique)
+#pragma unroll
+    for (int r = 0; r < S1M; ++r) {
+        float bw = 0.0f;
+        int32_t bt = 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const bool better = cu[c] > bw || (cu[c] == bw && cu[c] > 0.0f && ct[c] < bt);
+            bw = better ? cu[c] : bw;
+            bt = better ? ct[c] : bt;
+        }
+#pragma unroll
+        for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
+        const bool keep = r < a.s1 && bw > 0.0f;
+        to[r] = keep ? bt : 0;
+        wo[r] = keep ? bw : 0.0f;
+    }
+}
+
+template <typename T, int D, int G, int S1M> struct TileGeom {
+    static constexpr int VEC = Vec<T>::N;          // elements per 16-byte chunk
+    static constexpr int C = D / VEC;              // lanes per row
+    static constexpr int RPW = 32 / C;             // rows per warp pass
+    static constexpr int NPASS = 32 / RPW;         // passes per 32-row tile
+    static constexpr int ROW = D * (int)sizeof(T); // bytes per feature row
+    // per row: q rows of the group, then K and V rows of the S1M slots (chunk-interleaved
+    // per lane is not needed: every lane reads back only what it copied)
+    static constexpr int RQ = 0, RK = G * ROW, RV = RK + S1M * ROW, RBYTES = RV + S1M * ROW;
+    static constexpr int STAGE = RPW * RBYTES;
+    static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
+};
+
+// REFER = true: fused SER -> SEA (edges from the referral of sa's legs);
+// REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB>
+__global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
+{
+    using TG = TileGeom<T, D, G, S1M>;
+    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS;
+    static_assert(VEC % 2 == 0, "packed fp32x2 math");
+    extern __shared__ __align__(16) char smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    // per warp: edge tile (t, log2 w) then P stages
+    constexpr int TILE_BYTES = 32 * S1M * 8;
+    char *wbase = smem + (size_t)wid * (TILE_BYTES + P * TG::STAGE);
+    int32_t *tile_t = reinterpret_cast<int32_t *>(wbase);
+    float *tile_lw = reinterpret_cast<float *>(wbase + 32 * S1M * 4);
+    char *stages = wbase + TILE_BYTES;
+
+    const uint32_t rows = a.rows;
+    const uint32_t ntiles = (rows + 31) / 32;
+    const uint32_t W = gridDim.x * WPB;
+    const int rr = lane / C, c = lane % C;  // phase-2 row within the pass, chunk
+    const float sl2 = a.scale * LOG2E;
+    const T *Qg = static_cast<const T *>(a.q);
+    T *O = static_cast<T *>(a.o);
+
+    for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
+        const uint32_t r0 = tile * 32;
+
+        // ---- phase 1: the tile's edges, one thread per row ------------------------------
+        {
+            const uint32_t row = r0 + lane;
+            int32_t to[S1M];
+            float wo[S1M];
+#pragma unroll
+            for (int r = 0; r < S1M; ++r) {
+                to[r] = 0;
+                wo[r] = 0.0f;
+            }
+            if constexpr (!REFER) {
+                if (row < rows) {
+#pragma unroll
+                    for (int r = 0; r < S1M; ++r) {
+                        if (r < a.s) {
+                            const float w = __ldg(a.w + (size_t)row * a.s + r);
+                            const int32_t t = __ldg(a.idx + (size_t)row * a.s + r);
+                            if (w > 0.0f) {
+                                if (t < 0 || t >= a.n) {
+                                    raise_index_error();
+                                } else {
+                                    to[r] = t;
+                                    wo[r] = w;
+                                }
+                            }
+                        }
+                    }
+                }
+            } else if (row < rows) {
+                ser_thread<S2, S3, S1M>(sa, row, to, wo);
+                if (sa.out_idx != nullptr) {
+                    if (sa.s1 == S1M && S1M == 4) {
+                        *reinterpret_cast<int4 *>(sa.out_idx + (size_t)row * 4) = make_int4(to[0], to[1], to[2], to[3]);
+                        *reinterpret_cast<float4 *>(sa.out_w + (size_t)row * 4) = make_float4(wo[0], wo[1], wo[2], wo[3]);
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < S1M; ++r) {
+                            if (r < sa.s1) {
+                                sa.out_idx[(size_t)row * sa.s1 + r] = to[r];
+                                sa.out_w[(size_t)row * sa.s1 + r] = wo[r];
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int r = 0; r < S1M; ++r) {
+                tile_t[lane * S1M + r] = to[r];
+                tile_lw[lane * S1M + r] = wo[r] > 0.0f ? lg2(wo[r]) : -INFINITY;
+            }
+        }
+        __syncwarp();
+
+        // ---- phase 2: attention, RPW rows per pass, P passes of copies in flight -----------
+        auto issue = [&](int pass) {
+            if (pass < NPASS) {
+                const int lr = pass * RPW + rr;  // row within the tile
+                const uint32_t row = r0 + lr;
+                char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
+                if (row < rows) {
+                    uint32_t seq_base, h;
+                    a.map.split(row, seq_base, h);
+                    const char *qs = reinterpret_cast<const char *>(Qg + (size_t)row * G * D);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) cp_async16(st + TG::RQ + g * TG::ROW + c * 16, qs + g * TG::ROW + c * 16);
+#pragma unroll
+                    for (int jj = 0; jj < S1M; ++jj) {
+                        if (tile_lw[lr * S1M + jj] != -INFINITY) {
+                            const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * TG::ROW + c * 16;
+                            cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
+                            cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
+                        }
+                    }
+                }
+            }
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int pass = 0; pass < P; ++pass) issue(pass);
+
+        for (int pass = 0; pass < NPASS; ++pass) {
+            cp_async_wait<P - 1>();
+            const int lr = pass * RPW + rr;
+            const uint32_t row = r0 + lr;
+            const bool valid = row < rows;
+            const char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
+
+            float lw[S1M];
+            bool act[S1M];
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                lw[jj] = tile_lw[lr * S1M + jj];
+                act[jj] = valid && lw[jj] != -INFINITY;
+            }
+            // q chunks of the G heads as fp32 pairs
+            float2 q2[G][VEC / 2];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float f[VEC];
+                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16)
+                                : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                for (int x = 0; x < VEC / 2; ++x) q2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
+            }
+            // scores (all S1M slots, masked after the reduction so shuffles stay uniform)
+            float z[G][S1M];
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                float kf[VEC];
+                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16)
+                                  : make_uint4(0, 0, 0, 0), kf);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float dot = seg_sum<C>(chunk_dot<VEC / 2>(q2[g], kf));
+                    z[g][jj] = act[jj] ? fmaf(dot, sl2, lw[jj]) : -INFINITY;
+                }
+            }
+            // softmax and weighted V per head
+            float2 acc[G][VEC / 2];
+            float m[G], l[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                m[g] = z[g][0];
+#pragma unroll
+                for (int jj = 1; jj < S1M; ++jj) m[g] = fmaxf(m[g], z[g][jj]);
+                l[g] = 0.0f;
+#pragma unroll
+                for (int x = 0; x < VEC / 2; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
+            }
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                if (!act[jj]) continue;  // per lane; no shuffles below
+                float vf[VEC];
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float p = ex2(z[g][jj] - m[g]);
+                    l[g] += p;
+                    const float2 p2 = make_float2(p, p);
+#pragma unroll
+                    for (int x = 0; x < VEC / 2; ++x)
+                        acc[g][x] = __ffma2_rn(p2, make_float2(vf[2 * x], vf[2 * x + 1]), acc[g][x]);
+                }
+            }
+            if (valid) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const bool nonempty = l[g] > 0.0f;
+                    const float inv = nonempty ? __frcp_rn(l[g]) : 0.0f;
+                    float of[VEC];
+#pragma unroll
+                    for (int x = 0; x < VEC / 2; ++x) {
+                        of[2 * x] = acc[g][x].x * inv;
+                        of[2 * x + 1] = acc[g][x].y * inv;
+                    }
+                    *reinterpret_cast<uint4 *>(O + ((size_t)row * G + g) * D + c * VEC) = pack<T>(of);
+                    if (a.lse != nullptr && c == 0)
+                        a.lse[(size_t)row * G + g] = nonempty ? (m[g] + lg2(l[g])) * LN2 : -INFINITY;
+                }
+            }
+            issue(pass + P);
+        }
+        cp_async_wait<0>();
+        __syncwarp();  // the tile's edge table is rewritten by the next tile's phase 1
+    }
+}
+
+}  // namespace gm

@@ -62,9 +62,14 @@ __device__ __forceinline__ void sea_row(const SeaArgs &a, uint32_t row, uint32_t
     const T *V = static_cast<const T *>(a.v);
     const float sl2 = a.scale * LOG2E;
 
-    float qf[NI][VEC];
+    float2 q2[NI][VEC / 2];
 #pragma unroll
-    for (int it = 0; it < NI; ++it) unpack<T>(qraw[it], qf[it]);
+    for (int it = 0; it < NI; ++it) {
+        float f[VEC];
+        unpack<T>(qraw[it], f);
+#pragma unroll
+        for (int x = 0; x < VEC / 2; ++x) q2[it][x] = make_float2(f[2 * x], f[2 * x + 1]);
+    }
 
     float m[NI], l[NI], acc[NI][VEC];
 #pragma unroll
@@ -108,9 +113,7 @@ __device__ __forceinline__ void sea_row(const SeaArgs &a, uint32_t row, uint32_t
             unpack<T>(kr[jj], kf);
 #pragma unroll
             for (int it = 0; it < NI; ++it) {
-                float dot = 0.0f;
-#pragma unroll
-                for (int x = 0; x < VEC; ++x) dot = fmaf(qf[it][x], kf[x], dot);
+                const float dot = chunk_dot<VEC / 2>(q2[it], kf);
                 z[it][jj] = on[jj] ? fmaf(seg_sum<C>(dot), sl2, lw2[jj]) : -INFINITY;
             }
         }
