@@ -78,6 +78,7 @@ def shard_seed(wl: I.Workload, rank: int) -> I.Workload:
 
 
 def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of x over all ranks (the bench reports the slowest rank)."""
     if world == 1:
         return x
     import torch.distributed as dist

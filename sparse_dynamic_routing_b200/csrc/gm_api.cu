@@ -4,6 +4,7 @@
 #include <cstdint>
 
 #include "../../include/gm.h"
+#include "gm_bwd_tile.cuh"
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
 #include "gm_sea.cuh"
@@ -112,8 +113,20 @@ unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int
     return (unsigned)(need < fit ? need : fit);
 }
 
-constexpr int TILE_P = 3;     // passes of copies in flight per warp
-constexpr int WPB_TILE = 4;
+#ifndef GM_TILE_P
+#define GM_TILE_P 2
+#endif
+#ifndef GM_WPB_TILE
+#define GM_WPB_TILE 4
+#endif
+#ifndef GM_BWD_TILE_P
+#define GM_BWD_TILE_P 2
+#endif
+#ifndef GM_WPB_BWD_TILE
+#define GM_WPB_BWD_TILE 4
+#endif
+constexpr int TILE_P = GM_TILE_P;  // passes of copies in flight per warp
+constexpr int WPB_TILE = GM_WPB_TILE;
 
 // Shapes the tiled forward covers: 2..16 lanes per feature row, at most 16 fp32 values of
 // q per lane for the whole group, head_dim 64 or 128.
@@ -170,9 +183,31 @@ template <typename T, int D, int G> struct SeaFwd {
     }
 };
 
+constexpr int BWD_TILE_P = GM_BWD_TILE_P;
+constexpr int WPB_BWD_TILE = GM_WPB_BWD_TILE;
+
+template <typename T, int D, int G, int S1M>
+gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
+{
+    using TG = gm::BwdTileGeom<T, D, G, S1M>;
+    auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE>;
+    const size_t smem = (size_t)WPB_BWD_TILE * (32 * S1M * 8 + BWD_TILE_P * TG::STAGE);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return GM_ERR_CUDA;
+    const int64_t tiles = ((int64_t)a.rows + 31) / 32;
+    const unsigned grid = persistent_blocks(kern, WPB_BWD_TILE * 32, smem, tiles, WPB_BWD_TILE);
+    kern<<<grid, WPB_BWD_TILE * 32, smem, st>>>(a);
+    return launched();
+}
+
 template <typename T, int D, int G> struct SeaBwd {
     static gm_status run(const SeaBwdArgs &a, cudaStream_t st)
     {
+        if constexpr (TileOK<T, D, G>::value) {
+            if (a.s <= 2) return launch_bwd_tile<T, D, G, 2>(a, st);
+            if (a.s <= 4) return launch_bwd_tile<T, D, G, 4>(a, st);
+        }
         gm::sea_bwd_kernel<T, D, G, WPB_BWD><<<blocks_for(a.rows, WPB_BWD), WPB_BWD * 32, 0, st>>>(a);
         return launched();
     }

@@ -1,0 +1,246 @@
+// gm_bwd_tile.cuh - SEA backward, tiled for small edge budgets (s <= 4, head_dim 64/128).
+//
+// Same mathematics as sea_bwd_kernel (gm_sea_bwd.cuh); the work division of the tiled
+// forward (gm_fused_tile.cuh): a warp owns tiles of 32 consecutive edge rows; phase 1 loads
+// the tile's edges one thread per row into shared memory; phase 2 processes RPW rows per
+// pass with C lanes per row, each lane owning one 16-byte chunk of every feature row for all
+// G query heads, with q, dO, K and V chunks staged by the lane itself via cp.async P passes
+// ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
+// dp_j = dO.v_j, D = sum_j p_j dp_j and dz_j = p_j (dp_j - D):
+//   dq          = scale sum_j dz_j k_j                       (stored)
+//   dK[t_j]    += scale sum_heads dz_j q                     (16-byte fp32 vector atomics)
+//   dV[t_j]    += sum_heads p_j dO                           (16-byte fp32 vector atomics)
+//   dlogw[j]    = sum_heads dz_j                             (stored)
+// Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
+#pragma once
+
+#include "gm_common.cuh"
+#include "gm_fused_tile.cuh"
+#include "gm_sea_bwd.cuh"
+
+namespace gm {
+
+template <typename T, int D, int G, int S1M> struct BwdTileGeom {
+    static constexpr int VEC = Vec<T>::N;
+    static constexpr int C = D / VEC;
+    static constexpr int RPW = 32 / C;
+    static constexpr int NPASS = 32 / RPW;
+    static constexpr int ROW = D * (int)sizeof(T);
+    static constexpr int RQ = 0, RG = G * ROW, RK = 2 * G * ROW, RV = RK + S1M * ROW;
+    static constexpr int RBYTES = RV + S1M * ROW;
+    static constexpr int STAGE = RPW * RBYTES;
+    static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
+};
+
+template <typename T, int D, int G, int S1M, int P, int WPB>
+__global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
+{
+    using TG = BwdTileGeom<T, D, G, S1M>;
+    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
+    extern __shared__ __align__(16) char smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    constexpr int TILE_BYTES = 32 * S1M * 8;
+    char *wbase = smem + (size_t)wid * (TILE_BYTES + P * TG::STAGE);
+    int32_t *tile_t = reinterpret_cast<int32_t *>(wbase);
+    float *tile_lw = reinterpret_cast<float *>(wbase + 32 * S1M * 4);
+    char *stages = wbase + TILE_BYTES;
+
+    const uint32_t rows = a.rows;
+    const uint32_t ntiles = (rows + 31) / 32;
+    const uint32_t W = gridDim.x * WPB;
+    const int rr = lane / C, c = lane % C;
+    const float sl2 = a.scale * LOG2E;
+
+    for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
+        const uint32_t r0 = tile * 32;
+
+        // ---- phase 1: the tile's edges, one thread per row ----------------------------------
+        {
+            const uint32_t row = r0 + lane;
+#pragma unroll
+            for (int r = 0; r < S1M; ++r) {
+                int32_t t = 0;
+                float lw = -INFINITY;
+                if (row < rows && r < a.s) {
+                    const float w = __ldg(a.w + (size_t)row * a.s + r);
+                    const int32_t ti = __ldg(a.idx + (size_t)row * a.s + r);
+                    if (w > 0.0f) {
+                        if (ti < 0 || ti >= a.n) {
+                            raise_index_error();
+                        } else {
+                            t = ti;
+                            lw = lg2(w);
+                        }
+                    }
+                }
+                tile_t[lane * S1M + r] = t;
+                tile_lw[lane * S1M + r] = lw;
+            }
+        }
+        __syncwarp();
+
+        // ---- phase 2 ----------------------------------------------------------------------------
+        auto issue = [&](int pass) {
+            if (pass < NPASS) {
+                const int lr = pass * RPW + rr;
+                const uint32_t row = r0 + lr;
+                char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
+                if (row < rows) {
+                    uint32_t seq_base, h;
+                    a.map.split(row, seq_base, h);
+                    const size_t qoff = (size_t)row * G * TG::ROW + c * 16;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        cp_async16(st + TG::RQ + g * TG::ROW + c * 16, static_cast<const char *>(a.q) + qoff + g * TG::ROW);
+                        cp_async16(st + TG::RG + g * TG::ROW + c * 16, static_cast<const char *>(a.dout) + qoff + g * TG::ROW);
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < S1M; ++jj) {
+                        if (tile_lw[lr * S1M + jj] != -INFINITY) {
+                            const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * TG::ROW + c * 16;
+                            cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
+                            cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
+                        }
+                    }
+                }
+            }
+            cp_async_commit();
+        };
+#pragma unroll
+        for (int pass = 0; pass < P; ++pass) issue(pass);
+
+        for (int pass = 0; pass < NPASS; ++pass) {
+            cp_async_wait<P - 1>();
+            const int lr = pass * RPW + rr;
+            const uint32_t row = r0 + lr;
+            const bool valid = row < rows;
+            const char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
+
+            float lw[S1M];
+            bool act[S1M];
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                lw[jj] = tile_lw[lr * S1M + jj];
+                act[jj] = valid && lw[jj] != -INFINITY;
+            }
+            float2 q2[G][NP], g2[G][NP];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float f[VEC];
+                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16)
+                                : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                for (int x = 0; x < NP; ++x) q2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
+                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RG + g * TG::ROW + c * 16)
+                                : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                for (int x = 0; x < NP; ++x) g2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
+            }
+            // scores and dO.V per slot and head
+            float z[G][S1M], dp[G][S1M];
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                float kf[VEC], vf[VEC];
+                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16)
+                                  : make_uint4(0, 0, 0, 0), kf);
+                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16)
+                                  : make_uint4(0, 0, 0, 0), vf);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float sk = seg_sum<C>(chunk_dot<NP>(q2[g], kf));
+                    const float sv = seg_sum<C>(chunk_dot<NP>(g2[g], vf));
+                    z[g][jj] = act[jj] ? fmaf(sk, sl2, lw[jj]) : -INFINITY;
+                    dp[g][jj] = sv;
+                }
+            }
+            // softmax, D, dz
+            float p[G][S1M], dz[G][S1M];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                float m = z[g][0];
+#pragma unroll
+                for (int jj = 1; jj < S1M; ++jj) m = fmaxf(m, z[g][jj]);
+                float l = 0.0f, sdp = 0.0f;
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    p[g][jj] = act[jj] ? ex2(z[g][jj] - m) : 0.0f;
+                    l += p[g][jj];
+                    sdp = fmaf(p[g][jj], dp[g][jj], sdp);
+                }
+                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                const float Dd = sdp * inv;
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    p[g][jj] *= inv;
+                    dz[g][jj] = p[g][jj] * (dp[g][jj] - Dd);
+                }
+            }
+            // dq = scale sum_j dz_j k_j ; scatter dK, dV ; dlogw
+            float2 dq2[G][NP];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int x = 0; x < NP; ++x) dq2[g][x] = make_float2(0.0f, 0.0f);
+            uint32_t seq_base = 0, h = 0;
+            a.map.split(valid ? row : 0u, seq_base, h);
+#pragma unroll
+            for (int jj = 0; jj < S1M; ++jj) {
+                if (!act[jj]) continue;  // per lane; no shuffles below
+                float kf[VEC];
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
+                float2 pk[NP], pv[NP];
+#pragma unroll
+                for (int x = 0; x < NP; ++x) pk[x] = pv[x] = make_float2(0.0f, 0.0f);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float sdz = a.scale * dz[g][jj];
+                    const float2 sdz2 = make_float2(sdz, sdz), p2 = make_float2(p[g][jj], p[g][jj]);
+#pragma unroll
+                    for (int x = 0; x < NP; ++x) {
+                        dq2[g][x] = __ffma2_rn(sdz2, make_float2(kf[2 * x], kf[2 * x + 1]), dq2[g][x]);
+                        pk[x] = __ffma2_rn(sdz2, q2[g][x], pk[x]);
+                        pv[x] = __ffma2_rn(p2, g2[g][x], pv[x]);
+                    }
+                }
+                const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * D + c * VEC;
+#pragma unroll
+                for (int x = 0; x < NP; x += 2) {
+                    red_add4(a.dk + off + 2 * x, pk[x].x, pk[x].y, pk[x + 1].x, pk[x + 1].y);
+                    red_add4(a.dv + off + 2 * x, pv[x].x, pv[x].y, pv[x + 1].x, pv[x + 1].y);
+                }
+            }
+            if (valid) {
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float *dqp = a.dq + ((size_t)row * G + g) * D + c * VEC;
+#pragma unroll
+                    for (int x = 0; x < NP; x += 2) {
+                        float4 r = make_float4(dq2[g][x].x, dq2[g][x].y, dq2[g][x + 1].x, dq2[g][x + 1].y);
+                        if (a.accumulate) {
+                            const float4 o = *reinterpret_cast<const float4 *>(dqp + 2 * x);
+                            r.x += o.x; r.y += o.y; r.z += o.z; r.w += o.w;
+                        }
+                        *reinterpret_cast<float4 *>(dqp + 2 * x) = r;
+                    }
+                }
+                if (c < a.s) {
+                    float dl = 0.0f;
+#pragma unroll
+                    for (int jj = 0; jj < S1M; ++jj) {
+                        float sum = 0.0f;
+#pragma unroll
+                        for (int g = 0; g < G; ++g) sum += dz[g][jj];
+                        dl = (jj == c) ? sum : dl;
+                    }
+                    float *pd = a.dlogw + (size_t)row * a.s + c;
+                    *pd = a.accumulate ? *pd + dl : dl;
+                }
+            }
+            issue(pass + P);
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+    }
+}
+
+}  // namespace gm
