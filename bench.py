@@ -202,19 +202,18 @@ def compulsory_bytes(wl: I.Workload, a1_idx, a1_w, ap_idx, ap_w) -> dict:
         "a1": tok * hkv * wl.s2 * 8, "a2_rows": a2_rows * wl.s3 * 8,
         "a_prime": tok * hkv * wl.s1 * 8, "kv_rows": kv_rows * kv_row * 2,
     }
-    zero = {"dk_dv": 2 * tok * hkv * d * 4}
     bwd = {
         "q_dout": 2 * feat_q, "edges": tok * hkv * wl.s1 * 8, "kv_rows": kv_rows * kv_row * 2,
         "dq": tok * hq * d * 4, "dlogw": tok * hkv * wl.s1 * 4,
-        "dk_dv_rows": kv_rows * d * 4 * 2,
+        "dk_dv": 2 * tok * hkv * d * 4,  # every gradient row is written once (zeros included)
     }
     logical_fwd = (2 * hq * d * es + hq * 4
                    + hkv * (wl.s2 * 8 + wl.s2 * wl.s3 * 8 + wl.s1 * 8 + wl.s1 * 2 * kv_row)) * tok
     return {
-        "fused_forward": sum(fwd.values()), "zero_fill": sum(zero.values()),
-        "backward": sum(bwd.values()), "fused_forward_logical": logical_fwd,
+        "fused_forward": sum(fwd.values()), "backward": sum(bwd.values()),
+        "fused_forward_logical": logical_fwd,
         "kv_rows_touched": kv_rows, "kv_rows_total": tok * hkv, "a2_rows_touched": a2_rows,
-        "detail": {"fused_forward": fwd, "zero_fill": zero, "backward": bwd},
+        "detail": {"fused_forward": fwd, "backward": bwd},
     }
 
 
@@ -313,6 +312,8 @@ def run_ours(args):
     dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev)
     dv = torch.empty_like(dk)
     dlw = torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev)
+    ws_bytes = gm.gm_sea_backward_workspace_size(g["q"].dtype, wl.s1, B, n, hq, hkv, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
     stream = torch.cuda.current_stream(dev)
 
     def step(ev=None):
@@ -324,11 +325,13 @@ def run_ours(args):
         if ev is not None:
             ev[1].record(stream)
         gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], ap_i, ap_w, wl.scale, dq=dq, dk=dk,
-                           dv=dv, dlogw=dlw, stream=stream)
+                           dv=dv, dlogw=dlw, workspace=ws, stream=stream)
         if ev is not None:
             ev[2].record(stream)
 
-    launches_per_step = 3  # fused forward, zero-fill, backward
+    # fused forward; backward = counter zero-fill, row pass, three scan passes, bucket fill,
+    # gather (with a workspace) or zero-fill + scatter row pass (without)
+    launches_per_step = 1 + (7 if ws is not None else 2)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -366,10 +369,11 @@ def run_ours(args):
                           ap_w.cpu().numpy())
     peak, peak_kind = peak_hbm()
     calls = {
-        "fused_forward": {"kernel": "ser_sea_fwd_kernel", "us": fwd_ms * 1e3,
+        "fused_forward": {"kernel": "sea_fwd_tile_kernel (fused SER->SEA)", "us": fwd_ms * 1e3,
                           "bytes": cb["fused_forward"]},
-        "backward": {"kernel": "zero2_kernel+sea_bwd_kernel", "us": bwd_ms * 1e3,
-                     "bytes": cb["backward"] + cb["zero_fill"]},
+        "backward": {"kernel": "gm_sea_backward (row pass + scan + bucket fill + gather)"
+                     if ws is not None else "gm_sea_backward (zero-fill + scatter row pass)",
+                     "us": bwd_ms * 1e3, "bytes": cb["backward"]},
     }
     for c in calls.values():
         c["GBps"] = c["bytes"] / (c["us"] * 1e-6) / 1e9
@@ -440,6 +444,8 @@ def measure_e2e(gm, wl, x, dev, stream, steps, world):
         "dlw": torch.empty((B, n, hkv, wl.s1), dtype=f32, device=dev),
     }
     outs_host = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in outs_dev.items()}
+    ws_bytes = gm.gm_sea_backward_workspace_size(dev_in["q"].dtype, wl.s1, B, n, hq, hkv, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
     h2d = sum(v.numel() * v.element_size() for v in pin_in.values())
     d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
 
@@ -453,7 +459,7 @@ def measure_e2e(gm, wl, x, dev, stream, steps, world):
                               stream=stream)
         gm.gm_sea_backward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["dout"], od["ap_i"],
                            od["ap_w"], wl.scale, dq=od["dq"], dk=od["dk"], dv=od["dv"],
-                           dlogw=od["dlw"], stream=stream)
+                           dlogw=od["dlw"], workspace=ws, stream=stream)
         for k, v in od.items():
             outs_host[k].copy_(v, non_blocking=True)
 

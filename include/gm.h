@@ -44,6 +44,7 @@
 #ifndef GM_H
 #define GM_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -140,27 +141,48 @@ gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
  * With p, z as in the forward (recomputed here from q, k, v, idx, w; no forward state is
  * needed) and dp_j = <dout, v[t_j]>, dz_j = p_j (dp_j - sum_l p_l dp_l):
  *   dq[b,i,hq]      = scale * sum_j dz_j k[b,t_j,h]
- *   dk[b,t_j,h]    += scale * dz_j q[b,i,hq]          (scatter-add over all rows)
- *   dv[b,t_j,h]    += p_j dout[b,i,hq]                (scatter-add over all rows)
+ *   dk[b,t,h]       = sum over the slots (b,i,h,j) with t_j = t of scale * dz_j q[b,i,hq]
+ *   dv[b,t,h]       = sum over the same slots of p_j dout[b,i,hq]
  *   dlogw[b,i,h,j]  = sum over the group's query heads of dz_j   (gradient w.r.t. ln w_j)
- * Inactive slots get 0 in dlogw and contribute nothing. All arithmetic is fp32; the
- * scatter-adds use fp32 atomics, so dk/dv summation order (not the set of terms) varies run
- * to run.
+ * (sums over hq in the group of h). Inactive slots get 0 in dlogw and contribute nothing.
+ * All arithmetic is fp32. dk/dv are sums of many terms whose order varies run to run (the
+ * set of terms does not), so their last bits may differ between calls.
+ *
+ * Two execution paths:
+ *   - with a workspace (workspace != NULL and the shape is covered, see
+ *     gm_sea_backward_workspace_size): dk/dv are gathered per target row from a reverse
+ *     edge index built in the workspace; each dk/dv row is written once, no atomics on them;
+ *   - without one: dk/dv are zeroed by a library kernel (unless accumulating) and
+ *     scatter-added with 16-byte fp32 atomics.
  *
  *   q, k, v, dout       device, `dtype`, 16-byte aligned
  *   idx, w              device, [B, n, hkv, s]
  *   dq                  device fp32 [B, n, hq, d], 16-byte aligned
  *   dk, dv              device fp32 [B, n, hkv, d], 16-byte aligned
  *   dlogw               device fp32 [B, n, hkv, s]
- *   accumulate          0: all four outputs are overwritten (dk/dv are zeroed first by a
- *                       library kernel on `stream`); 1: results are added to their contents
+ *   workspace           device scratch owned by the caller, 16-byte aligned, at least
+ *                       gm_sea_backward_workspace_size(...) bytes; its contents on entry do
+ *                       not matter and are garbage on return; may be NULL (atomic path);
+ *                       too small (but non-NULL) is GM_ERR_INVALID_ARG
+ *   accumulate          0: all four outputs are overwritten; 1: results are added to their
+ *                       current contents
  *   limits              as gm_sea_forward
  */
 gm_status gm_sea_backward(const void *q, const void *k, const void *v, const void *dout,
                           gm_dtype dtype, const int32_t *idx, const float *w, int s,
                           int B, int n, int hq, int hkv, int d, float scale,
                           float *dq, float *dk, float *dv, float *dlogw,
+                          void *workspace, size_t workspace_bytes,
                           int accumulate, cudaStream_t stream);
+
+/*
+ * gm_sea_backward_workspace_size - bytes of workspace gm_sea_backward needs for its gather
+ * path on this shape, or 0 when the gather path does not cover it (then pass NULL). Covered:
+ * s <= 4, head_dim 64 or 128 with hq/hkv <= 2 for GM_BF16, head_dim 64 with hq/hkv <= 4 for
+ * GM_F32. The size grows as 8*(B*n*hkv) + (4 + 8*hq/hkv)*(B*n*hkv*s) bytes plus padding.
+ * Pure host function; no CUDA call.
+ */
+size_t gm_sea_backward_workspace_size(gm_dtype dtype, int s, int B, int n, int hq, int hkv, int d);
 
 /*
  * gm_check_device_errors - synchronise `stream`, then read and clear this device's error

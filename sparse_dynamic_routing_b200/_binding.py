@@ -29,7 +29,8 @@ SIGNATURES = {
     "gm_ser_sea_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _vp, _ci, _ci,
                            _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp],
     "gm_sea_backward": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf,
-                        _vp, _vp, _vp, _vp, _ci, _vp],
+                        _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _ci, _vp],
+    "gm_sea_backward_workspace_size": [_ci, _ci, _ci, _ci, _ci, _ci, _ci],
     "gm_check_device_errors": [_vp],
     "gm_status_string": [_ci],
     "gm_version": [],
@@ -62,7 +63,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         for name, args in SIGNATURES.items():
             fn = getattr(lib, name)
             fn.argtypes = args
-            fn.restype = ctypes.c_char_p if name == "gm_status_string" else ctypes.c_int
+            fn.restype = {"gm_status_string": ctypes.c_char_p,
+                          "gm_sea_backward_workspace_size": ctypes.c_size_t}.get(name, ctypes.c_int)
         _lib = lib
     return _lib
 
@@ -189,9 +191,21 @@ def gm_ser_sea_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, s1: int, scale=None,
     return out_idx, out_w, o, lse
 
 
+def gm_sea_backward_workspace_size(dtype, s: int, B: int, n: int, hq: int, hkv: int,
+                                   d: int) -> int:
+    """Workspace bytes of the gather path of gm_sea_backward (0: not covered, pass None)."""
+    dt = GM_BF16 if dtype == torch.bfloat16 else GM_F32 if dtype == torch.float32 else -1
+    return int(load_library().gm_sea_backward_workspace_size(dt, s, B, n, hq, hkv, d))
+
+
 def gm_sea_backward(q, k, v, dout, idx, w, scale=None, dq=None, dk=None, dv=None, dlogw=None,
-                    accumulate=False, stream=None):
-    """SEA backward. Returns (dq, dk, dv, dlogw), all fp32."""
+                    accumulate=False, workspace="auto", stream=None):
+    """SEA backward. Returns (dq, dk, dv, dlogw), all fp32.
+
+    workspace: "auto" allocates the gather path's scratch with torch (when the shape is
+    covered); None forces the atomic path; or a uint8 CUDA tensor of at least
+    gm_sea_backward_workspace_size(...) bytes.
+    """
     B, n, hq, d = q.shape
     hkv, s = idx.shape[2], idx.shape[3]
     if k.shape != (B, n, hkv, d) or v.shape != k.shape or w.shape != idx.shape:
@@ -204,12 +218,20 @@ def gm_sea_backward(q, k, v, dout, idx, w, scale=None, dq=None, dk=None, dv=None
     dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dk is None else dk
     dv = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dv is None else dv
     dlogw = torch.empty((B, n, hkv, s), dtype=f32, device=dev) if dlogw is None else dlogw
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a CUDA tensor")
+        nbytes = gm_sea_backward_workspace_size(q.dtype, s, B, n, hq, hkv, d)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (
+        _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size())
     lib = load_library()
     st = lib.gm_sea_backward(
         _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _ptr(dout, name="dout"),
         _fdtype(q), _ptr(idx, torch.int32, "idx"), _ptr(w, f32, "w"), s,
         B, n, hq, hkv, d, _scale(scale, d), _ptr(dq, f32, "dq"), _ptr(dk, f32, "dk"),
-        _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), int(bool(accumulate)), _stream(stream))
+        _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), ws_ptr, ws_bytes,
+        int(bool(accumulate)), _stream(stream))
     _check(st, "gm_sea_backward")
     return dq, dk, dv, dlogw
 

@@ -4,6 +4,7 @@
 #include <cstdint>
 
 #include "../../include/gm.h"
+#include "gm_bwd_gather.cuh"
 #include "gm_bwd_tile.cuh"
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
@@ -186,11 +187,11 @@ template <typename T, int D, int G> struct SeaFwd {
 constexpr int BWD_TILE_P = GM_BWD_TILE_P;
 constexpr int WPB_BWD_TILE = GM_WPB_BWD_TILE;
 
-template <typename T, int D, int G, int S1M>
+template <typename T, int D, int G, int S1M, bool GATHER>
 gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
 {
     using TG = gm::BwdTileGeom<T, D, G, S1M>;
-    auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE>;
+    auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE, GATHER>;
     const size_t smem = (size_t)WPB_BWD_TILE * (32 * S1M * 8 + BWD_TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -205,11 +206,81 @@ template <typename T, int D, int G> struct SeaBwd {
     static gm_status run(const SeaBwdArgs &a, cudaStream_t st)
     {
         if constexpr (TileOK<T, D, G>::value) {
-            if (a.s <= 2) return launch_bwd_tile<T, D, G, 2>(a, st);
-            if (a.s <= 4) return launch_bwd_tile<T, D, G, 4>(a, st);
+            if (a.s <= 2) return launch_bwd_tile<T, D, G, 2, false>(a, st);
+            if (a.s <= 4) return launch_bwd_tile<T, D, G, 4, false>(a, st);
         }
         gm::sea_bwd_kernel<T, D, G, WPB_BWD><<<blocks_for(a.rows, WPB_BWD), WPB_BWD * 32, 0, st>>>(a);
         return launched();
+    }
+};
+
+// ---- gather-based backward (workspace) -------------------------------------------------------
+
+#ifndef GM_GATHER_TPW
+#define GM_GATHER_TPW 1
+#endif
+#ifndef GM_GATHER_U
+#define GM_GATHER_U 4
+#endif
+constexpr int WPB_GATHER = 8;
+constexpr int GATHER_TPW = GM_GATHER_TPW;  // target rows per warp
+constexpr int GATHER_U = GM_GATHER_U;      // edges per load group
+
+// The gather path covers the tiled shapes with s <= 4 and fewer than 2^31 edges.
+bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
+{
+    if (s > 4 || E >= MAX_ROWS) return false;
+    if (dtype == GM_BF16) return (d == 64 || d == 128) && G <= 2;
+    return d == 64 && G <= 4;
+}
+
+struct WsLayout {
+    size_t cnt, off, list, coef, bsum, total;
+    uint32_t nblk;
+};
+
+WsLayout ws_layout(int64_t R, int64_t E, int G)
+{
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    WsLayout L;
+    L.nblk = (uint32_t)((R + gm::SCAN_TILE - 1) / gm::SCAN_TILE);
+    L.cnt = 0;
+    L.off = L.cnt + up((size_t)R * 4);
+    L.list = L.off + up((size_t)(R + 1) * 4);
+    L.coef = L.list + up((size_t)E * 4);
+    L.bsum = L.coef + up((size_t)E * 2 * G * 4);
+    L.total = L.bsum + up((size_t)L.nblk * 4);
+    return L;
+}
+
+template <typename T, int D, int G> struct SeaBwdGather {
+    static gm_status run(SeaBwdArgs a, gm::GatherWs ws, const int32_t *idx, const float *w, cudaStream_t st)
+    {
+        if constexpr (TileOK<T, D, G>::value && 2 * (D / gm::Vec<T>::N) <= 32) {
+            const int64_t R = a.rows, E = R * a.s;
+            const gm::FastDiv sdiv((uint32_t)a.s);
+            gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, R);
+            if (launched() != GM_OK) return GM_ERR_CUDA;
+            a.coef = ws.coef;
+            a.cnt = ws.cnt;
+            const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
+            if (rs != GM_OK) return rs;
+            gm::scan_block_sums_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum);
+            gm::scan_block_offsets_kernel<<<1, gm::SCAN_THREADS, 0, st>>>(ws.bsum, ws.nblk, ws.off + R);
+            gm::scan_apply_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum, ws.off);
+            if (launched() != GM_OK) return GM_ERR_CUDA;
+            const int64_t want = (E + 255) / 256;
+            gm::bucket_fill_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
+                idx, w, a.s, a.n, a.map, sdiv, E, a.hkv, ws.off, ws.cnt, ws.list);
+            if (launched() != GM_OK) return GM_ERR_CUDA;
+            const int64_t runs = (R + GATHER_TPW - 1) / GATHER_TPW;
+            gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_TPW, GATHER_U>
+                <<<blocks_for(runs, WPB_GATHER), WPB_GATHER * 32, 0, st>>>(a.q, a.dout, a.dk, a.dv, ws, sdiv,
+                                                                           (uint32_t)R, a.accumulate);
+            return launched();
+        } else {
+            return GM_ERR_UNSUPPORTED;
+        }
     }
 };
 
@@ -280,11 +351,19 @@ gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     return dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
 }
 
+size_t gm_sea_backward_workspace_size(gm_dtype dtype, int s, int B, int n, int hq, int hkv, int d)
+{
+    if (B <= 0 || n <= 0 || hq < 1 || hkv < 1 || hq % hkv != 0 || s < 1) return 0;
+    const int64_t R = (int64_t)B * n * hkv;
+    if (R >= MAX_ROWS || !gather_supported(dtype, d, hq / hkv, s, R * s)) return 0;
+    return ws_layout(R, R * s, hq / hkv).total;
+}
+
 gm_status gm_sea_backward(const void *q, const void *k, const void *v, const void *dout,
                           gm_dtype dtype, const int32_t *idx, const float *w, int s,
                           int B, int n, int hq, int hkv, int d, float scale,
                           float *dq, float *dk, float *dv, float *dlogw,
-                          int accumulate, cudaStream_t stream)
+                          void *workspace, size_t workspace_bytes, int accumulate, cudaStream_t stream)
 {
     if (accumulate != 0 && accumulate != 1) return GM_ERR_INVALID_ARG;
     gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
@@ -292,6 +371,21 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     if (!dout || !dq || !dk || !dv || !dlogw) return GM_ERR_INVALID_ARG;
     if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
     const int64_t rows = (int64_t)B * n * hkv;
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, s, n, hkv, scale, accumulate,
+                 (uint32_t)rows, row_map(hkv, n)};
+
+    const size_t need = gm_sea_backward_workspace_size(dtype, s, B, n, hq, hkv, d);
+    if (workspace != nullptr && need > 0) {
+        if (workspace_bytes < need || !aligned16(workspace)) return GM_ERR_INVALID_ARG;
+        const WsLayout L = ws_layout(rows, rows * s, hq / hkv);
+        char *base = static_cast<char *>(workspace);
+        const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
+                              reinterpret_cast<int32_t *>(base + L.list), reinterpret_cast<float *>(base + L.coef),
+                              reinterpret_cast<int32_t *>(base + L.bsum), L.nblk};
+        return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream);
+    }
+
+    // no workspace (or a shape the gather path does not cover): fp32 scatter atomics
     if (!accumulate) {
         const int64_t count4 = rows * d / 4;
         const int64_t want = (count4 + 255) / 256;
@@ -300,8 +394,6 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
                                                     reinterpret_cast<float4 *>(dv), count4);
         if (launched() != GM_OK) return GM_ERR_CUDA;
     }
-    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, s, n, hkv, scale, accumulate,
-                 (uint32_t)rows, row_map(hkv, n)};
     return dispatch<SeaBwd>(dtype, d, hq / hkv, a, stream);
 }
 

@@ -8,9 +8,12 @@
 // ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
 // dp_j = dO.v_j, D = sum_j p_j dp_j and dz_j = p_j (dp_j - D):
 //   dq          = scale sum_j dz_j k_j                       (stored)
-//   dK[t_j]    += scale sum_heads dz_j q                     (16-byte fp32 vector atomics)
-//   dV[t_j]    += sum_heads p_j dO                           (16-byte fp32 vector atomics)
+//   dK[t_j]    += scale sum_heads dz_j q                     (GATHER = false: 16-byte fp32
+//   dV[t_j]    += sum_heads p_j dO                            vector atomics)
 //   dlogw[j]    = sum_heads dz_j                             (stored)
+// With GATHER = true the two scatter-adds are not done here: the kernel stores each active
+// edge's coefficients (scale dz_g, p_g) and counts edges per target row, and the gather
+// passes of gm_bwd_gather.cuh form dK and dV.
 // Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
 #pragma once
 
@@ -32,7 +35,7 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
     static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
 };
 
-template <typename T, int D, int G, int S1M, int P, int WPB>
+template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER>
 __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
     using TG = BwdTileGeom<T, D, G, S1M>;
@@ -202,11 +205,26 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                         pv[x] = __ffma2_rn(p2, g2[g][x], pv[x]);
                     }
                 }
-                const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * D + c * VEC;
+                const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                if constexpr (GATHER) {
+                    (void)pk;
+                    (void)pv;
+                    if (c == jj) {  // one lane per edge: coefficient record and target count
+                        float *rec = a.coef + ((size_t)row * a.s + jj) * (2 * G);
 #pragma unroll
-                for (int x = 0; x < NP; x += 2) {
-                    red_add4(a.dk + off + 2 * x, pk[x].x, pk[x].y, pk[x + 1].x, pk[x + 1].y);
-                    red_add4(a.dv + off + 2 * x, pv[x].x, pv[x].y, pv[x + 1].x, pv[x + 1].y);
+                        for (int g = 0; g < G; ++g) {
+                            rec[g] = a.scale * dz[g][jj];
+                            rec[G + g] = p[g][jj];
+                        }
+                        atomicAdd(a.cnt + key, 1);
+                    }
+                } else {
+                    const size_t off = (size_t)key * D + c * VEC;
+#pragma unroll
+                    for (int x = 0; x < NP; x += 2) {
+                        red_add4(a.dk + off + 2 * x, pk[x].x, pk[x].y, pk[x + 1].x, pk[x + 1].y);
+                        red_add4(a.dv + off + 2 * x, pv[x].x, pv[x].y, pv[x + 1].x, pv[x + 1].y);
+                    }
                 }
             }
             if (valid) {

@@ -30,6 +30,8 @@ struct SeaBwdArgs {
     const int32_t *idx;
     const float *w;
     float *dq, *dk, *dv, *dlogw;
+    float *coef;   // gather mode: per-edge records of 2G floats (else unused)
+    int32_t *cnt;  // gather mode: per-target edge counts (else unused)
     int s, n, hkv;
     float scale;
     int accumulate;

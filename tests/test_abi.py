@@ -37,6 +37,18 @@ def test_every_declared_symbol_is_exported(lib):
         assert name in bnd.SIGNATURES, f"{name} has no binding"
 
 
+def test_workspace_size(lib):
+    size = lib.gm_sea_backward_workspace_size
+    R, s = 8 * 4096 * 8, 4
+    got = size(bnd.GM_BF16, s, 8, 4096, 16, 8, 128)
+    # 8 B per target row (counts + offsets), 4 + 8*G B per edge (list + 2G coefficients)
+    assert got >= 8 * R + (4 + 16) * R * s and got < 8 * R + 20 * R * s + 4096
+    assert size(bnd.GM_BF16, 8, 8, 4096, 16, 8, 128) == 0  # s > 4: atomic path only
+    assert size(bnd.GM_BF16, 4, 8, 4096, 16, 8, 256) == 0
+    assert size(bnd.GM_F32, 2, 1, 128, 2, 1, 64) > 0
+    assert size(bnd.GM_BF16, 4, 0, 4096, 16, 8, 128) == 0
+
+
 def test_status_strings(lib):
     for st in range(5):
         assert bnd.status_string(st).startswith("GM_")
@@ -101,15 +113,19 @@ def test_backward_and_fused_argument_checks(lib):
     # dout misaligned in every case: a call that got past the checks under test would still
     # be rejected before its launch
     base = [FAKE, FAKE, FAKE, FAKE + 2, bnd.GM_BF16, FAKE, FAKE, 4, 1, 8, 4, 2, 128, 0.1,
-            FAKE, FAKE, FAKE, FAKE, 0, NULL]
+            FAKE, FAKE, FAKE, FAKE, NULL, 0, 0, NULL]
     a = list(base)
-    a[18] = 2  # accumulate must be 0 or 1
+    a[20] = 2  # accumulate must be 0 or 1
     assert f(*a) == bnd.GM_ERR_INVALID_ARG
     a = list(base)
     a[14] = FAKE + 4  # misaligned dq
     assert f(*a) == bnd.GM_ERR_INVALID_ARG
     a = list(base)
     a[17] = NULL  # no dlogw
+    assert f(*a) == bnd.GM_ERR_INVALID_ARG
+    a = list(base)
+    a[3] = FAKE  # aligned dout: now a too-small workspace is what fails
+    a[18], a[19] = FAKE, 16
     assert f(*a) == bnd.GM_ERR_INVALID_ARG
     g = lib.gm_ser_sea_forward
     fb = [FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, NULL, 4, FAKE, FAKE, FAKE, bnd.GM_BF16, 1, 8, 4,

@@ -130,19 +130,42 @@ def test_long_sequence_forward_and_backward():
     o, lse = gm.gm_sea_forward(g["q"], g["k"], g["v"], g["idx"], g["w"], wl.scale)
     assert_close(o, o_ref, TOL["bf16"], "o")
     assert_close(lse, lse_ref, TOL["bf16"], "lse")
-    dq, dk, dv, dlw = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"],
-                                         wl.scale)
-    assert_close(dq, dq_ref, TOL["bf16"], "dq")
-    assert_close(dk, dk_ref, TOL["bf16"], "dk")
-    assert_close(dv, dv_ref, TOL["bf16"], "dv")
-    assert_close(dlw, dlw_ref, TOL["bf16"], "dlogw")
-    # accumulate = 1 adds onto the buffers' contents
-    gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], wl.scale,
-                       dq=dq, dk=dk, dv=dv, dlogw=dlw, accumulate=True)
-    assert_close(dq, 2 * dq_ref, 2 * TOL["bf16"], "2 dq")
-    assert_close(dk, 2 * dk_ref, 2 * TOL["bf16"], "2 dk")
-    assert_close(dv, 2 * dv_ref, 2 * TOL["bf16"], "2 dv")
-    assert_close(dlw, 2 * dlw_ref, 2 * TOL["bf16"], "2 dlogw")
+    assert gm.gm_sea_backward_workspace_size(torch.bfloat16, wl.s, wl.B, wl.n, wl.hq, wl.hkv,
+                                             wl.d) > 0
+    for ws in ("auto", None):  # gather path, atomic path
+        dq, dk, dv, dlw = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"],
+                                             wl.scale, workspace=ws)
+        assert_close(dq, dq_ref, TOL["bf16"], f"dq ({ws})")
+        assert_close(dk, dk_ref, TOL["bf16"], f"dk ({ws})")
+        assert_close(dv, dv_ref, TOL["bf16"], f"dv ({ws})")
+        assert_close(dlw, dlw_ref, TOL["bf16"], f"dlogw ({ws})")
+        # accumulate = 1 adds onto the buffers' contents
+        gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], wl.scale,
+                           dq=dq, dk=dk, dv=dv, dlogw=dlw, accumulate=True, workspace=ws)
+        assert_close(dq, 2 * dq_ref, 2 * TOL["bf16"], f"2 dq ({ws})")
+        assert_close(dk, 2 * dk_ref, 2 * TOL["bf16"], f"2 dk ({ws})")
+        assert_close(dv, 2 * dv_ref, 2 * TOL["bf16"], f"2 dv ({ws})")
+        assert_close(dlw, 2 * dlw_ref, 2 * TOL["bf16"], f"2 dlogw ({ws})")
+    gm.gm_check_device_errors()
+
+
+def test_backward_paths_on_hot_rows():
+    # Every slot of a sequence points at a handful of rows (the padding row 0 included): the
+    # gather path meets buckets with thousands of edges, the atomic path heavy contention.
+    B, n, hq, hkv, d, s = 2, 700, 16, 8, 128, 4
+    x = random_case(21, B, n, hq, hkv, d, s, "bf16", zero_frac=0.1)
+    idx = x["idx"].clone()
+    idx[..., 0] = 0
+    idx[..., 1] = torch.minimum(torch.full_like(idx[..., 1], 5), idx[..., 1])
+    x["idx"] = idx
+    scale = 1.0 / np.sqrt(d)
+    ref = oracle.sea_backward(x["q"], x["k"], x["v"], x["dout"], x["idx"], x["w"], scale)
+    g = cuda(x)
+    for ws in ("auto", None):
+        got = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], scale,
+                                 workspace=ws)
+        for name, a_, b_ in zip(("dq", "dk", "dv", "dlogw"), got, ref[:4]):
+            assert_close(a_, b_, TOL["bf16"], f"{name} ({ws})")
     gm.gm_check_device_errors()
 
 
@@ -193,9 +216,11 @@ def test_sea_shapes_forward_backward(B, n, hq, hkv, d, s, dtype):
     tol = TOL[dtype]
     assert_close(o, o_ref, tol, "o")
     assert_close(lse, lse_ref, tol, "lse")
-    got = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], scale)
-    for name, a, b in zip(("dq", "dk", "dv", "dlogw"), got, ref[:4]):
-        assert_close(a, b, tol, name)
+    for ws in ("auto", None):
+        got = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], scale,
+                                 workspace=ws)
+        for name, a, b in zip(("dq", "dk", "dv", "dlogw"), got, ref[:4]):
+            assert_close(a, b, tol, f"{name} ({ws})")
     gm.gm_check_device_errors()
 
 
