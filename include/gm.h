@@ -59,7 +59,8 @@ typedef enum gm_status {
     GM_ERR_INVALID_ARG = 1,
     GM_ERR_UNSUPPORTED = 2,
     GM_ERR_CUDA = 3,
-    GM_ERR_INDEX_RANGE = 4
+    GM_ERR_INDEX_RANGE = 4,
+    GM_ERR_SCRATCH_TOO_SMALL = 5  /* gm_sea_backward_noalloc only */
 } gm_status;
 
 /* Element type of q, k, v, o and dout. */
@@ -183,6 +184,40 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
  * Pure host function; no CUDA call.
  */
 size_t gm_sea_backward_workspace_size(gm_dtype dtype, int s, int B, int n, int hq, int hkv, int d);
+
+/*
+ * gm_sea_backward_noalloc - gm_sea_backward for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it exists for the caller, not the method.
+ *
+ * Some callers may not allocate device memory at the point where they run the backward:
+ * code called from inside a memory allocator's own hooks (which must not re-enter it), a
+ * runtime that has given all device memory to its own pool and has no way to hand out a
+ * workspace for this call, or a step loop whose policy forbids allocation because
+ * cudaMalloc/cudaFree can synchronise the device and fragment memory. This entry point takes
+ * exactly the arguments of gm_sea_backward minus the workspace, and runs its gather path on
+ * a fixed scratch array that the library holds in device memory
+ * (gm_sea_backward_noalloc_max_scratch() bytes, 32 MiB, on every device that loads the
+ * library, until the process exits). It allocates nothing and calls no allocating routine.
+ *
+ *   - The first call on a device looks up the array's device address on that device (with it
+ *     current) and caches it; make that first call before any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's contents (every call
+ *     clears what it needs zeroed). Calls whose execution overlaps on the GPU (for instance on
+ *     two streams without ordering) race on it and give wrong results: serialise them.
+ *   - Shapes the gather path does not cover (see gm_sea_backward_workspace_size) return
+ *     GM_ERR_UNSUPPORTED; a covered shape whose scratch need exceeds the array returns
+ *     GM_ERR_SCRATCH_TOO_SMALL (about 88 bytes per edge row at s = 4, hq/hkv = 2: up to
+ *     ~380k rows B*n*hkv). Both are checked before anything is launched.
+ * Results: as gm_sea_backward with a workspace.
+ */
+gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, const void *dout,
+                                  gm_dtype dtype, const int32_t *idx, const float *w, int s,
+                                  int B, int n, int hq, int hkv, int d, float scale,
+                                  float *dq, float *dk, float *dv, float *dlogw,
+                                  int accumulate, cudaStream_t stream);
+
+/* Size in bytes of the fixed scratch array gm_sea_backward_noalloc uses. Pure host function. */
+size_t gm_sea_backward_noalloc_max_scratch(void);
 
 /*
  * gm_check_device_errors - synchronise `stream`, then read and clear this device's error

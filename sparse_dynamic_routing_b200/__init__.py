@@ -16,6 +16,7 @@ from ._binding import (  # noqa: F401
     LIB_PATH,
     gm_check_device_errors,
     gm_sea_backward,
+    gm_sea_backward_noalloc,
     gm_sea_backward_workspace_size,
     gm_sea_forward,
     gm_ser_forward,

@@ -17,7 +17,8 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgm_b200.so")
 
-GM_OK, GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED, GM_ERR_CUDA, GM_ERR_INDEX_RANGE = range(5)
+(GM_OK, GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED, GM_ERR_CUDA, GM_ERR_INDEX_RANGE,
+ GM_ERR_SCRATCH_TOO_SMALL) = range(6)
 GM_F32, GM_BF16 = 0, 1
 
 # Entry points of include/gm.h with their ctypes signatures.
@@ -31,6 +32,9 @@ SIGNATURES = {
     "gm_sea_backward": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf,
                         _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _ci, _vp],
     "gm_sea_backward_workspace_size": [_ci, _ci, _ci, _ci, _ci, _ci, _ci],
+    "gm_sea_backward_noalloc": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci,
+                                _cf, _vp, _vp, _vp, _vp, _ci, _vp],
+    "gm_sea_backward_noalloc_max_scratch": [],
     "gm_check_device_errors": [_vp],
     "gm_status_string": [_ci],
     "gm_version": [],
@@ -64,7 +68,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
             fn = getattr(lib, name)
             fn.argtypes = args
             fn.restype = {"gm_status_string": ctypes.c_char_p,
-                          "gm_sea_backward_workspace_size": ctypes.c_size_t}.get(name, ctypes.c_int)
+                          "gm_sea_backward_workspace_size": ctypes.c_size_t,
+                          "gm_sea_backward_noalloc_max_scratch": ctypes.c_size_t}.get(name, ctypes.c_int)
         _lib = lib
     return _lib
 
@@ -233,6 +238,35 @@ def gm_sea_backward(q, k, v, dout, idx, w, scale=None, dq=None, dk=None, dv=None
         _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), ws_ptr, ws_bytes,
         int(bool(accumulate)), _stream(stream))
     _check(st, "gm_sea_backward")
+    return dq, dk, dv, dlogw
+
+
+def gm_sea_backward_noalloc(q, k, v, dout, idx, w, scale=None, dq=None, dk=None, dv=None,
+                            dlogw=None, accumulate=False, stream=None):
+    """gm_sea_backward on the library's fixed device scratch (no workspace is allocated).
+
+    For callers that may not allocate device memory where they run the backward; see
+    include/gm.h. Output tensors are allocated here only when not given. Calls on one device
+    share the scratch: do not let them overlap on the GPU.
+    """
+    B, n, hq, d = q.shape
+    hkv, s = idx.shape[2], idx.shape[3]
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape or w.shape != idx.shape:
+        raise ValueError("tensor shapes disagree")
+    if dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError("dout must match q")
+    dev = q.device
+    f32 = torch.float32
+    dq = torch.empty((B, n, hq, d), dtype=f32, device=dev) if dq is None else dq
+    dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dk is None else dk
+    dv = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dv is None else dv
+    dlogw = torch.empty((B, n, hkv, s), dtype=f32, device=dev) if dlogw is None else dlogw
+    st = load_library().gm_sea_backward_noalloc(
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _ptr(dout, name="dout"),
+        _fdtype(q), _ptr(idx, torch.int32, "idx"), _ptr(w, f32, "w"), s,
+        B, n, hq, hkv, d, _scale(scale, d), _ptr(dq, f32, "dq"), _ptr(dk, f32, "dk"),
+        _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_sea_backward_noalloc")
     return dq, dk, dv, dlogw
 
 

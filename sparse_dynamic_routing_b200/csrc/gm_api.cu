@@ -2,6 +2,7 @@
 // the kernel instantiation for (dtype, head_dim, GQA group), launch on the caller's stream.
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/gm.h"
 #include "gm_bwd_gather.cuh"
@@ -284,6 +285,36 @@ template <typename T, int D, int G> struct SeaBwdGather {
     }
 };
 
+// ---- scratch for callers that cannot allocate ------------------------------------------------
+//
+// gm_sea_backward_noalloc runs the gather path of gm_sea_backward on this fixed, file-scope
+// device array instead of a caller workspace. Every device that loads the library holds it
+// (NOALLOC_SCRATCH_BYTES) until the process exits, and every call on that device shares it.
+constexpr size_t NOALLOC_SCRATCH_BYTES = (size_t)32 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[NOALLOC_MAX_DEVICES] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's name
+// is only a stand-in, so its address is looked up once per device (with that device
+// current) and cached.
+gm_status noalloc_scratch(void **out)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return GM_ERR_CUDA;
+    if (dev < 0 || dev >= NOALLOC_MAX_DEVICES) return GM_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GM_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return GM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -298,6 +329,9 @@ const char *gm_status_string(gm_status status)
     case GM_ERR_UNSUPPORTED: return "GM_ERR_UNSUPPORTED: shape not supported by this build";
     case GM_ERR_CUDA: return "GM_ERR_CUDA: CUDA launch or synchronisation failed";
     case GM_ERR_INDEX_RANGE: return "GM_ERR_INDEX_RANGE: an active edge index was outside [0, n)";
+    case GM_ERR_SCRATCH_TOO_SMALL:
+        return "GM_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than the library's fixed "
+               "array holds (see gm_sea_backward_noalloc_max_scratch)";
     default: return "unknown gm_status";
     }
 }
@@ -396,6 +430,27 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     }
     return dispatch<SeaBwd>(dtype, d, hq / hkv, a, stream);
 }
+
+gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, const void *dout,
+                                  gm_dtype dtype, const int32_t *idx, const float *w, int s,
+                                  int B, int n, int hq, int hkv, int d, float scale,
+                                  float *dq, float *dk, float *dv, float *dlogw,
+                                  int accumulate, cudaStream_t stream)
+{
+    if (accumulate != 0 && accumulate != 1) return GM_ERR_INVALID_ARG;
+    gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    const size_t need = gm_sea_backward_workspace_size(dtype, s, B, n, hq, hkv, d);
+    if (need == 0) return GM_ERR_UNSUPPORTED;
+    if (need > NOALLOC_SCRATCH_BYTES) return GM_ERR_SCRATCH_TOO_SMALL;
+    void *scratch = nullptr;
+    st = noalloc_scratch(&scratch);
+    if (st != GM_OK) return st;
+    return gm_sea_backward(q, k, v, dout, dtype, idx, w, s, B, n, hq, hkv, d, scale, dq, dk, dv, dlogw,
+                           scratch, NOALLOC_SCRATCH_BYTES, accumulate, stream);
+}
+
+size_t gm_sea_backward_noalloc_max_scratch(void) { return NOALLOC_SCRATCH_BYTES; }
 
 gm_status gm_check_device_errors(cudaStream_t stream)
 {
