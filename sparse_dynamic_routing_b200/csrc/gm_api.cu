@@ -217,15 +217,18 @@ template <typename T, int D, int G> struct SeaBwd {
 
 // ---- gather-based backward (workspace) -------------------------------------------------------
 
-#ifndef GM_GATHER_TPW
-#define GM_GATHER_TPW 1
-#endif
 #ifndef GM_GATHER_U
 #define GM_GATHER_U 4
 #endif
-constexpr int WPB_GATHER = 8;
-constexpr int GATHER_TPW = GM_GATHER_TPW;  // target rows per warp
-constexpr int GATHER_U = GM_GATHER_U;      // edges per load group
+#ifndef GM_GATHER_P
+#define GM_GATHER_P 3
+#endif
+#ifndef GM_WPB_GATHER
+#define GM_WPB_GATHER 4
+#endif
+constexpr int WPB_GATHER = GM_WPB_GATHER;
+constexpr int GATHER_U = GM_GATHER_U;  // records per copy group
+constexpr int GATHER_P = GM_GATHER_P;  // copy groups in flight per warp
 
 // The gather path covers the tiled shapes with s <= 4 and fewer than 2^31 edges.
 bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
@@ -236,7 +239,7 @@ bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
 }
 
 struct WsLayout {
-    size_t cnt, off, list, coef, bsum, total;
+    size_t cnt, off, bsum, skey, srow, scoef, total;
     uint32_t nblk;
 };
 
@@ -247,37 +250,43 @@ WsLayout ws_layout(int64_t R, int64_t E, int G)
     L.nblk = (uint32_t)((R + gm::SCAN_TILE - 1) / gm::SCAN_TILE);
     L.cnt = 0;
     L.off = L.cnt + up((size_t)R * 4);
-    L.list = L.off + up((size_t)(R + 1) * 4);
-    L.coef = L.list + up((size_t)E * 4);
-    L.bsum = L.coef + up((size_t)E * 2 * G * 4);
-    L.total = L.bsum + up((size_t)L.nblk * 4);
+    L.bsum = L.off + up((size_t)(R + 1) * 4);
+    L.skey = L.bsum + up((size_t)L.nblk * 4);
+    L.srow = L.skey + up((size_t)E * 4);
+    L.scoef = L.srow + up((size_t)E * 4);
+    L.total = L.scoef + up((size_t)E * 2 * G * 4);
     return L;
 }
 
 template <typename T, int D, int G> struct SeaBwdGather {
     static gm_status run(SeaBwdArgs a, gm::GatherWs ws, const int32_t *idx, const float *w, cudaStream_t st)
     {
-        if constexpr (TileOK<T, D, G>::value && 2 * (D / gm::Vec<T>::N) <= 32) {
+        if constexpr (TileOK<T, D, G>::value && 2 * (D / gm::Vec<T>::N) <= 32 && 2 * G <= 8) {
             const int64_t R = a.rows, E = R * a.s;
             const gm::FastDiv sdiv((uint32_t)a.s);
             gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, R);
-            if (launched() != GM_OK) return GM_ERR_CUDA;
-            a.coef = ws.coef;
-            a.cnt = ws.cnt;
-            const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
-            if (rs != GM_OK) return rs;
+            const int64_t want = (E + 255) / 256;
+            gm::edge_count_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
+                idx, w, a.n, a.map, sdiv, E, a.hkv, ws.cnt);
             gm::scan_block_sums_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum);
             gm::scan_block_offsets_kernel<<<1, gm::SCAN_THREADS, 0, st>>>(ws.bsum, ws.nblk, ws.off + R);
             gm::scan_apply_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum, ws.off);
             if (launched() != GM_OK) return GM_ERR_CUDA;
-            const int64_t want = (E + 255) / 256;
-            gm::bucket_fill_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
-                idx, w, a.s, a.n, a.map, sdiv, E, a.hkv, ws.off, ws.cnt, ws.list);
-            if (launched() != GM_OK) return GM_ERR_CUDA;
-            const int64_t runs = (R + GATHER_TPW - 1) / GATHER_TPW;
-            gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_TPW, GATHER_U>
-                <<<blocks_for(runs, WPB_GATHER), WPB_GATHER * 32, 0, st>>>(a.q, a.dout, a.dk, a.dv, ws, sdiv,
-                                                                           (uint32_t)R, a.accumulate);
+            a.cnt = ws.cnt;
+            a.off = ws.off;
+            a.skey = ws.skey;
+            a.srow = ws.srow;
+            a.scoef = ws.scoef;
+            const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
+            if (rs != GM_OK) return rs;
+            auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
+            const size_t smem = (size_t)WPB_GATHER * GATHER_P * GATHER_U * G * 32 * 16;
+            if (smem > 48 * 1024 &&
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+                return GM_ERR_CUDA;
+            const int64_t chunks = (E + 31) / 32;  // upper bound: the active count is on the device
+            kern<<<blocks_for(chunks, WPB_GATHER), WPB_GATHER * 32, smem, st>>>(a.q, a.dout, a.dk, a.dv, ws,
+                                                                               (uint32_t)R, a.accumulate);
             return launched();
         } else {
             return GM_ERR_UNSUPPORTED;
@@ -405,8 +414,8 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     if (!dout || !dq || !dk || !dv || !dlogw) return GM_ERR_INVALID_ARG;
     if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
     const int64_t rows = (int64_t)B * n * hkv;
-    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, s, n, hkv, scale, accumulate,
-                 (uint32_t)rows, row_map(hkv, n)};
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, nullptr, nullptr, nullptr,
+                 s, n, hkv, scale, accumulate, (uint32_t)rows, row_map(hkv, n)};
 
     const size_t need = gm_sea_backward_workspace_size(dtype, s, B, n, hq, hkv, d);
     if (workspace != nullptr && need > 0) {
@@ -414,8 +423,9 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
         const WsLayout L = ws_layout(rows, rows * s, hq / hkv);
         char *base = static_cast<char *>(workspace);
         const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                              reinterpret_cast<int32_t *>(base + L.list), reinterpret_cast<float *>(base + L.coef),
-                              reinterpret_cast<int32_t *>(base + L.bsum), L.nblk};
+                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.skey),
+                              reinterpret_cast<int32_t *>(base + L.srow), reinterpret_cast<float *>(base + L.scoef),
+                              L.nblk};
         return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream);
     }
 

@@ -2,20 +2,21 @@
 //
 // The scatter dK[t_j] += scale dz_j q, dV[t_j] += p_j dO of the SEA backward (the derivative
 // of the attention in "Graph Machine: Towards Better Pretraining via Edges", ai.info summary,
-// "Key Contributions" item 3) is done as a gather over a reverse edge index instead of as
+// "Key Contributions" item 3) is done as a gather over edges sorted by target instead of as
 // fp32 read-modify-write atomics on the gradient rows:
-//   1. the row pass (sea_bwd_tile_kernel with GATHER = true) stores dq and d ln w as usual and,
-//      per active edge e = row * s + j, a record of 2G floats (scale dz_g, then p_g, over the
-//      query heads g of the group), and counts the edges of every target row (b, t, h) with
-//      an integer atomic;
+//   1. a count pass counts the active edges of every target row (b, t, h) (integer atomics);
 //   2. an exclusive scan of the counts gives each target row its bucket [off[r], off[r+1]);
-//   3. the fill pass drops every active edge id into its target's bucket;
-//   4. the gather pass (one warp per run of consecutive target rows) sums scale dz_g q_g over
-//      each bucket into dK and p_g dO_g into dV, and writes each row exactly once - zeros
-//      where nothing points.
-// The order of edges inside a bucket comes from integer atomics and varies run to run, so
-// dK/dV sums vary in rounding order (not in the set of terms), as with atomics. There are no
-// spin-waits: the scan is reduce -> scan of block totals -> rescan, three launches.
+//   3. the row pass (sea_bwd_tile_kernel with GATHER = true) stores dq and d ln w as usual and
+//      writes, for every active edge, a record (target row, source row, scale dz_g and p_g
+//      over the group's query heads g) straight into its target's bucket;
+//   4. the gather pass walks the sorted records in chunks of 32, one warp per chunk: a warp
+//      owns every target whose first record lies in its chunk (following it past the chunk
+//      end if needed), sums scale dz_g q_g into dK and p_g dO_g into dV, and writes each owned
+//      row once; the target rows nothing points at are written as zeros by the owner of the
+//      next non-empty target (or of the last one).
+// The order of records inside a bucket comes from integer atomics and varies run to run, so
+// dK/dV sums vary in rounding order (not in the set of terms). There are no spin-waits: the
+// scan is reduce -> scan of block totals -> rescan, three launches.
 #pragma once
 
 #include "gm_common.cuh"
@@ -24,11 +25,12 @@ namespace gm {
 
 // Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges).
 struct GatherWs {
-    int32_t *cnt;     // [R]      edge count per target row (left zeroed by the fill pass)
-    int32_t *off;     // [R + 1]  bucket offsets
-    int32_t *list;    // [E]      edge ids grouped by target row
-    float *coef;      // [E * 2G] per-edge coefficients
+    int32_t *cnt;     // [R]      edges per target row (counted, then consumed by the row pass)
+    int32_t *off;     // [R + 1]  bucket offsets; off[R] = number of active edges
     int32_t *bsum;    // [nblk]   scan block totals, then their offsets
+    int32_t *skey;    // [E]      target row of each sorted record
+    int32_t *srow;    // [E]      source edge row (b*n + i)*hkv + h of each sorted record
+    float *scoef;     // [E * 2G] scale dz_g then p_g of each sorted record
     uint32_t nblk;    // scan blocks of SCAN_TILE rows
 };
 
@@ -118,117 +120,192 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_apply_kernel(const int32_t 
     }
 }
 
-// Fill: every active edge id into its target's bucket (positions from the remaining count).
-__global__ void bucket_fill_kernel(const int32_t *idx, const float *w, int s, int n, RowMap map,
-                                   FastDiv sdiv, int64_t E, int hkv, const int32_t *off, int32_t *cnt,
-                                   int32_t *list)
+// Count: active edges per target row (range errors are reported by the row pass).
+__global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, RowMap map, FastDiv sdiv,
+                                  int64_t E, int hkv, int32_t *cnt)
 {
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < E; e += (int64_t)gridDim.x * blockDim.x) {
         const float we = w[e];
         const int32_t t = idx[e];
-        if (!(we > 0.0f) || t < 0 || t >= n) continue;  // inactive (range errors were reported by the row pass)
+        if (!(we > 0.0f) || t < 0 || t >= n) continue;
         const uint32_t row = sdiv.div((uint32_t)e);
         uint32_t seq_base, h;
         map.split(row, seq_base, h);
-        const uint32_t key = (seq_base + (uint32_t)t) * (uint32_t)hkv + h;
-        const int32_t rank = atomicSub(cnt + key, 1) - 1;
-        list[off[key] + rank] = (int32_t)e;
+        atomicAdd(cnt + (seq_base + (uint32_t)t) * (uint32_t)hkv + h, 1);
     }
 }
 
-// Gather: one warp per run of TPW consecutive target rows [r0, r0 + TPW). Lanes [0, C) own
-// dK chunk c, lanes [C, 2C) dV chunk c. The run's bucket offsets and up to 32 of its edge ids
-// are fetched with one coalesced load each; the edges are then taken U at a time straight
-// across target boundaries (every load of a group issued before any is used), and a target's
-// row is written when the walk passes its end - zeros for a target nothing points at.
-template <typename T, int D, int G, int WPB, int TPW, int U>
+// Gather: one warp per chunk of 32 sorted records. Lanes [0, C) own dK chunk c, lanes
+// [C, 2C) dV chunk c (16 bytes of every feature row). Each lane stages exactly the q (or
+// dO) chunks it will read with cp.async, U records per group, P groups ahead.
+template <typename T, int D, int G, int WPB, int U, int P>
 __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q, const void *dout, float *dk, float *dv,
-                                                                 GatherWs ws, FastDiv sdiv, uint32_t R, int accumulate)
+                                                                 GatherWs ws, uint32_t R, int accumulate)
 {
-    constexpr int VEC = Vec<T>::N, C = D / VEC, NP = VEC / 2;
-    static_assert(2 * C <= 32 && TPW < 32, "dK and dV halves fit one warp");
-    const int lane = threadIdx.x & 31;
-    const uint32_t run = blockIdx.x * WPB + (threadIdx.x >> 5);
-    const uint32_t r0 = run * TPW;
-    if (r0 >= R) return;  // warp-uniform
-    const int nt = (int)min((uint32_t)TPW, R - r0);
+    constexpr int VEC = Vec<T>::N, C = D / VEC, NP = VEC / 2, ROW = D * (int)sizeof(T);
+    constexpr int GROUP = U * G * 32 * 16;  // bytes of one group of records, all lanes
+    static_assert(2 * C <= 32, "dK and dV halves fit one warp");
+    static_assert(2 * G <= 8, "coefficients of one record fit two 16-byte loads");
+    extern __shared__ __align__(16) char smem[];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    char *ring = smem + (size_t)wid * P * GROUP;
     const int role = lane / C, c = lane % C;
     const bool working = role < 2;
-    const T *src = static_cast<const T *>(role == 0 ? q : dout);
+    const char *src = static_cast<const char *>(role == 0 ? q : dout);
     float *dst_base = (role == 0 ? dk : dv) + c * VEC;
 
-    // bucket boundaries of the run: lane L holds off[r0 + L], L <= nt
-    const int32_t my_off = lane <= nt ? __ldg(ws.off + r0 + lane) : 0;
-    const int beg = __shfl_sync(FULL, my_off, 0), end = __shfl_sync(FULL, my_off, nt);
-    const int32_t my_e = beg + lane < end ? __ldg(ws.list + beg + lane) : 0;
+    const int total = ws.off[R];
+    const int64_t chunk = (int64_t)blockIdx.x * WPB + wid;
+    const int64_t p0 = chunk * 32;
 
     float2 acc[NP];
 #pragma unroll
     for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
-    int cur = 0;                                    // target of the run being accumulated
-    int cur_end = __shfl_sync(FULL, my_off, 1);     // its bucket end
 
-    auto flush = [&]() {  // write target `cur` and move to the next one
-        if (working) {
-            float *dst = dst_base + (size_t)(r0 + cur) * D;
+    auto write_row = [&](uint32_t t) {  // acc -> row t (added to it when accumulating)
+        if (!working) return;
+        float *dst = dst_base + (size_t)t * D;
 #pragma unroll
-            for (int x = 0; x < NP; x += 2) {
-                float4 o = make_float4(acc[x].x, acc[x].y, acc[x + 1].x, acc[x + 1].y);
-                if (accumulate) {
-                    const float4 old = *reinterpret_cast<const float4 *>(dst + 2 * x);
-                    o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
-                }
-                *reinterpret_cast<float4 *>(dst + 2 * x) = o;
+        for (int x = 0; x < NP; x += 2) {
+            float4 o = make_float4(acc[x].x, acc[x].y, acc[x + 1].x, acc[x + 1].y);
+            if (accumulate) {
+                const float4 old = *reinterpret_cast<const float4 *>(dst + 2 * x);
+                o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
             }
+            *reinterpret_cast<float4 *>(dst + 2 * x) = o;
         }
+    };
+    auto zero_rows = [&](int64_t from, int64_t to) {  // rows nothing points at: [from, to)
+        if (accumulate || !working) return;
+        const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int64_t t = from; t < to; ++t) {
+            float *dst = dst_base + (size_t)t * D;
 #pragma unroll
-        for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
-        ++cur;
-        cur_end = __shfl_sync(FULL, my_off, (cur + 1) & 31);
+            for (int x = 0; x < VEC; x += 4) *reinterpret_cast<float4 *>(dst + x) = z;
+        }
     };
 
-    for (int i = beg; i < end; i += U) {
-        int32_t e[U];
-        uint4 raw[U][G];
-        float cf[U][G];
+    if (total == 0) {  // no active edge anywhere: every row is zero, 32 rows per chunk
+        zero_rows(min(p0, (int64_t)R), min(p0 + 32, (int64_t)R));
+        return;
+    }
+    if (p0 >= total) return;  // warp-uniform
+
+    // the chunk's records
+    const int kend = (int)min((int64_t)32, (int64_t)total - p0);
+    const bool in = lane < kend;
+    const int32_t mkey = in ? __ldg(ws.skey + p0 + lane) : -1;
+    const int32_t mrow = in ? __ldg(ws.srow + p0 + lane) : 0;
+    float mcf[2 * G];
+#pragma unroll
+    for (int x = 0; x < 2 * G; ++x) mcf[x] = in ? __ldg(ws.scoef + (p0 + lane) * (2 * G) + x) : 0.0f;
+    const int32_t prev_key = p0 > 0 ? __ldg(ws.skey + p0 - 1) : -1;
+
+    // a leading run that continues the previous chunk's last target belongs to that chunk
+    const int start = __popc(__ballot_sync(FULL, in && mkey == prev_key));
+    if (start == kend) return;  // warp-uniform
+
+    auto issue = [&](int grp) {  // group grp of the window: records start + grp*U ...
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int k = i + u - beg;
-            const int32_t from_reg = __shfl_sync(FULL, my_e, k & 31);
-            e[u] = i + u >= end ? -1 : (k < 32 ? from_reg : __ldg(ws.list + i + u));
-        }
+            const int k = start + grp * U + u;
+            const int32_t row = __shfl_sync(FULL, mrow, k & 31);
+            if (k < kend && working) {
+                char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                raw[u][g] = make_uint4(0, 0, 0, 0);
-                cf[u][g] = 0.0f;
+                for (int g = 0; g < G; ++g)
+                    cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
             }
-            if (e[u] >= 0 && working) {
-                const uint32_t row = sdiv.div((uint32_t)e[u]);
-                const float *rec = ws.coef + (size_t)e[u] * (2 * G) + role * G;
+        }
+        cp_async_commit();
+    };
+
+    uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, start);
+    zero_rows((int64_t)prev_key + 1, cur);
+    const int ngroups = (kend - start + U - 1) / U;
+#pragma unroll
+    for (int grp = 0; grp < P; ++grp) issue(grp);
+    for (int grp = 0; grp < ngroups; ++grp) {
+        cp_async_wait<P - 1>();
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int k = start + grp * U + u;
+            const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
+            float cf[2 * G];
+#pragma unroll
+            for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
+            if (k >= kend) break;  // warp-uniform
+            if (key != cur) {      // warp-uniform: a new target starts here
+                write_row(cur);
+#pragma unroll
+                for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
+                zero_rows((int64_t)cur + 1, key);
+                cur = key;
+            }
+            if (working) {
+                const char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    cf[u][g] = __ldg(rec + g);
-                    raw[u][g] = ld16(src + ((size_t)row * G + g) * D + c * VEC);
+                    float f[VEC];
+                    unpack<T>(*reinterpret_cast<const uint4 *>(slot + g * 32 * 16), f);
+                    const float k2 = role == 0 ? cf[g] : cf[G + g];
+                    const float2 kk = make_float2(k2, k2);
+#pragma unroll
+                    for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
                 }
             }
         }
+        issue(grp + P);
+    }
+    cp_async_wait<0>();
+
+    // the last owned target may continue past the chunk: follow it (rare, hot rows)
+    int64_t pos = p0 + kend;
+    while (pos < total) {
+        const int64_t left = (int64_t)total - pos;
+        const bool in2 = lane < left;
+        const int32_t key2 = in2 ? __ldg(ws.skey + pos + lane) : -1;
+        const int run = __popc(__ballot_sync(FULL, in2 && (uint32_t)key2 == cur));
+        if (run == 0) break;  // warp-uniform
+        const int32_t row2 = in2 ? __ldg(ws.srow + pos + lane) : 0;
+        float cf2[2 * G];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            if (i + u >= end) break;                 // warp-uniform
-            while (i + u >= cur_end && cur < nt) flush();  // warp-uniform: targets that ended here
+        for (int x = 0; x < 2 * G; ++x) cf2[x] = in2 ? __ldg(ws.scoef + (pos + lane) * (2 * G) + x) : 0.0f;
+        for (int k0 = 0; k0 < run; k0 += U) {
+            uint4 raw[U][G];
+            float cf[U][2 * G];
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                float f[VEC];
-                unpack<T>(raw[u][g], f);
-                const float2 k2 = make_float2(cf[u][g], cf[u][g]);
+            for (int u = 0; u < U; ++u) {
+                const int k = k0 + u;
+                const int32_t row = __shfl_sync(FULL, row2, k & 31);
 #pragma unroll
-                for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(k2, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+                for (int x = 0; x < 2 * G; ++x) cf[u][x] = __shfl_sync(FULL, cf2[x], k & 31);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    raw[u][g] = make_uint4(0, 0, 0, 0);
+                    if (k < run && working)
+                        raw[u][g] = ld16(src + ((size_t)row * G + g) * ROW + c * 16);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (k0 + u >= run || !working) continue;
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float f[VEC];
+                    unpack<T>(raw[u][g], f);
+                    const float k2 = role == 0 ? cf[u][g] : cf[u][G + g];
+                    const float2 kk = make_float2(k2, k2);
+#pragma unroll
+                    for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+                }
             }
         }
+        pos += run;
+        if (run < 32) break;  // the target ended inside this window
     }
-    while (cur < nt) flush();  // the last target, and any empty ones after it
+    write_row(cur);
+    if (pos >= total) zero_rows((int64_t)cur + 1, R);  // owner of the last target: trailing rows
 }
 
 }  // namespace gm

@@ -11,9 +11,9 @@
 //   dK[t_j]    += scale sum_heads dz_j q                     (GATHER = false: 16-byte fp32
 //   dV[t_j]    += sum_heads p_j dO                            vector atomics)
 //   dlogw[j]    = sum_heads dz_j                             (stored)
-// With GATHER = true the two scatter-adds are not done here: the kernel stores each active
-// edge's coefficients (scale dz_g, p_g) and counts edges per target row, and the gather
-// passes of gm_bwd_gather.cuh form dK and dV.
+// With GATHER = true the two scatter-adds are not done here: the kernel writes each active
+// edge's record (target row, source row, scale dz_g, p_g) into its target's bucket, and the
+// gather pass of gm_bwd_gather.cuh forms dK and dV.
 // Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
 #pragma once
 
@@ -209,14 +209,20 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                 if constexpr (GATHER) {
                     (void)pk;
                     (void)pv;
-                    if (c == jj) {  // one lane per edge: coefficient record and target count
-                        float *rec = a.coef + ((size_t)row * a.s + jj) * (2 * G);
+                    if (c == jj) {  // one lane per edge: its record, into its target's bucket
+                        const int32_t pos = a.off[key] + atomicSub(a.cnt + key, 1) - 1;
+                        // the count pass applies the same activity test, so pos stays inside the
+                        // bucket; the bound below only keeps a broken invariant from writing
+                        // outside the record arrays
+                        if ((uint32_t)pos >= a.rows * (uint32_t)a.s) continue;
+                        a.skey[pos] = (int32_t)key;
+                        a.srow[pos] = (int32_t)row;
+                        float *rec = a.scoef + (size_t)pos * (2 * G);
 #pragma unroll
                         for (int g = 0; g < G; ++g) {
                             rec[g] = a.scale * dz[g][jj];
                             rec[G + g] = p[g][jj];
                         }
-                        atomicAdd(a.cnt + key, 1);
                     }
                 } else {
                     const size_t off = (size_t)key * D + c * VEC;

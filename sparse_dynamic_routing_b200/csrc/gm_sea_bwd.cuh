@@ -30,8 +30,12 @@ struct SeaBwdArgs {
     const int32_t *idx;
     const float *w;
     float *dq, *dk, *dv, *dlogw;
-    float *coef;   // gather mode: per-edge records of 2G floats (else unused)
-    int32_t *cnt;  // gather mode: per-target edge counts (else unused)
+    // gather mode only (see gm_bwd_gather.cuh): target counts (consumed), bucket offsets, and
+    // the sorted record arrays; unused by the atomic path
+    int32_t *cnt;
+    const int32_t *off;
+    int32_t *skey, *srow;
+    float *scoef;
     int s, n, hkv;
     float scale;
     int accumulate;
