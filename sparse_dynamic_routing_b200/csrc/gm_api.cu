@@ -239,22 +239,21 @@ bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
 }
 
 struct WsLayout {
-    size_t cnt, off, bsum, skey, srow, scoef, total;
+    size_t cnt, off, bsum, srec, total;
     uint32_t nblk;
 };
 
 WsLayout ws_layout(int64_t R, int64_t E, int G)
 {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    const int words = (2 + 2 * G + 3) / 4 * 4;  // gm::Rec<G>::WORDS
     WsLayout L;
     L.nblk = (uint32_t)((R + gm::SCAN_TILE - 1) / gm::SCAN_TILE);
     L.cnt = 0;
     L.off = L.cnt + up((size_t)R * 4);
     L.bsum = L.off + up((size_t)(R + 1) * 4);
-    L.skey = L.bsum + up((size_t)L.nblk * 4);
-    L.srow = L.skey + up((size_t)E * 4);
-    L.scoef = L.srow + up((size_t)E * 4);
-    L.total = L.scoef + up((size_t)E * 2 * G * 4);
+    L.srec = L.bsum + up((size_t)L.nblk * 4);
+    L.total = L.srec + up((size_t)E * words * 4);
     return L;
 }
 
@@ -274,9 +273,7 @@ template <typename T, int D, int G> struct SeaBwdGather {
             if (launched() != GM_OK) return GM_ERR_CUDA;
             a.cnt = ws.cnt;
             a.off = ws.off;
-            a.skey = ws.skey;
-            a.srow = ws.srow;
-            a.scoef = ws.scoef;
+            a.srec = ws.srec;
             const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
             if (rs != GM_OK) return rs;
             auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
@@ -414,7 +411,7 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     if (!dout || !dq || !dk || !dv || !dlogw) return GM_ERR_INVALID_ARG;
     if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
     const int64_t rows = (int64_t)B * n * hkv;
-    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, nullptr, nullptr, nullptr,
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, nullptr,
                  s, n, hkv, scale, accumulate, (uint32_t)rows, row_map(hkv, n)};
 
     const size_t need = gm_sea_backward_workspace_size(dtype, s, B, n, hq, hkv, d);
@@ -423,8 +420,7 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
         const WsLayout L = ws_layout(rows, rows * s, hq / hkv);
         char *base = static_cast<char *>(workspace);
         const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.skey),
-                              reinterpret_cast<int32_t *>(base + L.srow), reinterpret_cast<float *>(base + L.scoef),
+                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.srec),
                               L.nblk};
         return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream);
     }

@@ -23,14 +23,52 @@
 
 namespace gm {
 
+// A sorted record: target row, source edge row (b*n + i)*hkv + h, then scale dz_g and p_g
+// for the G query heads (fp32 bits), padded to whole 16-byte words (32 bytes for G = 2), so
+// the row pass writes and the gather pass reads it in full sectors.
+template <int G> struct Rec {
+    static constexpr int WORDS = (2 + 2 * G + 3) / 4 * 4;
+};
+
+template <int G>
+__device__ __forceinline__ void write_record(int32_t *srec, int32_t pos, uint32_t key, uint32_t row,
+                                             const float (&cf)[2 * G])
+{
+    int32_t w[Rec<G>::WORDS];
+    w[0] = (int32_t)key;
+    w[1] = (int32_t)row;
+#pragma unroll
+    for (int x = 0; x < 2 * G; ++x) w[2 + x] = __float_as_int(cf[x]);
+#pragma unroll
+    for (int x = 2 + 2 * G; x < Rec<G>::WORDS; ++x) w[x] = 0;
+    int4 *dst = reinterpret_cast<int4 *>(srec + (size_t)pos * Rec<G>::WORDS);
+#pragma unroll
+    for (int x = 0; x < Rec<G>::WORDS / 4; ++x) dst[x] = make_int4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
+}
+
+template <int G>
+__device__ __forceinline__ void read_record(const int32_t *srec, int64_t pos, int32_t &key, int32_t &row,
+                                            float (&cf)[2 * G])
+{
+    int32_t w[Rec<G>::WORDS];
+    const int4 *src = reinterpret_cast<const int4 *>(srec + pos * Rec<G>::WORDS);
+#pragma unroll
+    for (int x = 0; x < Rec<G>::WORDS / 4; ++x) {
+        const int4 v = __ldg(src + x);
+        w[4 * x] = v.x; w[4 * x + 1] = v.y; w[4 * x + 2] = v.z; w[4 * x + 3] = v.w;
+    }
+    key = w[0];
+    row = w[1];
+#pragma unroll
+    for (int x = 0; x < 2 * G; ++x) cf[x] = __int_as_float(w[2 + x]);
+}
+
 // Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges).
 struct GatherWs {
     int32_t *cnt;     // [R]      edges per target row (counted, then consumed by the row pass)
     int32_t *off;     // [R + 1]  bucket offsets; off[R] = number of active edges
     int32_t *bsum;    // [nblk]   scan block totals, then their offsets
-    int32_t *skey;    // [E]      target row of each sorted record
-    int32_t *srow;    // [E]      source edge row (b*n + i)*hkv + h of each sorted record
-    float *scoef;     // [E * 2G] scale dz_g then p_g of each sorted record
+    int32_t *srec;    // [E * Rec<G>::WORDS] records sorted by target row
     uint32_t nblk;    // scan blocks of SCAN_TILE rows
 };
 
@@ -194,12 +232,12 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
     // the chunk's records
     const int kend = (int)min((int64_t)32, (int64_t)total - p0);
     const bool in = lane < kend;
-    const int32_t mkey = in ? __ldg(ws.skey + p0 + lane) : -1;
-    const int32_t mrow = in ? __ldg(ws.srow + p0 + lane) : 0;
+    int32_t mkey = -1, mrow = 0;
     float mcf[2 * G];
 #pragma unroll
-    for (int x = 0; x < 2 * G; ++x) mcf[x] = in ? __ldg(ws.scoef + (p0 + lane) * (2 * G) + x) : 0.0f;
-    const int32_t prev_key = p0 > 0 ? __ldg(ws.skey + p0 - 1) : -1;
+    for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
+    if (in) read_record<G>(ws.srec, p0 + lane, mkey, mrow, mcf);
+    const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
 
     // a leading run that continues the previous chunk's last target belongs to that chunk
     const int start = __popc(__ballot_sync(FULL, in && mkey == prev_key));
@@ -264,13 +302,13 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
     while (pos < total) {
         const int64_t left = (int64_t)total - pos;
         const bool in2 = lane < left;
-        const int32_t key2 = in2 ? __ldg(ws.skey + pos + lane) : -1;
-        const int run = __popc(__ballot_sync(FULL, in2 && (uint32_t)key2 == cur));
-        if (run == 0) break;  // warp-uniform
-        const int32_t row2 = in2 ? __ldg(ws.srow + pos + lane) : 0;
+        int32_t key2 = -1, row2 = 0;
         float cf2[2 * G];
 #pragma unroll
-        for (int x = 0; x < 2 * G; ++x) cf2[x] = in2 ? __ldg(ws.scoef + (pos + lane) * (2 * G) + x) : 0.0f;
+        for (int x = 0; x < 2 * G; ++x) cf2[x] = 0.0f;
+        if (in2) read_record<G>(ws.srec, pos + lane, key2, row2, cf2);
+        const int run = __popc(__ballot_sync(FULL, in2 && (uint32_t)key2 == cur));
+        if (run == 0) break;  // warp-uniform
         for (int k0 = 0; k0 < run; k0 += U) {
             uint4 raw[U][G];
             float cf[U][2 * G];

@@ -17,6 +17,7 @@
 // Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
 #pragma once
 
+#include "gm_bwd_gather.cuh"
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
 #include "gm_sea_bwd.cuh"
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                 if (row < rows) {
                     uint32_t seq_base, h;
                     a.map.split(row, seq_base, h);
-                    const size_t qoff = (size_t)row * G * TG::ROW + c * 16;
+                    const size_t qoff = (size_t)row * (G * TG::ROW) + c * 16;
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
                         cp_async16(st + TG::RQ + g * TG::ROW + c * 16, static_cast<const char *>(a.q) + qoff + g * TG::ROW);
@@ -100,7 +101,8 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * TG::ROW + c * 16;
+                            const uint32_t kvrow = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                            const size_t off = (size_t)kvrow * TG::ROW + c * 16;
                             cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
                             cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
                         }
@@ -205,32 +207,41 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                         pv[x] = __ffma2_rn(p2, g2[g][x], pv[x]);
                     }
                 }
-                const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
-                if constexpr (GATHER) {
-                    (void)pk;
-                    (void)pv;
-                    if (c == jj) {  // one lane per edge: its record, into its target's bucket
-                        const int32_t pos = a.off[key] + atomicSub(a.cnt + key, 1) - 1;
-                        // the count pass applies the same activity test, so pos stays inside the
-                        // bucket; the bound below only keeps a broken invariant from writing
-                        // outside the record arrays
-                        if ((uint32_t)pos >= a.rows * (uint32_t)a.s) continue;
-                        a.skey[pos] = (int32_t)key;
-                        a.srow[pos] = (int32_t)row;
-                        float *rec = a.scoef + (size_t)pos * (2 * G);
-#pragma unroll
-                        for (int g = 0; g < G; ++g) {
-                            rec[g] = a.scale * dz[g][jj];
-                            rec[G + g] = p[g][jj];
-                        }
-                    }
-                } else {
+                if constexpr (!GATHER) {
+                    const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
                     const size_t off = (size_t)key * D + c * VEC;
 #pragma unroll
                     for (int x = 0; x < NP; x += 2) {
                         red_add4(a.dk + off + 2 * x, pk[x].x, pk[x].y, pk[x + 1].x, pk[x + 1].y);
                         red_add4(a.dv + off + 2 * x, pv[x].x, pv[x].y, pv[x + 1].x, pv[x + 1].y);
                     }
+                } else {
+                    (void)pk;
+                    (void)pv;
+                }
+            }
+            if constexpr (GATHER) {
+                // lane c < S1M files slot c's record into its target's bucket: one integer atomic
+                // per pass for all slots, then one 32-byte record
+                bool mine = false;
+                float rc[2 * G];
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    if (c == jj) {
+                        mine = act[jj];
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            rc[g] = a.scale * dz[g][jj];
+                            rc[G + g] = p[g][jj];
+                        }
+                    }
+                }
+                if (c < S1M && mine) {
+                    const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + c]) * (uint32_t)a.hkv + h;
+                    const int32_t pos = a.off[key] + atomicSub(a.cnt + key, 1) - 1;
+                    // the count pass applies the same activity test, so pos stays inside the
+                    // bucket; the bound only keeps a broken invariant from writing outside
+                    if ((uint32_t)pos < a.rows * (uint32_t)a.s) write_record<G>(a.srec, pos, key, row, rc);
                 }
             }
             if (valid) {

@@ -244,13 +244,14 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 if (row < rows) {
                     uint32_t seq_base, h;
                     a.map.split(row, seq_base, h);
-                    const char *qs = reinterpret_cast<const char *>(Qg + (size_t)row * G * D);
+                    const char *qs = reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW);
 #pragma unroll
                     for (int g = 0; g < G; ++g) cp_async16(st + TG::RQ + g * TG::ROW + c * 16, qs + g * TG::ROW + c * 16);
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const size_t off = ((size_t)(seq_base + (uint32_t)tile_t[lr * S1M + jj]) * a.hkv + h) * TG::ROW + c * 16;
+                            const uint32_t kvrow = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                            const size_t off = (size_t)kvrow * TG::ROW + c * 16;
                             cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
                             cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
                         }

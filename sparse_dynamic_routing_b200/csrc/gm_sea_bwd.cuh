@@ -34,8 +34,7 @@ struct SeaBwdArgs {
     // the sorted record arrays; unused by the atomic path
     int32_t *cnt;
     const int32_t *off;
-    int32_t *skey, *srow;
-    float *scoef;
+    int32_t *srec;
     int s, n, hkv;
     float scale;
     int accumulate;
