@@ -1,4 +1,4 @@
-"""CPU oracle of the Graph Machine sparse layer (SER, SEA forward, SEA backward).
+"""CPU oracle of the Graph Machine sparse layer (SER and its backward, SEA and its backward).
 
 TEST INFRASTRUCTURE. Only the tests, the package smoke check and the benchmark's CPU-baseline
 leg import this module. It wraps the plain C library built from gm_oracle.c (compiled on
@@ -32,6 +32,9 @@ def _load():
         lib.oracle_num_threads.restype = ci
         lib.oracle_ser.restype = ctypes.c_int64
         lib.oracle_ser.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci, ci, ci, ci]
+        lib.oracle_ser_backward.restype = ctypes.c_int64
+        lib.oracle_ser_backward.argtypes = [i32p, f32p, ci, i32p, f32p, ci, f32p, ci, ci, ci, ci, ci,
+                                            f64p, f64p]
         lib.oracle_sea_forward.restype = ctypes.c_int64
         lib.oracle_sea_forward.argtypes = [f32p, f32p, f32p, i32p, f32p, ci, ci, ci, ci, ci, ci,
                                            ctypes.c_double, ctypes.c_void_p, ctypes.c_int64,
@@ -71,6 +74,27 @@ def ser(a1_idx, a1_w, a2_idx, a2_w, s1: int):
     if bad < 0:
         raise ValueError("s2*s3 exceeds the oracle's candidate buffer")
     return out_i, out_w, int(bad)
+
+
+def ser_backward(a1_idx, a1_w, a2_idx, a2_w, gout, grad_is_log: bool = False):
+    """Gradients of the kept referral weights with respect to both legs' weights (fp64).
+
+    gout [B, n, k, s1]: gradient w.r.t. A'.w (or w.r.t. ln A'.w when grad_is_log).
+    Returns (dw1 [B,n,k,s2], dw2 [B,n,k,s3], bad_refs).
+    """
+    i1, w1 = _np(a1_idx, np.int32), _np(a1_w, np.float32)
+    i2, w2 = _np(a2_idx, np.int32), _np(a2_w, np.float32)
+    g = _np(gout, np.float32)
+    B, n, k, s2 = i1.shape
+    s3, s1 = i2.shape[3], g.shape[3]
+    assert i2.shape[:3] == (B, n, k) and g.shape[:3] == (B, n, k)
+    dw1 = np.zeros(i1.shape, np.float64)
+    dw2 = np.zeros(i2.shape, np.float64)
+    bad = _load().oracle_ser_backward(i1, w1, s2, i2, w2, s3, g, s1, int(bool(grad_is_log)),
+                                      B, n, k, dw1, dw2)
+    if bad < 0:
+        raise ValueError("s2*s3 exceeds the oracle's candidate buffer")
+    return dw1, dw2, int(bad)
 
 
 def sea_forward(q, k, v, idx, w, scale: float | None = None, rows=None):

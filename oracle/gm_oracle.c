@@ -1,6 +1,6 @@
 /*
  * gm_oracle.c - CPU oracle of the Graph Machine sparse layer: sparse edge referral (SER),
- * sparse edge attention (SEA) and the SEA backward pass.
+ * sparse edge attention (SEA), and the backward passes of both.
  *
  * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the benchmark's
  * CPU-baseline leg load this library; the CUDA library shares no code with it and never
@@ -40,6 +40,8 @@
  *   R7  GQA: query head hq reads KV head hq / (Hq / Hkv) (contiguous groups).
  *   R8  an active slot whose index lies outside [0, n) is skipped and counted; the count is
  *       the return value of each entry point.
+ *   R9  SER backward: only the kept (top-s1, weight > 0) merged weights carry gradient; the
+ *       selection itself is piecewise constant and passes none; indices get none.
  *
  * Layouts are contiguous row-major: features [B, n, H, d], edges [B, n, k, s].
  */
@@ -141,6 +143,105 @@ int64_t oracle_ser(const int32_t *a1_idx, const float *a1_w, int s2,
         for (int r = 0; r < s1; ++r) {
             out_idx[row * s1 + r] = r < nu ? ut[r] : 0;
             out_w[row * s1 + r] = r < nu ? uw[r] : 0.0f;
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * SER backward   [MPE2]; readings R1-R5, R8, R9.
+ *
+ * gout [B, n, k, s1]: gradient with respect to the kept weights A'.w (or, if grad_is_log, with
+ * respect to ln A'.w, converted here as g / W). For each row the forward's candidates, merge
+ * and selection are recomputed exactly as in oracle_ser; then for every candidate
+ * c = (a, e) whose target t_c was kept in slot r (W_r > 0):
+ *     dw1[b,i,h,a]  += g_r * w2[b,j,h,e]          (j = A1.idx[b,i,h,a])
+ *     dw2[b,j,h,e]  += g_r * w1[b,i,h,a]          (summed over every row that reaches it)
+ * in fp64. Work is split over (b, h) planes: a row only reaches second-leg rows of its own
+ * sequence and channel, so each plane owns its dw1 and dw2 entries.
+ * ---------------------------------------------------------------------------------------- */
+int64_t oracle_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                            const int32_t *a2_idx, const float *a2_w, int s3,
+                            const float *gout, int s1, int grad_is_log,
+                            int B, int n, int k, double *dw1, double *dw2)
+{
+    int64_t bad = 0;
+    if (s2 * s3 > ORACLE_MAX_CAND) return -1;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (int64_t plane = 0; plane < (int64_t)B * k; ++plane) {
+        const int64_t b = plane / k;
+        const int h = (int)(plane % k);
+        for (int i = 0; i < n; ++i) {
+            const int64_t row = ((int64_t)b * n + i) * k + h;
+            for (int a = 0; a < s2; ++a) dw1[row * s2 + a] = 0.0;
+            for (int e = 0; e < s3; ++e) dw2[row * s3 + e] = 0.0;
+        }
+        for (int i = 0; i < n; ++i) {
+            const int64_t row = ((int64_t)b * n + i) * k + h;
+            /* forward, exactly as oracle_ser */
+            int32_t cand_t[ORACLE_MAX_CAND], cand_a[ORACLE_MAX_CAND];
+            float cand_u[ORACLE_MAX_CAND];
+            int64_t cand_r2[ORACLE_MAX_CAND];
+            int nc = 0;
+            for (int a = 0; a < s2; ++a) {
+                const float w1 = a1_w[row * s2 + a];
+                if (!(w1 > 0.0f)) continue;
+                const int32_t j = a1_idx[row * s2 + a];
+                if (j < 0 || j >= n) { ++bad; continue; }
+                const int64_t row_j = ((int64_t)b * n + j) * k + h;
+                for (int e = 0; e < s3; ++e) {
+                    const float w2 = a2_w[row_j * s3 + e];
+                    if (!(w2 > 0.0f)) continue;
+                    const int32_t t = a2_idx[row_j * s3 + e];
+                    if (t < 0 || t >= n) { ++bad; continue; }
+                    const float u = w1 * w2;
+                    if (u == 0.0f) continue;
+                    cand_t[nc] = t;
+                    cand_u[nc] = u;
+                    cand_a[nc] = a;
+                    cand_r2[nc] = row_j * s3 + e;
+                    ++nc;
+                }
+            }
+            int32_t ut[ORACLE_MAX_CAND];
+            float uw[ORACLE_MAX_CAND];
+            int nu = 0;
+            for (int c = 0; c < nc; ++c) {
+                int m = 0;
+                while (m < nu && ut[m] != cand_t[c]) ++m;
+                if (m == nu) {
+                    ut[nu] = cand_t[c];
+                    uw[nu] = cand_u[c];
+                    ++nu;
+                } else {
+                    uw[m] = uw[m] + cand_u[c];
+                }
+            }
+            for (int x = 1; x < nu; ++x) {
+                const int32_t tt = ut[x];
+                const float ww = uw[x];
+                int y = x - 1;
+                while (y >= 0 && (uw[y] < ww || (uw[y] == ww && ut[y] > tt))) {
+                    ut[y + 1] = ut[y];
+                    uw[y + 1] = uw[y];
+                    --y;
+                }
+                ut[y + 1] = tt;
+                uw[y + 1] = ww;
+            }
+            /* backward through the kept merged weights */
+            const int kept = nu < s1 ? nu : s1;
+            for (int r = 0; r < kept; ++r) {
+                double g = (double)gout[row * s1 + r];
+                if (grad_is_log) g /= (double)uw[r];
+                for (int c = 0; c < nc; ++c) {
+                    if (cand_t[c] != ut[r]) continue;
+                    const int a = cand_a[c];
+                    dw1[row * s2 + a] += g * (double)a2_w[cand_r2[c]];
+                    dw2[cand_r2[c]] += g * (double)a1_w[row * s2 + a];
+                }
+            }
         }
     }
     return bad;
