@@ -10,7 +10,8 @@
  *   - sparse edge attention (SEA): K/V gathered at each position's edge indices per KV head,
  *     shared by the query heads of the GQA group, score = scale * q.k + ln w, softmax over
  *     the entries, weighted sum of V;
- *   - the SEA backward pass.
+ *   - the backward passes of both (SEA: dq, dk, dv, d ln w; SER: gradients of the kept
+ *     referral weights with respect to both legs' weights).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -92,6 +93,36 @@ gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
                          const int32_t *a2_idx, const float *a2_w, int s3,
                          int32_t *out_idx, float *out_w, int s1,
                          int B, int n, int k, cudaStream_t stream);
+
+/*
+ * gm_ser_backward - gradients of gm_ser_forward's kept weights with respect to both legs'
+ * weights.
+ * Source: ai.info summary, "Methodology in Plain English", referral paragraph (hard top-s
+ * selection; only retained weights get gradients; indices get none).
+ *
+ * The referral of every row is recomputed exactly as gm_ser_forward computes it (same
+ * candidates, merge and selection). For every candidate c = (a, e) of row (b,i,h) whose
+ * target was kept in output slot r with weight W_r > 0, and g_r = gout[b,i,h,r] (divided by
+ * W_r when grad_is_log = 1, i.e. when gout is the gradient with respect to ln A'.w, as
+ * gm_sea_backward's dlogw is):
+ *   dw1[b,i,h,a]  += g_r * a2_w[b,j,h,e]      (j = a1_idx[b,i,h,a])
+ *   dw2[b,j,h,e]  += g_r * a1_w[b,i,h,a]      (summed over every row that reaches it)
+ * Candidates cut by the top-s1 get nothing. fp32 throughout; dw1 is summed in a fixed order,
+ * dw2 with fp32 atomics (order varies run to run).
+ *
+ *   a1_idx/a1_w, a2_idx/a2_w, s1   as gm_ser_forward (k edge channels)
+ *   gout        device fp32 [B, n, k, s1]
+ *   grad_is_log 0: gout is dL/dA'.w; 1: gout is dL/d ln A'.w
+ *   dw1         device fp32 [B, n, k, s2], written (added to if accumulate)
+ *   dw2         device fp32 [B, n, k, s3], zeroed by a library kernel then scatter-added
+ *               (added to without zeroing if accumulate)
+ *   limits      as gm_ser_forward
+ */
+gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                          const int32_t *a2_idx, const float *a2_w, int s3,
+                          const float *gout, int s1, int grad_is_log,
+                          int B, int n, int k, float *dw1, float *dw2, int accumulate,
+                          cudaStream_t stream);
 
 /*
  * gm_sea_forward - sparse edge attention.

@@ -7,6 +7,7 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_sea_forward      sparse edge attention
     gm_ser_sea_forward  both in one kernel
     gm_sea_backward     gradients of sparse edge attention
+    gm_ser_backward     gradients of the kept referral weights
 """
 from ._binding import (  # noqa: F401
     GM_BF16,
@@ -19,6 +20,7 @@ from ._binding import (  # noqa: F401
     gm_sea_backward_noalloc,
     gm_sea_backward_workspace_size,
     gm_sea_forward,
+    gm_ser_backward,
     gm_ser_forward,
     gm_ser_sea_forward,
     gm_version,

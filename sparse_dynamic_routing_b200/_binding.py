@@ -25,6 +25,8 @@ GM_F32, GM_BF16 = 0, 1
 _vp, _ci, _cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "gm_ser_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
+    "gm_ser_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _vp, _vp, _ci,
+                        _vp],
     "gm_sea_forward": [_vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp,
                        _vp],
     "gm_ser_sea_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _vp, _ci, _ci,
@@ -135,6 +137,28 @@ def gm_ser_forward(a1_idx, a1_w, a2_idx, a2_w, s1: int, out_idx=None, out_w=None
         B, n, k, _stream(stream))
     _check(st, "gm_ser_forward")
     return out_idx, out_w
+
+
+def gm_ser_backward(a1_idx, a1_w, a2_idx, a2_w, gout, grad_is_log=False, dw1=None, dw2=None,
+                    accumulate=False, stream=None):
+    """Gradients of the kept referral weights w.r.t. both legs' weights. Returns (dw1, dw2)."""
+    B, n, k, s2 = a1_idx.shape
+    s3, s1 = a2_idx.shape[3], gout.shape[3]
+    if a2_idx.shape[:3] != (B, n, k) or gout.shape[:3] != (B, n, k):
+        raise ValueError("edge tensor shapes disagree")
+    if a1_w.shape != a1_idx.shape or a2_w.shape != a2_idx.shape:
+        raise ValueError("edge weight shapes disagree with their indices")
+    dev = a1_idx.device
+    f32 = torch.float32
+    dw1 = torch.empty((B, n, k, s2), dtype=f32, device=dev) if dw1 is None else dw1
+    dw2 = torch.empty((B, n, k, s3), dtype=f32, device=dev) if dw2 is None else dw2
+    st = load_library().gm_ser_backward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, torch.int32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3,
+        _ptr(gout, f32, "gout"), s1, int(bool(grad_is_log)), B, n, k,
+        _ptr(dw1, f32, "dw1"), _ptr(dw2, f32, "dw2"), int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_ser_backward")
+    return dw1, dw2
 
 
 def gm_sea_forward(q, k, v, idx, w, scale=None, o=None, lse=None, want_lse=True, stream=None):

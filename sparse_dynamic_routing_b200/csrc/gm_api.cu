@@ -12,6 +12,7 @@
 #include "gm_sea.cuh"
 #include "gm_sea_bwd.cuh"
 #include "gm_ser.cuh"
+#include "gm_ser_bwd.cuh"
 
 namespace {
 
@@ -127,8 +128,12 @@ unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int
 #ifndef GM_WPB_BWD_TILE
 #define GM_WPB_BWD_TILE 4
 #endif
+#ifndef GM_TILE_CPL
+#define GM_TILE_CPL 1
+#endif
 constexpr int TILE_P = GM_TILE_P;  // passes of copies in flight per warp
 constexpr int WPB_TILE = GM_WPB_TILE;
+constexpr int TILE_CPL = GM_TILE_CPL;  // 16-byte chunks of a feature row per lane
 
 // Shapes the tiled forward covers: 2..16 lanes per feature row, at most 16 fp32 values of
 // q per lane for the whole group, head_dim 64 or 128.
@@ -140,8 +145,8 @@ template <typename T, int D, int G> struct TileOK {
 template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M>
 gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
 {
-    using TG = gm::TileGeom<T, D, G, S1M>;
-    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE>;
+    using TG = gm::TileGeom<T, D, G, S1M, TILE_CPL>;
+    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL>;
     const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -353,6 +358,27 @@ gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k,
               (uint32_t)((int64_t)B * n * k), row_map(k, n)};
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
+    return launched();
+}
+
+gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                          const int32_t *a2_idx, const float *a2_w, int s3,
+                          const float *gout, int s1, int grad_is_log,
+                          int B, int n, int k, float *dw1, float *dw2, int accumulate,
+                          cudaStream_t stream)
+{
+    if ((grad_is_log != 0 && grad_is_log != 1) || (accumulate != 0 && accumulate != 1)) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, k);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!gout || !dw1 || !dw2) return GM_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * n * k;
+    if (!accumulate) {
+        gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dw2), rows * s3);
+        if (launched() != GM_OK) return GM_ERR_CUDA;
+    }
+    const SerArgs f{a1_idx, a1_w, a2_idx, a2_w, nullptr, nullptr, s1, s2, s3, n, k, (uint32_t)rows, row_map(k, n)};
+    const gm::SerBwdArgs b{f, gout, grad_is_log, dw1, dw2, accumulate};
+    gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
     return launched();
 }
 

@@ -229,118 +229,96 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
     }
     if (p0 >= total) return;  // warp-uniform
 
-    // the chunk's records
-    const int kend = (int)min((int64_t)32, (int64_t)total - p0);
-    const bool in = lane < kend;
+    // the chunk's records (window [wbase, wbase + 32) of the sorted list, one per lane)
+    int64_t wbase = p0;
+    int wlen = (int)min((int64_t)32, (int64_t)total - wbase);
     int32_t mkey = -1, mrow = 0;
     float mcf[2 * G];
+    auto load_window = [&]() {
+        mkey = -1;
+        mrow = 0;
 #pragma unroll
-    for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
-    if (in) read_record<G>(ws.srec, p0 + lane, mkey, mrow, mcf);
+        for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
+        if (lane < wlen) read_record<G>(ws.srec, wbase + lane, mkey, mrow, mcf);
+    };
+    load_window();
     const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
 
     // a leading run that continues the previous chunk's last target belongs to that chunk
-    const int start = __popc(__ballot_sync(FULL, in && mkey == prev_key));
-    if (start == kend) return;  // warp-uniform
-
-    auto issue = [&](int grp) {  // group grp of the window: records start + grp*U ...
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = start + grp * U + u;
-            const int32_t row = __shfl_sync(FULL, mrow, k & 31);
-            if (k < kend && working) {
-                char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-                    cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
-            }
-        }
-        cp_async_commit();
-    };
+    const int start = __popc(__ballot_sync(FULL, lane < wlen && mkey == prev_key));
+    if (start == wlen) return;  // warp-uniform
 
     uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, start);
     zero_rows((int64_t)prev_key + 1, cur);
-    const int ngroups = (kend - start + U - 1) / U;
-#pragma unroll
-    for (int grp = 0; grp < P; ++grp) issue(grp);
-    for (int grp = 0; grp < ngroups; ++grp) {
-        cp_async_wait<P - 1>();
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int k = start + grp * U + u;
-            const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
-            float cf[2 * G];
-#pragma unroll
-            for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
-            if (k >= kend) break;  // warp-uniform
-            if (key != cur) {      // warp-uniform: a new target starts here
-                write_row(cur);
-#pragma unroll
-                for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
-                zero_rows((int64_t)cur + 1, key);
-                cur = key;
-            }
-            if (working) {
-                const char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float f[VEC];
-                    unpack<T>(*reinterpret_cast<const uint4 *>(slot + g * 32 * 16), f);
-                    const float k2 = role == 0 ? cf[g] : cf[G + g];
-                    const float2 kk = make_float2(k2, k2);
-#pragma unroll
-                    for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
-                }
-            }
-        }
-        issue(grp + P);
-    }
-    cp_async_wait<0>();
 
-    // the last owned target may continue past the chunk: follow it (rare, hot rows)
-    int64_t pos = p0 + kend;
-    while (pos < total) {
-        const int64_t left = (int64_t)total - pos;
-        const bool in2 = lane < left;
-        int32_t key2 = -1, row2 = 0;
-        float cf2[2 * G];
-#pragma unroll
-        for (int x = 0; x < 2 * G; ++x) cf2[x] = 0.0f;
-        if (in2) read_record<G>(ws.srec, pos + lane, key2, row2, cf2);
-        const int run = __popc(__ballot_sync(FULL, in2 && (uint32_t)key2 == cur));
-        if (run == 0) break;  // warp-uniform
-        for (int k0 = 0; k0 < run; k0 += U) {
-            uint4 raw[U][G];
-            float cf[U][2 * G];
+    // Accumulate records [lo, hi) of the current window, U per copy group, P groups in
+    // flight; a change of key writes the finished target (and zeroes any empty rows between).
+    auto process = [&](int lo, int hi) {
+        auto issue = [&](int grp) {
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int k = k0 + u;
-                const int32_t row = __shfl_sync(FULL, row2, k & 31);
+                const int k = lo + grp * U + u;
+                const int32_t row = __shfl_sync(FULL, mrow, k & 31);
+                if (k < hi && working) {
+                    char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
 #pragma unroll
-                for (int x = 0; x < 2 * G; ++x) cf[u][x] = __shfl_sync(FULL, cf2[x], k & 31);
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    raw[u][g] = make_uint4(0, 0, 0, 0);
-                    if (k < run && working)
-                        raw[u][g] = ld16(src + ((size_t)row * G + g) * ROW + c * 16);
+                    for (int g = 0; g < G; ++g)
+                        cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
                 }
             }
+            cp_async_commit();
+        };
+        const int ngroups = (hi - lo + U - 1) / U;
+#pragma unroll
+        for (int grp = 0; grp < P; ++grp) issue(grp);
+        for (int grp = 0; grp < ngroups; ++grp) {
+            cp_async_wait<P - 1>();
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                if (k0 + u >= run || !working) continue;
+                const int k = lo + grp * U + u;
+                const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
+                float cf[2 * G];
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    float f[VEC];
-                    unpack<T>(raw[u][g], f);
-                    const float k2 = role == 0 ? cf[u][g] : cf[u][G + g];
-                    const float2 kk = make_float2(k2, k2);
+                for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
+                if (k >= hi) break;  // warp-uniform
+                if (key != cur) {    // warp-uniform: a new target starts here
+                    write_row(cur);
 #pragma unroll
-                    for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+                    for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
+                    zero_rows((int64_t)cur + 1, key);
+                    cur = key;
+                }
+                if (working) {
+                    const char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        float f[VEC];
+                        unpack<T>(*reinterpret_cast<const uint4 *>(slot + g * 32 * 16), f);
+                        const float k2 = role == 0 ? cf[g] : cf[G + g];
+                        const float2 kk = make_float2(k2, k2);
+#pragma unroll
+                        for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+                    }
                 }
             }
+            issue(grp + P);
         }
-        pos += run;
-        if (run < 32) break;  // the target ended inside this window
+        cp_async_wait<0>();
+    };
+
+    process(start, wlen);
+    // the last owned target may continue past the chunk (hot rows): follow it window by
+    // window with the same pipeline
+    int64_t pos = wbase + wlen;
+    while (wlen == 32 && pos < total) {
+        wbase = pos;
+        wlen = (int)min((int64_t)32, (int64_t)total - wbase);
+        load_window();
+        const int run = __popc(__ballot_sync(FULL, lane < wlen && (uint32_t)mkey == cur));
+        if (run == 0) break;  // warp-uniform
+        process(0, run);
+        pos = wbase + run;
+        if (run < wlen) break;  // the target ended inside this window
     }
     write_row(cur);
     if (pos >= total) zero_rows((int64_t)cur + 1, R);  // owner of the last target: trailing rows

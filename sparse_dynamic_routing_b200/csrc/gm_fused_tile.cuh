@@ -141,9 +141,9 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
-template <typename T, int D, int G, int S1M> struct TileGeom {
+template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static constexpr int VEC = Vec<T>::N;          // elements per 16-byte chunk
-    static constexpr int C = D / VEC;              // lanes per row
+    static constexpr int C = D / (VEC * CPL);      // lanes per row (CPL chunks per lane)
     static constexpr int RPW = 32 / C;             // rows per warp pass
     static constexpr int NPASS = 32 / RPW;         // passes per 32-row tile
     static constexpr int ROW = D * (int)sizeof(T); // bytes per feature row
@@ -156,11 +156,11 @@ template <typename T, int D, int G, int S1M> struct TileGeom {
 
 // REFER = true: fused SER -> SEA (edges from the referral of sa's legs);
 // REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
-template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB>
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL>
 __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
-    using TG = TileGeom<T, D, G, S1M>;
-    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS;
+    using TG = TileGeom<T, D, G, S1M, CPL>;
+    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
     static_assert(VEC % 2 == 0, "packed fp32x2 math");
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -246,14 +246,20 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                     a.map.split(row, seq_base, h);
                     const char *qs = reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW);
 #pragma unroll
-                    for (int g = 0; g < G; ++g) cp_async16(st + TG::RQ + g * TG::ROW + c * 16, qs + g * TG::ROW + c * 16);
+                    for (int g = 0; g < G; ++g)
+#pragma unroll
+                        for (int cc = 0; cc < CPL; ++cc)
+                            cp_async16(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16, qs + g * TG::ROW + (c * CPL + cc) * 16);
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
                             const uint32_t kvrow = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
-                            const size_t off = (size_t)kvrow * TG::ROW + c * 16;
-                            cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
-                            cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
+#pragma unroll
+                            for (int cc = 0; cc < CPL; ++cc) {
+                                const size_t off = (size_t)kvrow * TG::ROW + (c * CPL + cc) * 16;
+                                cp_async16(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16, static_cast<const char *>(a.k) + off);
+                                cp_async16(st + TG::RV + jj * TG::ROW + (c * CPL + cc) * 16, static_cast<const char *>(a.v) + off);
+                            }
                         }
                     }
                 }
@@ -278,30 +284,39 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 act[jj] = valid && lw[jj] != -INFINITY;
             }
             // q chunks of the G heads as fp32 pairs
-            float2 q2[G][VEC / 2];
+            float2 q2[G][CPL * NP];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
-                float f[VEC];
-                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16)
-                                : make_uint4(0, 0, 0, 0), f);
 #pragma unroll
-                for (int x = 0; x < VEC / 2; ++x) q2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
+                for (int cc = 0; cc < CPL; ++cc) {
+                    float f[VEC];
+                    unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16)
+                                    : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                    for (int x = 0; x < NP; ++x) q2[g][cc * NP + x] = make_float2(f[2 * x], f[2 * x + 1]);
+                }
             }
             // scores (all S1M slots, masked after the reduction so shuffles stay uniform)
             float z[G][S1M];
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
-                float kf[VEC];
-                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16)
-                                  : make_uint4(0, 0, 0, 0), kf);
+                float kf[CPL * VEC];
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    float f[VEC];
+                    unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16)
+                                      : make_uint4(0, 0, 0, 0), f);
+#pragma unroll
+                    for (int x = 0; x < VEC; ++x) kf[cc * VEC + x] = f[x];
+                }
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float dot = seg_sum<C>(chunk_dot<VEC / 2>(q2[g], kf));
+                    const float dot = seg_sum<C>(chunk_dot<CPL * NP>(q2[g], kf));
                     z[g][jj] = act[jj] ? fmaf(dot, sl2, lw[jj]) : -INFINITY;
                 }
             }
             // softmax and weighted V per head
-            float2 acc[G][VEC / 2];
+            float2 acc[G][CPL * NP];
             float m[G], l[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -310,20 +325,26 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 for (int jj = 1; jj < S1M; ++jj) m[g] = fmaxf(m[g], z[g][jj]);
                 l[g] = 0.0f;
 #pragma unroll
-                for (int x = 0; x < VEC / 2; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
+                for (int x = 0; x < CPL * NP; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
             }
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
                 if (!act[jj]) continue;  // per lane; no shuffles below
-                float vf[VEC];
-                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
+                float vf[CPL * VEC];
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) {
+                    float f[VEC];
+                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + (c * CPL + cc) * 16), f);
+#pragma unroll
+                    for (int x = 0; x < VEC; ++x) vf[cc * VEC + x] = f[x];
+                }
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
                     const float p = ex2(z[g][jj] - m[g]);
                     l[g] += p;
                     const float2 p2 = make_float2(p, p);
 #pragma unroll
-                    for (int x = 0; x < VEC / 2; ++x)
+                    for (int x = 0; x < CPL * NP; ++x)
                         acc[g][x] = __ffma2_rn(p2, make_float2(vf[2 * x], vf[2 * x + 1]), acc[g][x]);
                 }
             }
@@ -332,13 +353,16 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 for (int g = 0; g < G; ++g) {
                     const bool nonempty = l[g] > 0.0f;
                     const float inv = nonempty ? __frcp_rn(l[g]) : 0.0f;
-                    float of[VEC];
 #pragma unroll
-                    for (int x = 0; x < VEC / 2; ++x) {
-                        of[2 * x] = acc[g][x].x * inv;
-                        of[2 * x + 1] = acc[g][x].y * inv;
+                    for (int cc = 0; cc < CPL; ++cc) {
+                        float of[VEC];
+#pragma unroll
+                        for (int x = 0; x < NP; ++x) {
+                            of[2 * x] = acc[g][cc * NP + x].x * inv;
+                            of[2 * x + 1] = acc[g][cc * NP + x].y * inv;
+                        }
+                        *reinterpret_cast<uint4 *>(O + ((size_t)row * G + g) * D + (c * CPL + cc) * VEC) = pack<T>(of);
                     }
-                    *reinterpret_cast<uint4 *>(O + ((size_t)row * G + g) * D + c * VEC) = pack<T>(of);
                     if (a.lse != nullptr && c == 0)
                         a.lse[(size_t)row * G + g] = nonempty ? (m[g] + lg2(l[g])) * LN2 : -INFINITY;
                 }

@@ -319,3 +319,80 @@ def test_out_of_range_index_is_skipped_and_flagged():
     with pytest.raises(gm.GMIndexRangeError):
         gm.gm_check_device_errors()
     assert_ser_equal(gi, gw, oi, ow)
+
+
+# ---- SER backward -------------------------------------------------------------------------------
+
+
+def assert_rel(got, want, what, rtol=1e-5):
+    """fp32 sums of a few products per entry: relative error bounded by a few ulps of the
+    largest term; atol scales with the largest magnitude."""
+    got = host(got).double().numpy().reshape(want.shape)
+    scale = max(float(np.abs(want).max()), 1e-30)
+    err = np.abs(got - want)
+    bad = err > rtol * np.abs(want) + rtol * scale
+    assert not bad.any(), f"{what}: max error {err.max():.3g} (scale {scale:.3g})"
+
+
+@pytest.mark.parametrize("s2,s3,s1,n", [(2, 2, 2, 128), (4, 4, 4, 300), (4, 4, 2, 97),
+                                        (3, 5, 7, 61), (8, 4, 32, 40), (1, 1, 1, 33)])
+def test_ser_backward_shapes(s2, s3, s1, n):
+    rng = np.random.default_rng(s2 * 100 + s3 * 10 + s1)
+    B, k = 2, 3
+
+    def legs(s):
+        hi = np.broadcast_to(np.arange(1, n + 1)[None, :, None, None], (B, n, k, s))
+        idx = rng.integers(0, hi).astype(np.int32)
+        w = rng.dirichlet(np.ones(s) * 0.7, (B, n, k)).astype(np.float32)
+        w[rng.random(w.shape) < 0.1] = 0.0
+        return idx, w
+
+    i1, w1 = legs(s2)
+    i2, w2 = legs(s3)
+    g = rng.standard_normal((B, n, k, s1)).astype(np.float32)
+    want1, want2, _ = oracle.ser_backward(i1, w1, i2, w2, g)
+    t = lambda a: torch.from_numpy(a).cuda()  # noqa: E731
+    d1, d2 = gm.gm_ser_backward(t(i1), t(w1), t(i2), t(w2), t(g))
+    assert_rel(d1, want1, "dw1")
+    assert_rel(d2, want2, "dw2")
+    # accumulate adds onto the buffers
+    gm.gm_ser_backward(t(i1), t(w1), t(i2), t(w2), t(g), dw1=d1, dw2=d2, accumulate=True)
+    assert_rel(d1, 2 * want1, "2 dw1")
+    assert_rel(d2, 2 * want2, "2 dw2")
+    gm.gm_check_device_errors()
+
+
+def test_ser_backward_full_size_layer():
+    wl = I.WORKLOADS["layer_b8_n4096_s4_local"]
+    x = I.make(wl)
+    rng = np.random.default_rng(77)
+    g = rng.standard_normal((wl.B, wl.n, wl.hkv, wl.s1)).astype(np.float32)
+    want1, want2, _ = oracle.ser_backward(x["a1_idx"], x["a1_w"], x["a2_idx"], x["a2_w"], g)
+    d1, d2 = gm.gm_ser_backward(x["a1_idx"].cuda(), x["a1_w"].cuda(), x["a2_idx"].cuda(),
+                                x["a2_w"].cuda(), torch.from_numpy(g).cuda())
+    assert_rel(d1, want1, "dw1")
+    assert_rel(d2, want2, "dw2", rtol=1e-4)  # up to thousands of fp32 atomic terms per entry
+    gm.gm_check_device_errors()
+
+
+def test_training_chain_through_both_backwards_f32():
+    # forward SER -> SEA, backward SEA -> d ln w -> SER backward, against the oracle's chain
+    wl = I.WORKLOADS["tiny_b1_n128_s2_f32"]
+    x = I.make(wl, grad=True)
+    oi, ow, _ = oracle.ser(x["a1_idx"], x["a1_w"], x["a2_idx"], x["a2_w"], wl.s1)
+    _, _, _, dlw_ref, _ = oracle.sea_backward(x["q"], x["k"], x["v"], x["dout"], oi, ow, wl.scale)
+    want1, want2, _ = oracle.ser_backward(x["a1_idx"], x["a1_w"], x["a2_idx"], x["a2_w"],
+                                          dlw_ref.astype(np.float32), grad_is_log=True)
+    g = cuda(x)
+    ai, aw, _, _ = gm.gm_ser_sea_forward(g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"],
+                                         g["a2_idx"], g["a2_w"], wl.s1, wl.scale)
+    _, _, _, dlw = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], ai, aw, wl.scale)
+    d1, d2 = gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"], dlw,
+                                grad_is_log=True)
+    assert_rel(d1, want1, "dw1", rtol=1e-3)
+    assert_rel(d2, want2, "dw2", rtol=1e-3)
+    # d ln w / W through the flag equals dividing first
+    e1, e2 = gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"],
+                                torch.where(aw > 0, dlw / aw, torch.zeros_like(dlw)))
+    assert torch.allclose(d1, e1, rtol=1e-6, atol=1e-6) and torch.allclose(d2, e2, rtol=1e-6, atol=1e-6)
+    gm.gm_check_device_errors()
