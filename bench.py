@@ -236,7 +236,7 @@ def ncu_traffic(kernel: str, workload: str):
         if line.startswith("#") or not line.strip():
             continue
         f = dict(kv.split("=", 1) for kv in line.split())
-        if f.get("kernel") == kernel and f.get("workload") == workload:
+        if f.get("kernel") == kernel.replace(" ", "_") and f.get("workload") == workload:
             if f.get("source") != cur:
                 return None
             return float(f["dram_bytes_per_launch"])
@@ -329,7 +329,7 @@ def run_ours(args):
         if ev is not None:
             ev[2].record(stream)
 
-    # fused forward; backward = counter zero-fill, row pass, three scan passes, bucket fill,
+    # fused forward; backward = counter zero-fill, count pass, three scan passes, row pass,
     # gather (with a workspace) or zero-fill + scatter row pass (without)
     launches_per_step = 1 + (7 if ws is not None else 2)
 
@@ -371,7 +371,7 @@ def run_ours(args):
     calls = {
         "fused_forward": {"kernel": "sea_fwd_tile_kernel (fused SER->SEA)", "us": fwd_ms * 1e3,
                           "bytes": cb["fused_forward"]},
-        "backward": {"kernel": "gm_sea_backward (row pass + scan + bucket fill + gather)"
+        "backward": {"kernel": "gm_sea_backward (count + scan + row pass + gather)"
                      if ws is not None else "gm_sea_backward (zero-fill + scatter row pass)",
                      "us": bwd_ms * 1e3, "bytes": cb["backward"]},
     }
