@@ -229,7 +229,7 @@ template <typename T, int D, int G> struct SeaBwd {
 #define GM_GATHER_P 3
 #endif
 #ifndef GM_WPB_GATHER
-#define GM_WPB_GATHER 4
+#define GM_WPB_GATHER 2
 #endif
 constexpr int WPB_GATHER = GM_WPB_GATHER;
 constexpr int GATHER_U = GM_GATHER_U;  // records per copy group

@@ -132,12 +132,12 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 float f[VEC];
-                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16)
-                                : make_uint4(0, 0, 0, 0), f);
+                // an invalid row (ragged tail) computes on whatever the stage holds and stores
+                // nothing
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16), f);
 #pragma unroll
                 for (int x = 0; x < NP; ++x) q2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
-                unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RG + g * TG::ROW + c * 16)
-                                : make_uint4(0, 0, 0, 0), f);
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RG + g * TG::ROW + c * 16), f);
 #pragma unroll
                 for (int x = 0; x < NP; ++x) g2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
             }
@@ -146,16 +146,14 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
                 float kf[VEC], vf[VEC];
-                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16)
-                                  : make_uint4(0, 0, 0, 0), kf);
-                unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16)
-                                  : make_uint4(0, 0, 0, 0), vf);
+                // an inactive slot's stage holds stale data: its score and dO.V are masked below
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
+                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float sk = seg_sum<C>(chunk_dot<NP>(q2[g], kf));
-                    const float sv = seg_sum<C>(chunk_dot<NP>(g2[g], vf));
-                    z[g][jj] = act[jj] ? fmaf(sk, sl2, lw[jj]) : -INFINITY;
-                    dp[g][jj] = sv;
+                for (int g = 0; g < G; ++g) {  // q.k and dO.v reduced together (packed adds)
+                    const float2 r = seg_sum2<C>(make_float2(chunk_dot<NP>(q2[g], kf), chunk_dot<NP>(g2[g], vf)));
+                    z[g][jj] = act[jj] ? fmaf(r.x, sl2, lw[jj]) : -INFINITY;
+                    dp[g][jj] = act[jj] ? r.y : 0.0f;
                 }
             }
             // softmax, D, dz

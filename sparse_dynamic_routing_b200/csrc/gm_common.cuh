@@ -180,6 +180,17 @@ template <int C> __device__ __forceinline__ float seg_sum(float x)
     return x;
 }
 
+// seg_sum of two values at once (packed fp32x2 add per step).
+template <int C> __device__ __forceinline__ float2 seg_sum2(float2 x)
+{
+#pragma unroll
+    for (int off = C / 2; off > 0; off >>= 1) {
+        const float2 y = make_float2(__shfl_xor_sync(FULL, x.x, off), __shfl_xor_sync(FULL, x.y, off));
+        x = __fadd2_rn(x, y);
+    }
+    return x;
+}
+
 // Sum across the RPI segments that share a chunk index (lanes c, c + C, c + 2C, ...).
 template <int C> __device__ __forceinline__ float cross_seg_sum(float x)
 {

@@ -290,8 +290,9 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) {
                     float f[VEC];
-                    unpack<T>(valid ? *reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16)
-                                    : make_uint4(0, 0, 0, 0), f);
+                    // an invalid row (ragged tail) computes on whatever the stage holds and
+                    // stores nothing
+                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16), f);
 #pragma unroll
                     for (int x = 0; x < NP; ++x) q2[g][cc * NP + x] = make_float2(f[2 * x], f[2 * x + 1]);
                 }
@@ -304,15 +305,23 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) {
                     float f[VEC];
-                    unpack<T>(act[jj] ? *reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16)
-                                      : make_uint4(0, 0, 0, 0), f);
+                    // an inactive slot's stage holds stale data: its score is masked below
+                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16), f);
 #pragma unroll
                     for (int x = 0; x < VEC; ++x) kf[cc * VEC + x] = f[x];
                 }
+                // the heads' partial dots are reduced two at a time (packed adds)
 #pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float dot = seg_sum<C>(chunk_dot<CPL * NP>(q2[g], kf));
-                    z[g][jj] = act[jj] ? fmaf(dot, sl2, lw[jj]) : -INFINITY;
+                for (int g = 0; g < G; g += 2) {
+                    if (g + 1 < G) {
+                        const float2 d2 = seg_sum2<C>(make_float2(chunk_dot<CPL * NP>(q2[g], kf),
+                                                                  chunk_dot<CPL * NP>(q2[g + 1], kf)));
+                        z[g][jj] = act[jj] ? fmaf(d2.x, sl2, lw[jj]) : -INFINITY;
+                        z[g + 1][jj] = act[jj] ? fmaf(d2.y, sl2, lw[jj]) : -INFINITY;
+                    } else {
+                        const float dot = seg_sum<C>(chunk_dot<CPL * NP>(q2[g], kf));
+                        z[g][jj] = act[jj] ? fmaf(dot, sl2, lw[jj]) : -INFINITY;
+                    }
                 }
             }
             // softmax and weighted V per head
