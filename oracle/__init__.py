@@ -1,4 +1,4 @@
-"""CPU oracle of the Graph Machine sparse layer (SER and its backward, SEA and its backward).
+"""CPU oracle of the Graph Machine sparse layer (leg sparsification, SER, SEA, and their backward passes).
 
 TEST INFRASTRUCTURE. Only the tests, the package smoke check and the benchmark's CPU-baseline
 leg import this module. It wraps the plain C library built from gm_oracle.c (compiled on
@@ -42,6 +42,12 @@ def _load():
         lib.oracle_sea_backward.restype = ctypes.c_int64
         lib.oracle_sea_backward.argtypes = [f32p, f32p, f32p, f32p, i32p, f32p, ci, ci, ci, ci,
                                             ci, ci, ctypes.c_double, f64p, f64p, f64p, f64p]
+        lib.oracle_leg_sparsify.restype = ctypes.c_int64
+        lib.oracle_leg_sparsify.argtypes = [i32p, f32p, ci, ci, f32p, f32p, ctypes.c_int64,
+                                            i32p, f32p, ci, i32p, f32p, ci, ci, ci]
+        lib.oracle_leg_backward.restype = ctypes.c_int64
+        lib.oracle_leg_backward.argtypes = [i32p, f32p, ci, ci, f32p, f32p, ctypes.c_int64,
+                                            f32p, ci, f32p, ci, ci, ci, f64p, f64p, f64p]
         _lib = lib
     return _lib
 
@@ -147,3 +153,59 @@ def ser_sea_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, s1: int, scale=None, ro
     oi, ow, bad1 = ser(a1_idx, a1_w, a2_idx, a2_w, s1)
     o, lse, bad2 = sea_forward(q, k, v, oi, ow, scale, rows)
     return oi, ow, o, lse, bad1 + bad2
+
+
+def _mix(m, B, n, k):
+    """Mixing coefficients [B, n, k, k] (per token) or [k, k] (shared) -> (array, token stride)."""
+    m = _np(m, np.float32)
+    if m.shape == (k, k):
+        return m, 0
+    assert m.shape == (B, n, k, k), m.shape
+    return m, k * k
+
+
+def leg_sparsify(e_idx, e_w, mix1, mix2, s2: int, s3: int):
+    """The pair of legs of every (b, i, h) from the stored edges E [B, n, k, s0].
+
+    Leg 1 = Sparsify_s2 of the stored edges of the same token mixed by mix1[.., h, :], leg 2
+    the same with mix2 and s3. Returns (a1_idx, a1_w, a2_idx, a2_w, bad_refs).
+    """
+    ei, ew = _np(e_idx, np.int32), _np(e_w, np.float32)
+    B, n, k, s0 = ei.shape
+    assert ew.shape == ei.shape
+    m1, st1 = _mix(mix1, B, n, k)
+    m2, st2 = _mix(mix2, B, n, k)
+    assert st1 == st2, "both legs' coefficients must be per token, or both shared"
+    a1i = np.zeros((B, n, k, s2), np.int32)
+    a1w = np.zeros((B, n, k, s2), np.float32)
+    a2i = np.zeros((B, n, k, s3), np.int32)
+    a2w = np.zeros((B, n, k, s3), np.float32)
+    bad = _load().oracle_leg_sparsify(ei, ew, s0, k, m1, m2, st1, a1i, a1w, s2, a2i, a2w, s3,
+                                      B, n)
+    if bad < 0:
+        raise ValueError("k*s0 exceeds the oracle's candidate buffer")
+    return a1i, a1w, a2i, a2w, int(bad)
+
+
+def leg_backward(e_idx, e_w, mix1, mix2, g1, g2):
+    """Gradients of the kept leg weights w.r.t. the stored weights and both mixes (fp64).
+
+    g1 [B, n, k, s2], g2 [B, n, k, s3]. Returns (dew [B,n,k,s0], dmix1 [B,n,k,k],
+    dmix2 [B,n,k,k], bad_refs); the mixes' gradients are per token even when shared.
+    """
+    ei, ew = _np(e_idx, np.int32), _np(e_w, np.float32)
+    B, n, k, s0 = ei.shape
+    m1, st1 = _mix(mix1, B, n, k)
+    m2, st2 = _mix(mix2, B, n, k)
+    assert st1 == st2
+    ga, gb = _np(g1, np.float32), _np(g2, np.float32)
+    s2, s3 = ga.shape[3], gb.shape[3]
+    assert ga.shape[:3] == (B, n, k) and gb.shape[:3] == (B, n, k)
+    dew = np.zeros(ei.shape, np.float64)
+    dm1 = np.zeros((B, n, k, k), np.float64)
+    dm2 = np.zeros((B, n, k, k), np.float64)
+    bad = _load().oracle_leg_backward(ei, ew, s0, k, m1, m2, st1, ga, s2, gb, s3, B, n,
+                                      dew, dm1, dm2)
+    if bad < 0:
+        raise ValueError("k*s0 exceeds the oracle's candidate buffer")
+    return dew, dm1, dm2, int(bad)

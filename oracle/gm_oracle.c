@@ -24,6 +24,8 @@
  *          = scaled q.k + log(mixed edge weight), no RoPE.
  *   [MPE4] same section, hybrid paragraph: a padding token at the start of each sequence
  *          absorbs underflowing edge indices.
+ *   [MF4]  "Main Findings", bullet on more edges: the cross-edge mixing is full (every stored
+ *          channel feeds every leg channel), so its cost grows as k^2.
  *
  * Readings where the pages are silent (the CUDA library applies the same ones):
  *   R1  A1 and A2 share the edge channel h (leg mixing happens upstream).
@@ -42,6 +44,21 @@
  *       the return value of each entry point.
  *   R9  SER backward: only the kept (top-s1, weight > 0) merged weights carry gradient; the
  *       selection itself is piecewise constant and passes none; indices get none.
+ *   R10 leg mixing: leg L (L = 1, 2) of edge channel h at token (b, i) takes every stored edge
+ *       (c, a) of that token - all k channels c, all s0 slots a - as a candidate with target
+ *       E.idx[b,i,c,a] and weight fl32(M_L[b,i,h,c] * E.w[b,i,c,a]), in ascending c*s0 + a.
+ *       The mixing coefficients M_L >= 0 are inputs (how they are computed from the node
+ *       features is upstream); one [k, k] matrix shared by all tokens is the case of a zero
+ *       token stride.
+ *   R11 each leg is then merged, ordered and cut to its budget (s2 for leg 1, s3 for leg 2)
+ *       exactly as SER's steps (R2-R5): the "sparsify" of both steps is one operation.
+ *   R12 leg backward: as R9, only the kept merged leg weights carry gradient, to both the
+ *       stored weights and the mixing coefficients. Each kept weight is differentiated as the
+ *       sum over the active stored edges that reach its target of coefficient x weight, so an
+ *       active edge whose product was zero (a zero coefficient) still passes the gradient of
+ *       its coefficient: R3's dropping of zero products shapes the forward's candidate set,
+ *       not the derivative. The gradient of the coefficients is returned per token,
+ *       [B, n, k, k], also when they were shared (the caller sums it).
  *
  * Layouts are contiguous row-major: features [B, n, H, d], edges [B, n, k, s].
  */
@@ -410,6 +427,186 @@ int64_t oracle_sea_backward(const float *q, const float *kk, const float *vv, co
         free(t);
         free(slot);
         free(orow);
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Leg sparsification   [MPE2] (the stored edges are mixed into a pair of legs and each leg is
+ * sparsified before the composition), [MF4]; readings R3, R4, R5, R8, R10, R11.
+ *
+ * Shared by the forward and the backward below: merge the candidates of one row by target
+ * (ascending candidate order, fp32 adds) and order the distinct targets by weight descending,
+ * then target ascending. Returns the number of distinct targets.
+ * ---------------------------------------------------------------------------------------- */
+static int merge_and_order(const int32_t *cand_t, const float *cand_u, int nc,
+                           int32_t *ut, float *uw)
+{
+    int nu = 0;
+    for (int c = 0; c < nc; ++c) {
+        int m = 0;
+        while (m < nu && ut[m] != cand_t[c]) ++m;
+        if (m == nu) {
+            ut[nu] = cand_t[c];
+            uw[nu] = cand_u[c];
+            ++nu;
+        } else {
+            uw[m] = uw[m] + cand_u[c];
+        }
+    }
+    for (int x = 1; x < nu; ++x) {
+        const int32_t tt = ut[x];
+        const float ww = uw[x];
+        int y = x - 1;
+        while (y >= 0 && (uw[y] < ww || (uw[y] == ww && ut[y] > tt))) {
+            ut[y + 1] = ut[y];
+            uw[y + 1] = uw[y];
+            --y;
+        }
+        ut[y + 1] = tt;
+        uw[y + 1] = ww;
+    }
+    return nu;
+}
+
+/* Candidates of leg channel h at one token (R10). valid[c*s0+a] says whether stored edge (c, a)
+ * is active and in range; cand_ca receives each candidate's c*s0 + a. Returns their number. */
+static int leg_candidates(const int32_t *e_idx_tok, const float *e_w_tok, const uint8_t *valid,
+                          const float *mix_tok, int h, int k, int s0,
+                          int32_t *cand_t, float *cand_u, int *cand_ca)
+{
+    int nc = 0;
+    for (int c = 0; c < k; ++c) {
+        const float m = mix_tok[h * k + c];
+        for (int a = 0; a < s0; ++a) {
+            const int ca = c * s0 + a;
+            if (!valid[ca]) continue;
+            const float u = m * e_w_tok[ca];          /* one fp32 rounding, as R2 */
+            if (u == 0.0f) continue;                   /* R3 */
+            cand_t[nc] = e_idx_tok[ca];
+            cand_u[nc] = u;
+            cand_ca[nc] = ca;
+            ++nc;
+        }
+    }
+    return nc;
+}
+
+/* Active, in-range stored edges of one token (R3, R8); returns how many active ones were out
+ * of range. */
+static int64_t leg_valid(const int32_t *e_idx_tok, const float *e_w_tok, int ks0, int n,
+                         uint8_t *valid)
+{
+    int64_t bad = 0;
+    for (int ca = 0; ca < ks0; ++ca) {
+        valid[ca] = 0;
+        if (!(e_w_tok[ca] > 0.0f)) continue;
+        if (e_idx_tok[ca] < 0 || e_idx_tok[ca] >= n) { ++bad; continue; }
+        valid[ca] = 1;
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Forward: for every (b, i, h), A1[b,i,h,:] = Sparsify_s2(mix of token i's stored edges by
+ * M1[b,i,h,:]) and A2[b,i,h,:] = Sparsify_s3(the same with M2). E is [B, n, k, s0]; M1 and M2
+ * are [B, n, k, k] read at token offset (b*n + i) * mix_tok_stride (k*k, or 0 for one shared
+ * [k, k] matrix). Returns the number of active stored edges out of range (each counted once).
+ * ---------------------------------------------------------------------------------------- */
+int64_t oracle_leg_sparsify(const int32_t *e_idx, const float *e_w, int s0, int k,
+                            const float *mix1, const float *mix2, int64_t mix_tok_stride,
+                            int32_t *a1_idx, float *a1_w, int s2,
+                            int32_t *a2_idx, float *a2_w, int s3, int B, int n)
+{
+    const int ks0 = k * s0;
+    int64_t bad = 0;
+    if (ks0 > ORACLE_MAX_CAND) return -1;
+
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+    for (int64_t tok = 0; tok < (int64_t)B * n; ++tok) {
+        const int32_t *ei = e_idx + tok * ks0;
+        const float *ew = e_w + tok * ks0;
+        uint8_t valid[ORACLE_MAX_CAND];
+        bad += leg_valid(ei, ew, ks0, n, valid);
+        for (int leg = 0; leg < 2; ++leg) {
+            const float *mix = (leg == 0 ? mix1 : mix2) + tok * mix_tok_stride;
+            const int sl = leg == 0 ? s2 : s3;
+            int32_t *oi = leg == 0 ? a1_idx : a2_idx;
+            float *ow = leg == 0 ? a1_w : a2_w;
+            for (int h = 0; h < k; ++h) {
+                int32_t cand_t[ORACLE_MAX_CAND], ut[ORACLE_MAX_CAND];
+                float cand_u[ORACLE_MAX_CAND], uw[ORACLE_MAX_CAND];
+                int cand_ca[ORACLE_MAX_CAND];
+                const int nc = leg_candidates(ei, ew, valid, mix, h, k, s0, cand_t, cand_u, cand_ca);
+                const int nu = merge_and_order(cand_t, cand_u, nc, ut, uw);
+                const int64_t row = tok * k + h;
+                for (int r = 0; r < sl; ++r) {           /* R4 padding, R5 */
+                    oi[row * sl + r] = r < nu ? ut[r] : 0;
+                    ow[row * sl + r] = r < nu ? uw[r] : 0.0f;
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Backward of the leg sparsification   [MPE2]; readings R10-R12.
+ *
+ * g1 [B, n, k, s2] and g2 [B, n, k, s3]: gradients with respect to the kept leg weights. The
+ * forward's candidates, merge and selection are recomputed; then for every candidate (c, a)
+ * merged into a kept slot r (W_r > 0) of leg L, channel h:
+ *     dew[b,i,c,a]      += g_L[b,i,h,r] * M_L[b,i,h,c]
+ *     dmix_L[b,i,h,c]   += g_L[b,i,h,r] * E.w[b,i,c,a]
+ * in fp64, over every active stored edge (c, a) reaching t_r, including those whose product
+ * was zero (R12). Each token owns its outputs, so tokens run in parallel.
+ * ---------------------------------------------------------------------------------------- */
+int64_t oracle_leg_backward(const int32_t *e_idx, const float *e_w, int s0, int k,
+                            const float *mix1, const float *mix2, int64_t mix_tok_stride,
+                            const float *g1, int s2, const float *g2, int s3, int B, int n,
+                            double *dew, double *dmix1, double *dmix2)
+{
+    const int ks0 = k * s0;
+    int64_t bad = 0;
+    if (ks0 > ORACLE_MAX_CAND) return -1;
+
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+    for (int64_t tok = 0; tok < (int64_t)B * n; ++tok) {
+        const int32_t *ei = e_idx + tok * ks0;
+        const float *ew = e_w + tok * ks0;
+        uint8_t valid[ORACLE_MAX_CAND];
+        bad += leg_valid(ei, ew, ks0, n, valid);
+        for (int ca = 0; ca < ks0; ++ca) dew[tok * ks0 + ca] = 0.0;
+        for (int x = 0; x < k * k; ++x) {
+            dmix1[tok * k * k + x] = 0.0;
+            dmix2[tok * k * k + x] = 0.0;
+        }
+        for (int leg = 0; leg < 2; ++leg) {
+            const float *mix = (leg == 0 ? mix1 : mix2) + tok * mix_tok_stride;
+            const int sl = leg == 0 ? s2 : s3;
+            const float *g = leg == 0 ? g1 : g2;
+            double *dmix = (leg == 0 ? dmix1 : dmix2) + tok * k * k;
+            for (int h = 0; h < k; ++h) {
+                int32_t cand_t[ORACLE_MAX_CAND], ut[ORACLE_MAX_CAND];
+                float cand_u[ORACLE_MAX_CAND], uw[ORACLE_MAX_CAND];
+                int cand_ca[ORACLE_MAX_CAND];
+                const int nc = leg_candidates(ei, ew, valid, mix, h, k, s0, cand_t, cand_u, cand_ca);
+                const int nu = merge_and_order(cand_t, cand_u, nc, ut, uw);
+                const int kept = nu < sl ? nu : sl;
+                const int64_t row = tok * k + h;
+                /* every active stored edge whose target was kept carries the derivative,
+                 * also one whose product with its coefficient was zero (R12) */
+                for (int r = 0; r < kept; ++r) {
+                    const double gr = (double)g[row * sl + r];
+                    for (int ca = 0; ca < ks0; ++ca) {
+                        if (!valid[ca] || ei[ca] != ut[r]) continue;
+                        const int c = ca / s0;
+                        dew[tok * ks0 + ca] += gr * (double)mix[h * k + c];
+                        dmix[h * k + c] += gr * (double)ew[ca];
+                    }
+                }
+            }
+        }
     }
     return bad;
 }

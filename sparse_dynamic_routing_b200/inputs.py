@@ -14,7 +14,12 @@ backbone, 4,096-token packed sequences; "Main Findings": 2 or 4 positions per KV
   token that sits at the start of every packed sequence), optionally mixed with a local
   window {max(0, i - window + 1)..i};
 * edge weights fp32 of shape [B, n, k, s]: one Dirichlet(alpha) draw in fp64 per
-  (b, i, channel) row over its s slots, rounded to fp32.
+  (b, i, channel) row over its s slots, rounded to fp32;
+* for the leg sparsification in front of the referral ("Methodology in Plain English",
+  referral paragraph: the stored edges are mixed into a pair of legs), the stored edges E
+  [B, n, k, s1] drawn as above and two sets of mixing coefficients [B, n, k, k]: one
+  Dirichlet(1) draw in fp64 per (b, i, leg channel) over the k stored channels, rounded to
+  fp32 (non-negative, summing to one, like a softmax over channel logits).
 
 Every stream (q, k, v, dO, indices, weights, and per layer for the stacked workload) has its
 own numpy Generator seeded from (seed, stream id[, layer]), so any one tensor can be redrawn
@@ -28,7 +33,7 @@ import numpy as np
 import torch
 
 # stream ids
-_Q, _K, _V, _DO, _IDX1, _W1, _IDX2, _W2 = range(8)
+_Q, _K, _V, _DO, _IDX1, _W1, _IDX2, _W2, _EIDX, _EW, _MIX1, _MIX2 = range(12)
 
 
 @dataclass(frozen=True)
@@ -170,3 +175,22 @@ def layer_features(wl: Workload, layer: int) -> dict:
         "k": features(wl.seed, _K, (wl.B, wl.n, wl.hkv, wl.d), dt, layer),
         "v": features(wl.seed, _V, (wl.B, wl.n, wl.hkv, wl.d), dt, layer),
     }
+
+
+def mixing(wl: Workload, which: int, layer: int = 0) -> torch.Tensor:
+    """fp32 [B, n, hkv, hkv] mixing coefficients of leg `which` (1 or 2): Dirichlet(1) rows."""
+    rng = _rng(wl.seed, _MIX1 if which == 1 else _MIX2, layer)
+    m = rng.dirichlet(np.ones(wl.hkv, dtype=np.float64), size=(wl.B, wl.n, wl.hkv))
+    return torch.from_numpy(np.ascontiguousarray(m.astype(np.float32)))
+
+
+def leg_inputs(wl: Workload, layer: int = 0) -> dict:
+    """Stored edges e_idx/e_w [B, n, hkv, s1] and mix1/mix2 [B, n, hkv, hkv] (CPU tensors).
+
+    The legs built from them have budgets wl.s2 and wl.s3.
+    """
+    idx = edge_indices(_rng(wl.seed, _EIDX, layer), wl.B, wl.n, wl.hkv, wl.s1,
+                       wl.local_frac, wl.window)
+    w = edge_weights(_rng(wl.seed, _EW, layer), wl.B, wl.n, wl.hkv, wl.s1, wl.alpha)
+    return {"e_idx": torch.from_numpy(idx), "e_w": torch.from_numpy(w),
+            "mix1": mixing(wl, 1, layer), "mix2": mixing(wl, 2, layer)}

@@ -9,6 +9,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 from sparse_dynamic_routing_b200 import inputs as I
 
@@ -86,3 +87,18 @@ def test_streams_are_independent_and_reproducible():
     st = I.WORKLOADS["stack21_b16_n4096_s4"].with_(B=1, n=64)
     l0, l1 = I.layer_features(st, 0), I.layer_features(st, 1)
     assert not np.array_equal(l0["q"].float().numpy(), l1["q"].float().numpy())
+
+
+def test_leg_inputs_recipe():
+    wl = I.WORKLOADS["layer_b8_n4096_s4_local"].with_(B=2, n=256)
+    x = I.leg_inputs(wl)
+    assert x["e_idx"].shape == (2, 256, 8, 4) and x["e_w"].shape == (2, 256, 8, 4)
+    assert x["mix1"].shape == (2, 256, 8, 8) and x["mix1"].dtype == torch.float32
+    i = torch.arange(256)[None, :, None, None]
+    assert bool((x["e_idx"] >= 0).all()) and bool((x["e_idx"] <= i).all())
+    for m in (x["mix1"], x["mix2"]):
+        assert bool((m >= 0).all())
+        assert torch.allclose(m.double().sum(-1), torch.ones(2, 256, 8, dtype=torch.float64), atol=1e-6)
+    assert not torch.equal(x["mix1"], x["mix2"])
+    y = I.leg_inputs(wl)
+    assert all(torch.equal(x[key], y[key]) for key in x)
