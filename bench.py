@@ -58,6 +58,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=5)
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the separately timed calls around the step (legs, SER backward)")
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle sample")
     return p.parse_args(argv)
@@ -391,6 +393,10 @@ def run_ours(args):
         "bytes_per_launch": dom["bytes"], "bytes_kind": "compulsory",
     }
 
+    extra = None
+    if not args.no_extra:
+        extra = measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak)
+
     e2e = None
     if not args.no_e2e:
         e2e = measure_e2e(gm, wl, x, dev, stream, args.e2e_steps, world)
@@ -416,6 +422,7 @@ def run_ours(args):
             "roofline": roofline,
             "calls": {k: {kk: (round(vv, 3) if isinstance(vv, float) else vv)
                           for kk, vv in c.items()} for k, c in calls.items()},
+            "extra_calls": extra,
             "kv_rows_touched_frac": cb["kv_rows_touched"] / cb["kv_rows_total"],
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step * args.steps,
             "clocks": clocks, "source_hash": source_hash(),
@@ -424,6 +431,68 @@ def run_ours(args):
         import torch.distributed as dist
         dist.destroy_process_group()
     return result
+
+
+def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
+    """The calls around the step, each timed alone with CUDA events, L2 flushed between reps.
+
+    leg_sparsify builds the step's two legs from the workload's stored edges; ser_backward
+    takes the step's d ln w back to the legs; leg_backward takes those leg gradients back to
+    the stored weights and the mixing coefficients. Bytes are compulsory: every input read
+    once, every output written once (ser_backward's second-leg rows counted in full).
+    """
+    le = {k: v.to(dev) for k, v in I.leg_inputs(wl).items()}
+    B, n, k = wl.B, wl.n, wl.hkv
+    tok = B * n
+    f32 = torch.float32
+    a1i = torch.empty((B, n, k, wl.s2), dtype=torch.int32, device=dev)
+    a1w = torch.empty((B, n, k, wl.s2), dtype=f32, device=dev)
+    a2i = torch.empty((B, n, k, wl.s3), dtype=torch.int32, device=dev)
+    a2w = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
+    dw1 = torch.empty((B, n, k, wl.s2), dtype=f32, device=dev)
+    dw2 = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
+    dew = torch.empty((B, n, k, wl.s1), dtype=f32, device=dev)
+    dm1 = torch.empty((B, n, k, k), dtype=f32, device=dev)
+    dm2 = torch.empty_like(dm1)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
+    leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
+    calls = {
+        "leg_sparsify": ("leg_fwd_kernel", e_b + mix_b + leg_b,
+                         lambda: gm.gm_leg_sparsify(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
+                                                    wl.s2, wl.s3, a1i, a1w, a2i, a2w, stream=stream)),
+        "ser_backward": ("zero_i32_kernel + ser_bwd_kernel",
+                         leg_b + tok * k * wl.s1 * 4 + grad_b + tok * k * wl.s3 * 4,
+                         lambda: gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"],
+                                                    dlw, grad_is_log=True, dw1=dw1, dw2=dw2,
+                                                    stream=stream)),
+        "leg_backward": ("leg_bwd_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
+                         lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
+                                                    dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,
+                                                    stream=stream)),
+    }
+    out = {}
+    for name, (kernel, nbytes, fn) in calls.items():
+        for _ in range(3):
+            fn()
+        times = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1) * 1e3)
+        us = statistics.median(times)
+        gbps = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"kernel": kernel, "us": round(us, 2), "bytes": nbytes,
+                     "GBps": round(gbps, 1), "frac": round(gbps / peak, 4)}
+    gm.gm_check_device_errors(stream)
+    out["note"] = ("timed alone, median of %d reps, L2 flushed (256 MB write) before each; "
+                   "not part of the step's value" % reps)
+    return out
 
 
 def measure_e2e(gm, wl, x, dev, stream, steps, world):

@@ -71,6 +71,70 @@ typedef enum gm_dtype {
 } gm_dtype;
 
 /*
+ * gm_leg_sparsify - the pair of referral legs of every (token, edge channel), built from the
+ * stored edges.
+ * Source: ai.info summary, "Methodology in Plain English", referral paragraph (the stored
+ * edges are mixed into pairs and each leg is sparsified before the composition) and "Main
+ * Findings", bullet on more edges (the cross-edge mixing is full: its cost grows as k^2).
+ * The pages give no formula; the reading here: leg L of channel h at token (b, i) mixes the
+ * token's own stored edges across all k stored channels.
+ *
+ * For each (b, i, h) and leg L (coefficients M_L, budget s_L = s2 for leg 1, s3 for leg 2):
+ * every stored edge (c, a), c < k, a < s0, with e_w[b,i,c,a] > 0 is a candidate with target
+ * e_idx[b,i,c,a] and weight fl32(M_L[b,i,h,c] * e_w[b,i,c,a]) (one rounding, no FMA), in
+ * ascending c*s0 + a. Zero products are dropped; candidates reaching the same target are
+ * summed in fp32 in that order; the s_L heaviest targets are written in order of weight
+ * descending, then target ascending, padded with (0, 0.0f). No renormalisation. This is
+ * gm_ser_forward's sparsify applied to the mixed candidates; the outputs are its legs.
+ *
+ *   e_idx, e_w        device, [B, n, k, s0]   stored edges (int32 targets, fp32 weights >= 0)
+ *   mix1, mix2        device fp32, coefficients >= 0 of leg 1 and leg 2: [B, n, k, k]
+ *                     (mix_token_stride = k*k) or one [k, k] matrix shared by every token
+ *                     (mix_token_stride = 0); element [h, c] mixes stored channel c into
+ *                     leg channel h
+ *   a1_idx, a1_w      device, [B, n, k, s2]   leg 1, written
+ *   a2_idx, a2_w      device, [B, n, k, s3]   leg 2, written; outputs must not alias inputs
+ *   limits            1 <= k*s0 <= 32, 1 <= s2, s3 <= 32
+ * An active stored edge whose target lies outside [0, n) is skipped and raises the device
+ * index-range flag (read by gm_check_device_errors). Deterministic, bit-identical to the
+ * definition above.
+ */
+gm_status gm_leg_sparsify(const int32_t *e_idx, const float *e_w, int s0,
+                          const float *mix1, const float *mix2, int64_t mix_token_stride,
+                          int32_t *a1_idx, float *a1_w, int s2,
+                          int32_t *a2_idx, float *a2_w, int s3,
+                          int B, int n, int k, cudaStream_t stream);
+
+/*
+ * gm_leg_backward - gradients of gm_leg_sparsify's kept leg weights with respect to the stored
+ * weights and both sets of mixing coefficients.
+ * Source: as gm_leg_sparsify; and the referral paragraph's rule that only retained weights get
+ * gradients (indices get none).
+ *
+ * The legs of every token are recomputed exactly as gm_leg_sparsify computes them. Each kept
+ * weight W_r of leg L, channel h is differentiated as the sum, over the active stored edges
+ * (c, a) that reach its target t_r, of M_L[h,c] * e_w[c,a]; with g_r = g_L[b,i,h,r]:
+ *   dew[b,i,c,a]       += g_r * M_L[b,i,h,c]
+ *   dmix_L[b,i,h,c]    += g_r * e_w[b,i,c,a]
+ * summed over h, both legs and the kept slots. An active edge whose product was zero (a zero
+ * coefficient) still contributes to dmix. Targets cut by the selection get nothing. fp32; each
+ * output is summed by one warp in a fixed order (deterministic, no atomics).
+ *
+ *   e_idx, e_w, mix1, mix2, mix_token_stride, s0, k   as gm_leg_sparsify
+ *   g1          device fp32 [B, n, k, s2]   gradient w.r.t. leg 1's weights (gm_ser_backward's dw1)
+ *   g2          device fp32 [B, n, k, s3]   gradient w.r.t. leg 2's weights (gm_ser_backward's dw2)
+ *   dew         device fp32 [B, n, k, s0]   written (added to if accumulate)
+ *   dmix1/2     device fp32 [B, n, k, k]    written (added to if accumulate), per token also
+ *               when the coefficients were shared (mix_token_stride = 0): the caller sums them
+ *   limits      as gm_leg_sparsify
+ */
+gm_status gm_leg_backward(const int32_t *e_idx, const float *e_w, int s0,
+                          const float *mix1, const float *mix2, int64_t mix_token_stride,
+                          const float *g1, int s2, const float *g2, int s3,
+                          int B, int n, int k, float *dew, float *dmix1, float *dmix2,
+                          int accumulate, cudaStream_t stream);
+
+/*
  * gm_ser_forward - sparse edge referral, A' = Sparsify_s1(A1 A2).
  * Source: ai.info summary, "Key Contributions" item 3 (A' = Sparsify_s1(A1 A2), up to s2*s3
  * candidates cut back to s1) and "Methodology in Plain English", referral paragraph (the

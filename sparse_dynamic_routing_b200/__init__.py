@@ -3,6 +3,8 @@
 The compute lives in the CUDA library libgm_b200.so (C ABI: include/gm.h); this package is
 its Python binding plus the seeded synthetic-input generators (`inputs`).
 
+    gm_leg_sparsify     both referral legs from the stored edges (mixed, then sparsified)
+    gm_leg_backward     gradients of the kept leg weights
     gm_ser_forward      sparse edge referral, A' = Sparsify_s1(A1 A2)
     gm_sea_forward      sparse edge attention
     gm_ser_sea_forward  both in one kernel
@@ -16,6 +18,8 @@ from ._binding import (  # noqa: F401
     GMIndexRangeError,
     LIB_PATH,
     gm_check_device_errors,
+    gm_leg_backward,
+    gm_leg_sparsify,
     gm_sea_backward,
     gm_sea_backward_noalloc,
     gm_sea_backward_workspace_size,

@@ -24,6 +24,10 @@ GM_F32, GM_BF16 = 0, 1
 # Entry points of include/gm.h with their ctypes signatures.
 _vp, _ci, _cf = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
+    "gm_leg_sparsify": [_vp, _vp, _ci, _vp, _vp, ctypes.c_int64, _vp, _vp, _ci, _vp, _vp, _ci,
+                        _ci, _ci, _ci, _vp],
+    "gm_leg_backward": [_vp, _vp, _ci, _vp, _vp, ctypes.c_int64, _vp, _ci, _vp, _ci, _ci, _ci,
+                        _ci, _vp, _vp, _vp, _ci, _vp],
     "gm_ser_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
     "gm_ser_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _vp, _vp, _ci,
                         _vp],
@@ -116,6 +120,62 @@ def _fdtype(t: torch.Tensor) -> int:
 
 def _scale(scale, d):
     return float(1.0 / math.sqrt(d)) if scale is None else float(scale)
+
+
+def _leg_shapes(e_idx, e_w, mix1, mix2):
+    B, n, k, s0 = e_idx.shape
+    if e_w.shape != e_idx.shape:
+        raise ValueError("stored edge weights disagree with their indices")
+    if mix1.shape != mix2.shape:
+        raise ValueError("both legs' coefficients must have the same shape")
+    if tuple(mix1.shape) == (k, k):
+        stride = 0
+    elif tuple(mix1.shape) == (B, n, k, k):
+        stride = k * k
+    else:
+        raise ValueError("mixing coefficients must be [B, n, k, k] or [k, k]")
+    return B, n, k, s0, stride
+
+
+def gm_leg_sparsify(e_idx, e_w, mix1, mix2, s2: int, s3: int, a1_idx=None, a1_w=None,
+                    a2_idx=None, a2_w=None, stream=None):
+    """Both referral legs from the stored edges. Returns (a1_idx, a1_w, a2_idx, a2_w)."""
+    B, n, k, s0, stride = _leg_shapes(e_idx, e_w, mix1, mix2)
+    dev = e_idx.device
+    i32, f32 = torch.int32, torch.float32
+    a1_idx = torch.empty((B, n, k, s2), dtype=i32, device=dev) if a1_idx is None else a1_idx
+    a1_w = torch.empty((B, n, k, s2), dtype=f32, device=dev) if a1_w is None else a1_w
+    a2_idx = torch.empty((B, n, k, s3), dtype=i32, device=dev) if a2_idx is None else a2_idx
+    a2_w = torch.empty((B, n, k, s3), dtype=f32, device=dev) if a2_w is None else a2_w
+    st = load_library().gm_leg_sparsify(
+        _ptr(e_idx, i32, "e_idx"), _ptr(e_w, f32, "e_w"), s0,
+        _ptr(mix1, f32, "mix1"), _ptr(mix2, f32, "mix2"), stride,
+        _ptr(a1_idx, i32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, i32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3, B, n, k, _stream(stream))
+    _check(st, "gm_leg_sparsify")
+    return a1_idx, a1_w, a2_idx, a2_w
+
+
+def gm_leg_backward(e_idx, e_w, mix1, mix2, g1, g2, dew=None, dmix1=None, dmix2=None,
+                    accumulate=False, stream=None):
+    """Gradients of the kept leg weights. Returns (dew [B,n,k,s0], dmix1, dmix2 [B,n,k,k])."""
+    B, n, k, s0, stride = _leg_shapes(e_idx, e_w, mix1, mix2)
+    s2, s3 = g1.shape[3], g2.shape[3]
+    if tuple(g1.shape[:3]) != (B, n, k) or tuple(g2.shape[:3]) != (B, n, k):
+        raise ValueError("leg gradients must be [B, n, k, s]")
+    dev = e_idx.device
+    f32 = torch.float32
+    dew = torch.empty((B, n, k, s0), dtype=f32, device=dev) if dew is None else dew
+    dmix1 = torch.empty((B, n, k, k), dtype=f32, device=dev) if dmix1 is None else dmix1
+    dmix2 = torch.empty((B, n, k, k), dtype=f32, device=dev) if dmix2 is None else dmix2
+    st = load_library().gm_leg_backward(
+        _ptr(e_idx, torch.int32, "e_idx"), _ptr(e_w, f32, "e_w"), s0,
+        _ptr(mix1, f32, "mix1"), _ptr(mix2, f32, "mix2"), stride,
+        _ptr(g1, f32, "g1"), s2, _ptr(g2, f32, "g2"), s3, B, n, k,
+        _ptr(dew, f32, "dew"), _ptr(dmix1, f32, "dmix1"), _ptr(dmix2, f32, "dmix2"),
+        int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_leg_backward")
+    return dew, dmix1, dmix2
 
 
 def gm_ser_forward(a1_idx, a1_w, a2_idx, a2_w, s1: int, out_idx=None, out_w=None, stream=None):

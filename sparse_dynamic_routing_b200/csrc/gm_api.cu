@@ -9,6 +9,7 @@
 #include "gm_bwd_tile.cuh"
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
+#include "gm_leg.cuh"
 #include "gm_sea.cuh"
 #include "gm_sea_bwd.cuh"
 #include "gm_ser.cuh"
@@ -48,6 +49,21 @@ gm_status check_ser(const int32_t *a1_idx, const float *a1_w, int s2, const int3
     if ((int64_t)B * n == 0) return GM_OK;
     if ((int64_t)B * n * k >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
     if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
+    return GM_OK;
+}
+
+constexpr int WPB_LEG = 8;   // warps (tokens) per block of the leg kernels
+
+gm_status check_leg(const int32_t *e_idx, const float *e_w, int s0, const float *mix1,
+                    const float *mix2, int64_t mix_token_stride, int s2, int s3, int B, int n,
+                    int k)
+{
+    if (B < 0 || n < 0 || k < 1 || s0 < 1 || s2 < 1 || s3 < 1) return GM_ERR_INVALID_ARG;
+    if (k * s0 > MAX_SLOTS || s2 > MAX_SLOTS || s3 > MAX_SLOTS) return GM_ERR_INVALID_ARG;
+    if (mix_token_stride != 0 && mix_token_stride != (int64_t)k * k) return GM_ERR_INVALID_ARG;
+    if ((int64_t)B * n == 0) return GM_OK;
+    if ((int64_t)B * n * k >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
+    if (!e_idx || !e_w || !mix1 || !mix2) return GM_ERR_INVALID_ARG;
     return GM_OK;
 }
 
@@ -379,6 +395,67 @@ gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
     const SerArgs f{a1_idx, a1_w, a2_idx, a2_w, nullptr, nullptr, s1, s2, s3, n, k, (uint32_t)rows, row_map(k, n)};
     const gm::SerBwdArgs b{f, gout, grad_is_log, dw1, dw2, accumulate};
     gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
+    return launched();
+}
+
+gm_status gm_leg_sparsify(const int32_t *e_idx, const float *e_w, int s0,
+                          const float *mix1, const float *mix2, int64_t mix_token_stride,
+                          int32_t *a1_idx, float *a1_w, int s2,
+                          int32_t *a2_idx, float *a2_w, int s3,
+                          int B, int n, int k, cudaStream_t stream)
+{
+    gm_status st = check_leg(e_idx, e_w, s0, mix1, mix2, mix_token_stride, s2, s3, B, n, k);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
+    gm::LegArgs a{};
+    a.e_idx = e_idx;
+    a.e_w = e_w;
+    a.mix1 = mix1;
+    a.mix2 = mix2;
+    a.mix_stride = (uint32_t)mix_token_stride;
+    a.a1_idx = a1_idx;
+    a.a1_w = a1_w;
+    a.a2_idx = a2_idx;
+    a.a2_w = a2_w;
+    a.k = k;
+    a.s0 = s0;
+    a.s2 = s2;
+    a.s3 = s3;
+    a.n = n;
+    a.tokens = (uint32_t)((int64_t)B * n);
+    gm::leg_fwd_kernel<WPB_LEG><<<blocks_for(a.tokens, WPB_LEG), WPB_LEG * 32, 0, stream>>>(a);
+    return launched();
+}
+
+gm_status gm_leg_backward(const int32_t *e_idx, const float *e_w, int s0,
+                          const float *mix1, const float *mix2, int64_t mix_token_stride,
+                          const float *g1, int s2, const float *g2, int s3,
+                          int B, int n, int k, float *dew, float *dmix1, float *dmix2,
+                          int accumulate, cudaStream_t stream)
+{
+    if (accumulate != 0 && accumulate != 1) return GM_ERR_INVALID_ARG;
+    gm_status st = check_leg(e_idx, e_w, s0, mix1, mix2, mix_token_stride, s2, s3, B, n, k);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!g1 || !g2 || !dew || !dmix1 || !dmix2) return GM_ERR_INVALID_ARG;
+    gm::LegArgs a{};
+    a.e_idx = e_idx;
+    a.e_w = e_w;
+    a.mix1 = mix1;
+    a.mix2 = mix2;
+    a.mix_stride = (uint32_t)mix_token_stride;
+    a.g1 = g1;
+    a.g2 = g2;
+    a.dew = dew;
+    a.dmix1 = dmix1;
+    a.dmix2 = dmix2;
+    a.accumulate = accumulate;
+    a.k = k;
+    a.s0 = s0;
+    a.s2 = s2;
+    a.s3 = s3;
+    a.n = n;
+    a.tokens = (uint32_t)((int64_t)B * n);
+    gm::leg_bwd_kernel<WPB_LEG><<<blocks_for(a.tokens, WPB_LEG), WPB_LEG * 32, 0, stream>>>(a);
     return launched();
 }
 

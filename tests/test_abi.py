@@ -135,3 +135,27 @@ def test_backward_and_fused_argument_checks(lib):
     fb2 = list(fb)
     fb2[2], fb2[5] = 8, 8  # 64 candidates
     assert g(*fb2) == bnd.GM_ERR_INVALID_ARG
+
+
+def test_leg_argument_checks(lib):
+    f = lib.gm_leg_sparsify
+    # e_idx, e_w, s0, mix1, mix2, stride, a1_idx, a1_w, s2, a2_idx, a2_w, s3, B, n, k, stream
+    good = dict(s0=4, stride=64, s2=4, s3=4, B=1, n=8, k=8)
+    bad_cases = [dict(s0=0), dict(s0=5), dict(k=0), dict(s2=0), dict(s3=33), dict(stride=63),
+                 dict(stride=8), dict(n=-1), dict(B=-2)]
+    for change in bad_cases:
+        a = dict(good, **change)
+        st = f(FAKE, FAKE, a["s0"], FAKE, FAKE, a["stride"], FAKE, FAKE, a["s2"], FAKE, FAKE,
+               a["s3"], a["B"], a["n"], a["k"], NULL)
+        assert st == bnd.GM_ERR_INVALID_ARG, change
+    # null outputs / inputs
+    assert f(FAKE, FAKE, 4, FAKE, NULL, 64, FAKE, FAKE, 4, FAKE, FAKE, 4, 1, 8, 8, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, FAKE, FAKE, 0, FAKE, FAKE, 4, NULL, FAKE, 4, 1, 8, 8, NULL) == bnd.GM_ERR_INVALID_ARG
+    # an empty problem is a no-op that succeeds without touching any pointer
+    assert f(NULL, NULL, 4, NULL, NULL, 64, NULL, NULL, 4, NULL, NULL, 4, 0, 8, 8, NULL) == bnd.GM_OK
+    g = lib.gm_leg_backward
+    # e_idx, e_w, s0, mix1, mix2, stride, g1, s2, g2, s3, B, n, k, dew, dmix1, dmix2, acc, stream
+    assert g(FAKE, FAKE, 4, FAKE, FAKE, 64, FAKE, 4, FAKE, 4, 1, 8, 8, FAKE, FAKE, NULL, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 4, FAKE, FAKE, 64, FAKE, 4, FAKE, 4, 1, 8, 8, FAKE, FAKE, FAKE, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 9, FAKE, FAKE, 64, FAKE, 4, FAKE, 4, 1, 8, 8, FAKE, FAKE, FAKE, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert g(NULL, NULL, 4, NULL, NULL, 0, NULL, 4, NULL, 4, 3, 0, 8, NULL, NULL, NULL, 0, NULL) == bnd.GM_OK

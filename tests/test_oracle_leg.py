@@ -221,3 +221,25 @@ def test_leg_backward_hand_worked_example():
     assert dew[0, 3].tolist() == [[2.0, 0.0], [1.0, -0.5]]
     assert dm1[0, 3].tolist() == [[1.0, -0.25], [0.0, 0.0]]
     assert not dm2.any()
+
+
+def test_chain_gradient_of_first_leg_coefficients_respects_softmax_shift_invariance():
+    # Scaling leg 1's row (i, h) by a factor scales every candidate of referral row (i, h) and so
+    # the whole referral row; attention adds ln of it to every score and is unchanged. Hence
+    # sum_c M1[i,h,c] * dM1[i,h,c] = 0 for every row, while the entries themselves are not zero.
+    from sparse_dynamic_routing_b200 import inputs as I
+    wl = I.WORKLOADS["tiny_b1_n128_s2_f32"].with_(hq=4, hkv=2, n=48)
+    x = I.make(wl, grad=True)
+    le = I.leg_inputs(wl)
+    a1i, a1w, a2i, a2w, _ = oracle.leg_sparsify(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
+                                                wl.s2, wl.s3)
+    oi, ow, _ = oracle.ser(a1i, a1w, a2i, a2w, wl.s1)
+    _, _, _, dlw, _ = oracle.sea_backward(x["q"], x["k"], x["v"], x["dout"], oi, ow, wl.scale)
+    d1, d2, _ = oracle.ser_backward(a1i, a1w, a2i, a2w, dlw.astype(np.float32), grad_is_log=True)
+    _, dm1, dm2, _ = oracle.leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
+                                         d1.astype(np.float32), d2.astype(np.float32))
+    m1 = le["mix1"].numpy().astype(np.float64)
+    terms = m1 * dm1
+    assert np.abs(dm1).max() > 1e-3
+    # fp32 rounding of the intermediate gradients (d ln w, dw1) bounds the residue
+    np.testing.assert_allclose(terms.sum(-1), 0.0, atol=1e-5 * np.abs(terms).sum(-1).max())
