@@ -454,19 +454,21 @@ def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     dew = torch.empty((B, n, k, wl.s1), dtype=f32, device=dev)
     dm1 = torch.empty((B, n, k, k), dtype=f32, device=dev)
     dm2 = torch.empty_like(dm1)
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    # L2 is evicted by reading a 256 MB buffer (a write would leave dirty lines whose
+    # write-back the next timed call would pay for)
+    flush = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
     e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
     leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
     calls = {
-        "leg_sparsify": ("leg_fwd_kernel", e_b + mix_b + leg_b,
+        "leg_sparsify": ("leg_fwd_tile_kernel", e_b + mix_b + leg_b,
                          lambda: gm.gm_leg_sparsify(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     wl.s2, wl.s3, a1i, a1w, a2i, a2w, stream=stream)),
-        "ser_backward": ("zero_i32_kernel + ser_bwd_kernel",
+        "ser_backward": ("zero_i32_kernel + ser_bwd_thread_kernel",
                          leg_b + tok * k * wl.s1 * 4 + grad_b + tok * k * wl.s3 * 4,
                          lambda: gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"],
                                                     dlw, grad_is_log=True, dw1=dw1, dw2=dw2,
                                                     stream=stream)),
-        "leg_backward": ("leg_bwd_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
+        "leg_backward": ("leg_bwd_tile_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
                          lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,
                                                     stream=stream)),
@@ -475,22 +477,24 @@ def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     for name, (kernel, nbytes, fn) in calls.items():
         for _ in range(3):
             fn()
-        times = []
+        # all reps are queued before one synchronize: the flush keeps the device busy while
+        # the host queues the next call, so no event brackets host-side launch latency
+        evs = []
         for _ in range(reps):
-            flush.fill_(1)
+            flush.sum()
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             fn()
             e1.record(stream)
-            torch.cuda.synchronize(dev)
-            times.append(e0.elapsed_time(e1) * 1e3)
-        us = statistics.median(times)
+            evs.append((e0, e1))
+        torch.cuda.synchronize(dev)
+        us = statistics.median(e0.elapsed_time(e1) * 1e3 for e0, e1 in evs)
         gbps = nbytes / (us * 1e-6) / 1e9
         out[name] = {"kernel": kernel, "us": round(us, 2), "bytes": nbytes,
                      "GBps": round(gbps, 1), "frac": round(gbps / peak, 4)}
     gm.gm_check_device_errors(stream)
-    out["note"] = ("timed alone, median of %d reps, L2 flushed (256 MB write) before each; "
+    out["note"] = ("timed alone, median of %d reps, L2 flushed (256 MB read) before each; "
                    "not part of the step's value" % reps)
     return out
 

@@ -10,6 +10,7 @@
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
 #include "gm_leg.cuh"
+#include "gm_leg_tile.cuh"
 #include "gm_sea.cuh"
 #include "gm_sea_bwd.cuh"
 #include "gm_ser.cuh"
@@ -22,6 +23,7 @@ using gm::SeaBwdArgs;
 using gm::SerArgs;
 
 constexpr int WPB_SER = 8;   // warps (edge rows) per block
+constexpr int WPB_SER_THREAD = 4;  // warps per block of the thread-per-row SER backward
 constexpr int WPB_SEA = GM_WPB_SEA;
 constexpr int WPB_BWD = GM_WPB_BWD;
 constexpr int MAX_SLOTS = 32;
@@ -65,6 +67,36 @@ gm_status check_leg(const int32_t *e_idx, const float *e_w, int s0, const float 
     if ((int64_t)B * n * k >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
     if (!e_idx || !e_w || !mix1 || !mix2) return GM_ERR_INVALID_ARG;
     return GM_OK;
+}
+
+constexpr int WPB_LEG_TILE = 4;
+constexpr int LEG_TILE_SM = 4;  // largest leg budget of the thread-per-row kernels
+
+template <int K, int S0>
+gm_status launch_leg_tile(const gm::LegArgs &a, bool backward, cudaStream_t stream)
+{
+    using Geo = gm::LegTileGeom<K, S0>;
+    const int64_t warps = ((int64_t)a.tokens + Geo::TPW - 1) / Geo::TPW;
+    const unsigned blocks = (unsigned)((warps + WPB_LEG_TILE - 1) / WPB_LEG_TILE);
+    if (backward)
+        gm::leg_bwd_tile_kernel<K, S0, LEG_TILE_SM, WPB_LEG_TILE><<<blocks, WPB_LEG_TILE * 32, 0, stream>>>(a);
+    else
+        gm::leg_fwd_tile_kernel<K, S0, LEG_TILE_SM, WPB_LEG_TILE><<<blocks, WPB_LEG_TILE * 32, 0, stream>>>(a);
+    return launched();
+}
+
+// The thread-per-row kernels cover k in {4, 8, 16}, s0 in {2, 4} (k*s0 <= 32) and leg budgets
+// up to LEG_TILE_SM; returns GM_ERR_UNSUPPORTED for every other shape (the caller then runs
+// the warp-per-token kernel).
+gm_status try_leg_tile(const gm::LegArgs &a, bool backward, cudaStream_t stream)
+{
+    if (a.s2 > LEG_TILE_SM || a.s3 > LEG_TILE_SM) return GM_ERR_UNSUPPORTED;
+    if (a.k == 8 && a.s0 == 4) return launch_leg_tile<8, 4>(a, backward, stream);
+    if (a.k == 8 && a.s0 == 2) return launch_leg_tile<8, 2>(a, backward, stream);
+    if (a.k == 4 && a.s0 == 4) return launch_leg_tile<4, 4>(a, backward, stream);
+    if (a.k == 4 && a.s0 == 2) return launch_leg_tile<4, 2>(a, backward, stream);
+    if (a.k == 16 && a.s0 == 2) return launch_leg_tile<16, 2>(a, backward, stream);
+    return GM_ERR_UNSUPPORTED;
 }
 
 // Shapes shared by SEA forward and backward. Returns GM_OK, or the error to report.
@@ -394,6 +426,18 @@ gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
     }
     const SerArgs f{a1_idx, a1_w, a2_idx, a2_w, nullptr, nullptr, s1, s2, s3, n, k, (uint32_t)rows, row_map(k, n)};
     const gm::SerBwdArgs b{f, gout, grad_is_log, dw1, dw2, accumulate};
+    // per-thread rows for the small budgets the fused forward tiles (vector loads need
+    // 16-byte aligned legs)
+    const bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w);
+    const unsigned tblocks = blocks_for(rows, 32 * WPB_SER_THREAD);
+    if (aligned && s2 == 4 && s3 == 4 && s1 <= 4) {
+        gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        return launched();
+    }
+    if (aligned && s2 == 2 && s3 == 2 && s1 <= 4) {
+        gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        return launched();
+    }
     gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
     return launched();
 }
@@ -423,6 +467,8 @@ gm_status gm_leg_sparsify(const int32_t *e_idx, const float *e_w, int s0,
     a.s3 = s3;
     a.n = n;
     a.tokens = (uint32_t)((int64_t)B * n);
+    const gm_status tile = try_leg_tile(a, false, stream);
+    if (tile != GM_ERR_UNSUPPORTED) return tile;
     gm::leg_fwd_kernel<WPB_LEG><<<blocks_for(a.tokens, WPB_LEG), WPB_LEG * 32, 0, stream>>>(a);
     return launched();
 }
@@ -455,6 +501,8 @@ gm_status gm_leg_backward(const int32_t *e_idx, const float *e_w, int s0,
     a.s3 = s3;
     a.n = n;
     a.tokens = (uint32_t)((int64_t)B * n);
+    const gm_status tile = try_leg_tile(a, true, stream);
+    if (tile != GM_ERR_UNSUPPORTED) return tile;
     gm::leg_bwd_kernel<WPB_LEG><<<blocks_for(a.tokens, WPB_LEG), WPB_LEG * 32, 0, stream>>>(a);
     return launched();
 }

@@ -73,6 +73,33 @@ __device__ __forceinline__ LegLane leg_lane(const LegArgs &a, uint32_t tok, int 
     return L;
 }
 
+// A small per-token array (one leg's [k, k] coefficients, or one leg's [k, s] gradients),
+// cached across the warp: with at most 64 elements lane l holds elements l and 32 + l in
+// registers, loaded before any row is processed so the token's loads overlap; element e is
+// then two shuffles away. Larger arrays read through L1.
+struct TokCache {
+    const float *p;
+    float r0, r1;
+    bool regs;
+    __device__ __forceinline__ void load(const float *base, int kk, int lane)
+    {
+        p = base;
+        regs = kk <= 64;
+        r0 = regs && lane < kk ? __ldg(base + lane) : 0.0f;
+        r1 = regs && lane + 32 < kk ? __ldg(base + 32 + lane) : 0.0f;
+    }
+    // element e (per lane; lanes with use == false get 0, but every lane takes part)
+    __device__ __forceinline__ float get(int e, bool use) const
+    {
+        if (regs) {  // warp-uniform
+            const float a = __shfl_sync(FULL, r0, e & 31);
+            const float b = __shfl_sync(FULL, r1, e & 31);
+            return use ? (e < 32 ? a : b) : 0.0f;
+        }
+        return use ? __ldg(p + e) : 0.0f;
+    }
+};
+
 // Merge the nonzero products u of one (leg, channel) row by target, in ascending lane order,
 // and return this lane's selection key (nonzero only on each target's first lane).
 __device__ __forceinline__ void leg_merge(const LegLane &L, float u, int lane, unsigned &key_hi,
@@ -100,15 +127,18 @@ __global__ void __launch_bounds__(WPB * 32) leg_fwd_kernel(LegArgs a)
     const int lane = threadIdx.x & 31;
     const uint32_t tok = blockIdx.x * WPB + (threadIdx.x >> 5);
     if (tok >= a.tokens) return;  // warp-uniform
+    TokCache M[2];
+    M[0].load(a.mix1 + (size_t)tok * a.mix_stride, a.k * a.k, lane);
+    M[1].load(a.mix2 + (size_t)tok * a.mix_stride, a.k * a.k, lane);
     const LegLane L = leg_lane(a, tok, lane);
 
+#pragma unroll
     for (int leg = 0; leg < 2; ++leg) {
-        const float *mix = (leg == 0 ? a.mix1 : a.mix2) + (size_t)tok * a.mix_stride;
         const int sl = leg == 0 ? a.s2 : a.s3;
         int32_t *oi = leg == 0 ? a.a1_idx : a.a2_idx;
         float *ow = leg == 0 ? a.a1_w : a.a2_w;
         for (int h = 0; h < a.k; ++h) {
-            const float m = L.act ? __ldg(mix + h * a.k + L.c) : 0.0f;
+            const float m = M[leg].get(h * a.k + L.c, L.act);
             const float u = L.act ? __fmul_rn(m, L.w) : 0.0f;
             unsigned key_hi, key_lo;
             leg_merge(L, u, lane, key_hi, key_lo);
@@ -139,18 +169,24 @@ __global__ void __launch_bounds__(WPB * 32) leg_bwd_kernel(LegArgs a)
     const int lane = threadIdx.x & 31;
     const uint32_t tok = blockIdx.x * WPB + (threadIdx.x >> 5);
     if (tok >= a.tokens) return;  // warp-uniform
+    TokCache M[2];
+    M[0].load(a.mix1 + (size_t)tok * a.mix_stride, a.k * a.k, lane);
+    M[1].load(a.mix2 + (size_t)tok * a.mix_stride, a.k * a.k, lane);
     const LegLane L = leg_lane(a, tok, lane);
     const int nc = a.k * a.s0;
     const bool head = lane < nc && lane == L.c * a.s0;  // first lane of its stored channel
 
+    TokCache G[2];
+    G[0].load(a.g1 + (size_t)tok * a.k * a.s2, a.k * a.s2, lane);
+    G[1].load(a.g2 + (size_t)tok * a.k * a.s3, a.k * a.s3, lane);
+
     float dew = 0.0f;
+#pragma unroll
     for (int leg = 0; leg < 2; ++leg) {
-        const float *mix = (leg == 0 ? a.mix1 : a.mix2) + (size_t)tok * a.mix_stride;
         const int sl = leg == 0 ? a.s2 : a.s3;
-        const float *g = leg == 0 ? a.g1 : a.g2;
         float *dmix = (leg == 0 ? a.dmix1 : a.dmix2) + (size_t)tok * a.k * a.k;
         for (int h = 0; h < a.k; ++h) {
-            const float m = L.act ? __ldg(mix + h * a.k + L.c) : 0.0f;
+            const float m = M[leg].get(h * a.k + L.c, L.act);
             const float u = L.act ? __fmul_rn(m, L.w) : 0.0f;
             unsigned key_hi, key_lo;
             leg_merge(L, u, lane, key_hi, key_lo);
@@ -164,7 +200,7 @@ __global__ void __launch_bounds__(WPB * 32) leg_bwd_kernel(LegArgs a)
                 if (L.act && (int32_t)~ml == L.t) slot = r;
                 if (key_hi == mh && key_lo == ml) key_hi = key_lo = 0u;
             }
-            const float gr = slot >= 0 ? __ldg(g + ((size_t)tok * a.k + h) * sl + slot) : 0.0f;
+            const float gr = G[leg].get(h * sl + (slot >= 0 ? slot : 0), slot >= 0);
             dew = fmaf(gr, m, dew);
             // dM[h, c] = sum over the channel's s0 lanes, ascending a
             const float x = gr * L.w;

@@ -14,6 +14,7 @@
 #pragma once
 
 #include "gm_common.cuh"
+#include "gm_fused_tile.cuh"
 #include "gm_ser.cuh"
 
 namespace gm {
@@ -116,6 +117,107 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
     }
     // ---- second leg: scatter to the shared second-leg rows ----------------------------------------
     if (slot >= 0) atomicAdd(b.dw2 + r2, g * w1);
+}
+
+// The same backward, one thread per edge row, for small exact budgets (S2, S3; s1 <= S1M):
+// the referral is recomputed in registers exactly as the fused forward's per-thread referral
+// (same products, pairwise merge in ascending candidate order, arg-max selection), each
+// candidate finds the kept slot of its target, the first-leg gradient of slot a is summed
+// in ascending e, and the second-leg gradients are scatter-added with fp32 atomics. It
+// spends a fraction of the warp-per-row kernel's instructions when the budgets are 2 or 4.
+template <int S2, int S3, int S1M, int WPB>
+__global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
+{
+    constexpr int NC = S2 * S3;
+    const SerArgs &a = b.f;
+    const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
+    if (row >= a.rows) return;  // no warp-wide operation below
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    int32_t j[S2];
+    float w1[S2];
+    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
+    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
+
+    int32_t ct[NC];
+    float cu[NC], w2c[NC];
+    size_t r2[S2];
+#pragma unroll
+    for (int x = 0; x < S2; ++x) {
+        bool act = w1[x] > 0.0f;
+        if (act && (j[x] < 0 || j[x] >= a.n)) {
+            raise_index_error();
+            act = false;
+        }
+        int32_t t2[S3];
+        float w2[S3];
+#pragma unroll
+        for (int e = 0; e < S3; ++e) {
+            t2[e] = 0;
+            w2[e] = 0.0f;
+        }
+        r2[x] = act ? ((size_t)(seq_base + (uint32_t)j[x]) * a.k + h) * S3 : 0;
+        if (act) {
+            ld_vec<S3>(a.a2_idx + r2[x], t2);
+            ld_vec<S3>(a.a2_w + r2[x], w2);
+        }
+#pragma unroll
+        for (int e = 0; e < S3; ++e) {
+            bool v = w2[e] > 0.0f;
+            if (v && (t2[e] < 0 || t2[e] >= a.n)) {
+                raise_index_error();
+                v = false;
+            }
+            ct[x * S3 + e] = t2[e];
+            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+            w2c[x * S3 + e] = w2[e];
+        }
+    }
+    bool cand[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) cand[c] = cu[c] != 0.0f;
+    merge_pairs<0, 1, NC>(ct, cu);
+    // selection (weight desc, target asc) and the upstream gradient of each kept slot
+    int32_t kt[S1M];
+    float kg[S1M];
+#pragma unroll
+    for (int r = 0; r < S1M; ++r) {
+        float bw = 0.0f;
+        int32_t bt = 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const bool better = cu[c] > bw || (cu[c] == bw && cu[c] > 0.0f && ct[c] < bt);
+            bw = better ? cu[c] : bw;
+            bt = better ? ct[c] : bt;
+        }
+#pragma unroll
+        for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
+        const bool keep = r < a.s1 && bw > 0.0f;
+        float g = keep ? __ldg(b.gout + (size_t)row * a.s1 + r) : 0.0f;
+        if (b.grad_is_log) g = keep ? g / bw : 0.0f;
+        kt[r] = keep ? bt : -1;  // -1 never equals a valid target
+        kg[r] = g;
+    }
+    // per candidate: the gradient of its kept target (0 if cut)
+    float gc[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        float g = 0.0f;
+#pragma unroll
+        for (int r = 0; r < S1M; ++r) g = (cand[c] && ct[c] == kt[r]) ? kg[r] : g;
+        gc[c] = g;
+    }
+#pragma unroll
+    for (int x = 0; x < S2; ++x) {
+        float d1 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < S3; ++e) d1 += gc[x * S3 + e] * w2c[x * S3 + e];
+        float *p = b.dw1 + (size_t)row * S2 + x;
+        *p = b.accumulate ? *p + d1 : d1;
+#pragma unroll
+        for (int e = 0; e < S3; ++e)
+            if (gc[x * S3 + e] != 0.0f) atomicAdd(b.dw2 + r2[x] + e, gc[x * S3 + e] * w1[x]);
+    }
 }
 
 }  // namespace gm

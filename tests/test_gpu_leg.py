@@ -67,6 +67,9 @@ LEG_SHAPES = [  # k, s0, s2, s3, n, shared
     (8, 4, 4, 4, 300, False), (8, 2, 2, 2, 128, False), (4, 4, 4, 16, 97, False),
     (2, 3, 5, 1, 61, True), (1, 1, 1, 1, 33, False), (16, 2, 4, 4, 50, False),
     (32, 1, 8, 3, 40, True), (3, 5, 2, 7, 45, False), (8, 4, 32, 1, 70, False),
+    # thread-per-row shapes with ragged token counts
+    (8, 4, 4, 4, 301, False), (8, 2, 3, 2, 97, True), (4, 4, 4, 1, 45, False),
+    (4, 2, 2, 3, 63, False), (16, 2, 4, 4, 51, True), (16, 2, 1, 2, 7, False),
 ]
 
 
