@@ -36,8 +36,14 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
     static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
 };
 
+// Resident blocks per SM the tile kernel is compiled for (its shared memory allows about four
+// at the largest stage): caps registers at 65536 / (32 * WPB * MINB) without forcing spills.
+#ifndef GM_BWD_TILE_MINB
+#define GM_BWD_TILE_MINB 4
+#endif
+
 template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER>
-__global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
+__global__ void __launch_bounds__(WPB * 32, GM_BWD_TILE_MINB) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
     using TG = BwdTileGeom<T, D, G, S1M>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
@@ -61,6 +67,10 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
         // ---- phase 1: the tile's edges, one thread per row ----------------------------------
         {
             const uint32_t row = r0 + lane;
+            // slots are stored as K/V rows ((b*n + t)*hkv + h): phase 2 issues its copies and
+            // keys its records without decomposing the row again
+            uint32_t seq_base = 0, h = 0;
+            if (row < rows) a.map.split(row, seq_base, h);
 #pragma unroll
             for (int r = 0; r < S1M; ++r) {
                 int32_t t = 0;
@@ -77,7 +87,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                         }
                     }
                 }
-                tile_t[lane * S1M + r] = t;
+                tile_t[lane * S1M + r] = (int32_t)((seq_base + (uint32_t)t) * (uint32_t)a.hkv + h);
                 tile_lw[lane * S1M + r] = lw;
             }
         }
@@ -90,8 +100,6 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
                 if (row < rows) {
-                    uint32_t seq_base, h;
-                    a.map.split(row, seq_base, h);
                     const size_t qoff = (size_t)row * (G * TG::ROW) + c * 16;
 #pragma unroll
                     for (int g = 0; g < G; ++g) {
@@ -101,7 +109,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const uint32_t kvrow = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                            const uint32_t kvrow = (uint32_t)tile_t[lr * S1M + jj];
                             const size_t off = (size_t)kvrow * TG::ROW + c * 16;
                             cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
                             cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
@@ -141,6 +149,81 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
 #pragma unroll
                 for (int x = 0; x < NP; ++x) g2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
             }
+            float p[G][S1M], dz[G][S1M];
+            constexpr int NV = 2 * G * S1M;  // (slot, head) pairs of q.k and dO.v per row
+            if constexpr (NV <= C) {
+                // Distributed softmax: the NV partial dots are reduced across the row's C lanes
+                // by a transposed butterfly (each step sends half of the remaining values to the
+                // partner lane), so lane L of the segment ends with value vi = L / SPREAD,
+                // vi = 2 (slot * G + head) + {0: q.k, 1: dO.v}; the softmax, D and dz then take
+                // one (slot, head) per lane pair, and dz (and, per record, p) are broadcast.
+                constexpr int SPREAD = C / NV;
+                float v[NV];
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    float kf[VEC], vf[VEC];
+                    // an inactive slot's stage holds stale data: its values are masked below
+                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
+                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        v[(jj * G + g) * 2] = chunk_dot<NP>(q2[g], kf);
+                        v[(jj * G + g) * 2 + 1] = chunk_dot<NP>(g2[g], vf);
+                    }
+                }
+#pragma unroll
+                for (int cnt = NV, off = C / 2; cnt > 1; cnt >>= 1, off >>= 1) {
+                    const bool up = (lane & off) != 0;
+#pragma unroll
+                    for (int i = 0; i < cnt / 2; ++i) {
+                        const float send = up ? v[i] : v[i + cnt / 2];
+                        const float keep = up ? v[i + cnt / 2] : v[i];
+                        v[i] = keep + __shfl_xor_sync(FULL, send, off);
+                    }
+                }
+                float x = v[0];
+#pragma unroll
+                for (int off = SPREAD / 2; off > 0; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+                const int vi = (lane & (C - 1)) / SPREAD;
+                const float other = __shfl_xor_sync(FULL, x, SPREAD);
+                const bool is_dp = (vi & 1) != 0;
+                const float sc = is_dp ? other : x, dpv = is_dp ? x : other;
+                const float mylw = tile_lw[lr * S1M + (vi >> 1) / G];
+                const bool myact = valid && mylw != -INFINITY;
+                const float zz = myact ? fmaf(sc, sl2, mylw) : -INFINITY;
+                float m = zz;  // over the slots of this lane's head
+#pragma unroll
+                for (int off = 2 * G * SPREAD; off < C; off <<= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, off));
+                const float e = myact ? ex2(zz - m) : 0.0f;
+                float l = e, sdp = myact ? e * dpv : 0.0f;
+#pragma unroll
+                for (int off = 2 * G * SPREAD; off < C; off <<= 1) {
+                    l += __shfl_xor_sync(FULL, l, off);
+                    sdp += __shfl_xor_sync(FULL, sdp, off);
+                }
+                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                const float pj = e * inv;
+                const float dzj = pj * ((myact ? dpv : 0.0f) - sdp * inv);
+                const int seg = lane & ~(C - 1);
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const int src = seg + (jj * G + g) * 2 * SPREAD;
+                        dz[g][jj] = __shfl_sync(FULL, dzj, src);
+                        if constexpr (!GATHER) p[g][jj] = __shfl_sync(FULL, pj, src);
+                    }
+                if constexpr (GATHER) {
+                    // a record needs p of its own slot c only
+                    const int jc = c < S1M ? c : 0;
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float pc = __shfl_sync(FULL, pj, seg + (jc * G + g) * 2 * SPREAD);
+#pragma unroll
+                        for (int jj = 0; jj < S1M; ++jj) p[g][jj] = (jj == jc) ? pc : 0.0f;
+                    }
+                }
+            } else {
             // scores and dO.V per slot and head
             float z[G][S1M], dp[G][S1M];
 #pragma unroll
@@ -157,7 +240,6 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                 }
             }
             // softmax, D, dz
-            float p[G][S1M], dz[G][S1M];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 float m = z[g][0];
@@ -178,14 +260,13 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                     dz[g][jj] = p[g][jj] * (dp[g][jj] - Dd);
                 }
             }
+            }
             // dq = scale sum_j dz_j k_j ; scatter dK, dV ; dlogw
             float2 dq2[G][NP];
 #pragma unroll
             for (int g = 0; g < G; ++g)
 #pragma unroll
                 for (int x = 0; x < NP; ++x) dq2[g][x] = make_float2(0.0f, 0.0f);
-            uint32_t seq_base = 0, h = 0;
-            a.map.split(valid ? row : 0u, seq_base, h);
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
                 if (!act[jj]) continue;  // per lane; no shuffles below
@@ -206,7 +287,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                     }
                 }
                 if constexpr (!GATHER) {
-                    const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                    const uint32_t key = (uint32_t)tile_t[lr * S1M + jj];
                     const size_t off = (size_t)key * D + c * VEC;
 #pragma unroll
                     for (int x = 0; x < NP; x += 2) {
@@ -235,7 +316,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_tile_kernel(SeaBwdArgs a)
                     }
                 }
                 if (c < S1M && mine) {
-                    const uint32_t key = (seq_base + (uint32_t)tile_t[lr * S1M + c]) * (uint32_t)a.hkv + h;
+                    const uint32_t key = (uint32_t)tile_t[lr * S1M + c];
                     const int32_t pos = a.off[key] + atomicSub(a.cnt + key, 1) - 1;
                     // the count pass applies the same activity test, so pos stays inside the
                     // bucket; the bound only keeps a broken invariant from writing outside

@@ -141,6 +141,13 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
+// Resident blocks per SM the forward tile kernel is compiled for (shared memory allows about
+// five at the largest stage): caps registers at 65536 / (32 * WPB * MINB) without forcing
+// spills.
+#ifndef GM_TILE_MINB
+#define GM_TILE_MINB 4
+#endif
+
 template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static constexpr int VEC = Vec<T>::N;          // elements per 16-byte chunk
     static constexpr int C = D / (VEC * CPL);      // lanes per row (CPL chunks per lane)
@@ -157,14 +164,14 @@ template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
 // REFER = true: fused SER -> SEA (edges from the referral of sa's legs);
 // REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
 template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL>
-__global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
+__global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
     using TG = TileGeom<T, D, G, S1M, CPL>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
     static_assert(VEC % 2 == 0, "packed fp32x2 math");
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    // per warp: edge tile (t, log2 w) then P stages
+    // per warp: edge tile (K/V row, log2 w) then P stages
     constexpr int TILE_BYTES = 32 * S1M * 8;
     char *wbase = smem + (size_t)wid * (TILE_BYTES + P * TG::STAGE);
     int32_t *tile_t = reinterpret_cast<int32_t *>(wbase);
@@ -227,9 +234,13 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                     }
                 }
             }
+            // K/V row of each slot ((b*n + t)*hkv + h), so phase 2 issues its copies without
+            // decomposing the row again
+            uint32_t seq_base = 0, h = 0;
+            if (row < rows) a.map.split(row, seq_base, h);
 #pragma unroll
             for (int r = 0; r < S1M; ++r) {
-                tile_t[lane * S1M + r] = to[r];
+                tile_t[lane * S1M + r] = (int32_t)((seq_base + (uint32_t)to[r]) * (uint32_t)a.hkv + h);
                 tile_lw[lane * S1M + r] = wo[r] > 0.0f ? lg2(wo[r]) : -INFINITY;
             }
         }
@@ -242,8 +253,6 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
                 if (row < rows) {
-                    uint32_t seq_base, h;
-                    a.map.split(row, seq_base, h);
                     const char *qs = reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW);
 #pragma unroll
                     for (int g = 0; g < G; ++g)
@@ -253,7 +262,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const uint32_t kvrow = (seq_base + (uint32_t)tile_t[lr * S1M + jj]) * (uint32_t)a.hkv + h;
+                            const uint32_t kvrow = (uint32_t)tile_t[lr * S1M + jj];
 #pragma unroll
                             for (int cc = 0; cc < CPL; ++cc) {
                                 const size_t off = (size_t)kvrow * TG::ROW + (c * CPL + cc) * 16;
@@ -297,6 +306,91 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                     for (int x = 0; x < NP; ++x) q2[g][cc * NP + x] = make_float2(f[2 * x], f[2 * x + 1]);
                 }
             }
+            float2 acc[G][CPL * NP];
+            float m[G], l[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int x = 0; x < CPL * NP; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
+            constexpr int NV = G * S1M;  // (slot, head) scores per row
+            if constexpr (NV <= C) {
+                // Distributed softmax. The NV partial dots are reduced across the row's C lanes
+                // by a transposed butterfly: each step sends half of the remaining values to
+                // the partner lane and keeps the other half, so every lane adds the same pairs
+                // as a full butterfly (x + partner) and the totals carry its exact bits. Lane L
+                // of the segment ends with score vi = L / SPREAD (vi = slot * G + head); the
+                // max, exponential and sum then take one value per lane.
+                constexpr int SPREAD = C / NV;
+                float v[NV];
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    float kf[CPL * VEC];
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) {
+                        float f[VEC];
+                        // an inactive slot's stage holds stale data: its score is masked below
+                        unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16), f);
+#pragma unroll
+                        for (int x = 0; x < VEC; ++x) kf[cc * VEC + x] = f[x];
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; ++g) v[jj * G + g] = chunk_dot<CPL * NP>(q2[g], kf);
+                }
+#pragma unroll
+                for (int cnt = NV, off = C / 2; cnt > 1; cnt >>= 1, off >>= 1) {
+                    const bool up = (lane & off) != 0;
+#pragma unroll
+                    for (int i = 0; i < cnt / 2; ++i) {
+                        const float send = up ? v[i] : v[i + cnt / 2];
+                        const float keep = up ? v[i + cnt / 2] : v[i];
+                        v[i] = keep + __shfl_xor_sync(FULL, send, off);
+                    }
+                }
+                float x = v[0];
+#pragma unroll
+                for (int off = SPREAD / 2; off > 0; off >>= 1) x += __shfl_xor_sync(FULL, x, off);
+                const int vi = (lane & (C - 1)) / SPREAD;
+                const float mylw = tile_lw[lr * S1M + vi / G];
+                const bool myact = valid && mylw != -INFINITY;
+                const float z = myact ? fmaf(x, sl2, mylw) : -INFINITY;
+                float mz = z;  // max over the slots of this lane's head
+#pragma unroll
+                for (int off = G * SPREAD; off < C; off <<= 1) mz = fmaxf(mz, __shfl_xor_sync(FULL, mz, off));
+                const float p = myact ? ex2(z - mz) : 0.0f;
+                float lz = p;
+#pragma unroll
+                for (int off = G * SPREAD; off < C; off <<= 1) lz += __shfl_xor_sync(FULL, lz, off);
+                const int seg = lane & ~(C - 1);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    m[g] = __shfl_sync(FULL, mz, seg + g * SPREAD);
+                    l[g] = __shfl_sync(FULL, lz, seg + g * SPREAD);
+                }
+                float pp[S1M][G];
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj)
+#pragma unroll
+                    for (int g = 0; g < G; ++g) pp[jj][g] = __shfl_sync(FULL, p, seg + (jj * G + g) * SPREAD);
+#pragma unroll
+                for (int jj = 0; jj < S1M; ++jj) {
+                    if (!act[jj]) continue;  // per lane; no shuffles below
+                    float vf[CPL * VEC];
+#pragma unroll
+                    for (int cc = 0; cc < CPL; ++cc) {
+                        float f[VEC];
+                        unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + (c * CPL + cc) * 16), f);
+#pragma unroll
+                        for (int x2 = 0; x2 < VEC; ++x2) vf[cc * VEC + x2] = f[x2];
+                    }
+#pragma unroll
+                    for (int g = 0; g < G; ++g) {
+                        const float2 p2 = make_float2(pp[jj][g], pp[jj][g]);
+#pragma unroll
+                        for (int x2 = 0; x2 < CPL * NP; ++x2)
+                            acc[g][x2] = __ffma2_rn(p2, make_float2(vf[2 * x2], vf[2 * x2 + 1]), acc[g][x2]);
+                    }
+                }
+            } else {
             // scores (all S1M slots, masked after the reduction so shuffles stay uniform)
             float z[G][S1M];
 #pragma unroll
@@ -325,16 +419,12 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                 }
             }
             // softmax and weighted V per head
-            float2 acc[G][CPL * NP];
-            float m[G], l[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 m[g] = z[g][0];
 #pragma unroll
                 for (int jj = 1; jj < S1M; ++jj) m[g] = fmaxf(m[g], z[g][jj]);
                 l[g] = 0.0f;
-#pragma unroll
-                for (int x = 0; x < CPL * NP; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
             }
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
@@ -356,6 +446,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_fwd_tile_kernel(SerArgs sa, SeaA
                     for (int x = 0; x < CPL * NP; ++x)
                         acc[g][x] = __ffma2_rn(p2, make_float2(vf[2 * x], vf[2 * x + 1]), acc[g][x]);
                 }
+            }
             }
             if (valid) {
 #pragma unroll
