@@ -48,6 +48,12 @@ def _load():
         lib.oracle_leg_backward.restype = ctypes.c_int64
         lib.oracle_leg_backward.argtypes = [i32p, f32p, ci, ci, f32p, f32p, ctypes.c_int64,
                                             f32p, ci, f32p, ci, ci, ci, f64p, f64p, f64p]
+        lib.oracle_ser_refresh.restype = ctypes.c_int64
+        lib.oracle_ser_refresh.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci, i32p, f32p,
+                                           ci, ci, ci, ci]
+        lib.oracle_ser_refresh_backward.restype = ctypes.c_int64
+        lib.oracle_ser_refresh_backward.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci,
+                                                    f32p, ci, ci, ci, ci, ci, f64p, f64p, f64p]
         _lib = lib
     return _lib
 
@@ -209,3 +215,41 @@ def leg_backward(e_idx, e_w, mix1, mix2, g1, g2):
     if bad < 0:
         raise ValueError("k*s0 exceeds the oracle's candidate buffer")
     return dew, dm1, dm2, int(bad)
+
+
+def ser_refresh(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, s1: int):
+    """A' = Sparsify_s1(A1 A2 + F) per (b, i, h): the referral with refresh edges F [B,n,k,sf]
+    joining its candidates after the two-hop paths. Returns (idx int32, w fp32, bad_refs)."""
+    i1, w1 = _np(a1_idx, np.int32), _np(a1_w, np.float32)
+    i2, w2 = _np(a2_idx, np.int32), _np(a2_w, np.float32)
+    fi, fw = _np(f_idx, np.int32), _np(f_w, np.float32)
+    B, n, k, s2 = i1.shape
+    s3, sf = i2.shape[3], fi.shape[3]
+    assert i2.shape[:3] == (B, n, k) and fi.shape[:3] == (B, n, k) and fw.shape == fi.shape
+    out_i = np.zeros((B, n, k, s1), np.int32)
+    out_w = np.zeros((B, n, k, s1), np.float32)
+    bad = _load().oracle_ser_refresh(i1, w1, s2, i2, w2, s3, fi, fw, sf, out_i, out_w, s1, B, n, k)
+    if bad < 0:
+        raise ValueError("s2*s3 + sf exceeds the oracle's candidate buffer")
+    return out_i, out_w, int(bad)
+
+
+def ser_refresh_backward(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, gout, grad_is_log: bool = False):
+    """Gradients of the kept weights of ser_refresh w.r.t. both legs and the refresh weights.
+
+    Returns (dw1 [B,n,k,s2], dw2 [B,n,k,s3], dfw [B,n,k,sf], bad_refs), fp64.
+    """
+    i1, w1 = _np(a1_idx, np.int32), _np(a1_w, np.float32)
+    i2, w2 = _np(a2_idx, np.int32), _np(a2_w, np.float32)
+    fi, fw = _np(f_idx, np.int32), _np(f_w, np.float32)
+    g = _np(gout, np.float32)
+    B, n, k, s2 = i1.shape
+    s3, sf, s1 = i2.shape[3], fi.shape[3], g.shape[3]
+    dw1 = np.zeros(i1.shape, np.float64)
+    dw2 = np.zeros(i2.shape, np.float64)
+    dfw = np.zeros(fi.shape, np.float64)
+    bad = _load().oracle_ser_refresh_backward(i1, w1, s2, i2, w2, s3, fi, fw, sf, g, s1,
+                                              int(bool(grad_is_log)), B, n, k, dw1, dw2, dfw)
+    if bad < 0:
+        raise ValueError("s2*s3 + sf exceeds the oracle's candidate buffer")
+    return dw1, dw2, dfw, int(bad)

@@ -26,6 +26,9 @@
  *          absorbs underflowing edge indices.
  *   [MF4]  "Main Findings", bullet on more edges: the cross-edge mixing is full (every stored
  *          channel feeds every leg channel), so its cost grows as k^2.
+ *   [MF5]  "Main Findings", bullet on refresh and realignment: refresh edges help; same
+ *          section as [MPE2], last sentence: refresh edges come from the input edges or from
+ *          the top positions of the latest dense attention layer.
  *
  * Readings where the pages are silent (the CUDA library applies the same ones):
  *   R1  A1 and A2 share the edge channel h (leg mixing happens upstream).
@@ -59,6 +62,12 @@
  *       its coefficient: R3's dropping of zero products shapes the forward's candidate set,
  *       not the derivative. The gradient of the coefficients is returned per token,
  *       [B, n, k, k], also when they were shared (the caller sums it).
+ *   R13 refresh edges: a set F of extra edges per (b, i, h) (the original input edges, or the
+ *       top positions of a dense attention layer, produced upstream) joins the referral's
+ *       candidates after the s2*s3 two-hop paths, with its own weights: A' =
+ *       Sparsify_s1(A1 A2 + F). Candidate order: the paths in ascending c = a*s3 + e, then
+ *       the refresh slots in ascending f; merge, order and cut as R2-R5. A kept target's
+ *       merged weight passes its gradient unchanged to every refresh slot that reaches it.
  *
  * Layouts are contiguous row-major: features [B, n, H, d], edges [B, n, k, s].
  */
@@ -603,6 +612,142 @@ int64_t oracle_leg_backward(const int32_t *e_idx, const float *e_w, int s0, int 
                         const int c = ca / s0;
                         dew[tok * ks0 + ca] += gr * (double)mix[h * k + c];
                         dmix[h * k + c] += gr * (double)ew[ca];
+                    }
+                }
+            }
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * SER with refresh edges: A' = Sparsify_s1(A1 A2 + F)   [MPE2], [MF5]; readings R1-R5, R8, R13.
+ *
+ * Candidates of row (b, i, h): the s2*s3 two-hop paths exactly as oracle_ser forms them, then
+ * the sf refresh slots f_idx/f_w[b,i,h,f] (weight > 0, index in range) with their own weights.
+ * cand_src[x] records where candidate x came from: the path slot pair (a, e) as a*s3 + e with
+ * its second-leg row, or a refresh slot as -(f + 1).
+ * ---------------------------------------------------------------------------------------- */
+static int ser_refresh_candidates(const int32_t *a1_idx, const float *a1_w, int s2,
+                                  const int32_t *a2_idx, const float *a2_w, int s3,
+                                  const int32_t *f_idx, const float *f_w, int sf,
+                                  int64_t row, int64_t b, int h, int n, int k,
+                                  int32_t *cand_t, float *cand_u, int *cand_src,
+                                  int64_t *cand_r2, int64_t *bad)
+{
+    int nc = 0;
+    for (int a = 0; a < s2; ++a) {
+        const float w1 = a1_w[row * s2 + a];
+        if (!(w1 > 0.0f)) continue;
+        const int32_t j = a1_idx[row * s2 + a];
+        if (j < 0 || j >= n) { ++*bad; continue; }
+        const int64_t row_j = ((int64_t)b * n + j) * k + h;
+        for (int e = 0; e < s3; ++e) {
+            const float w2 = a2_w[row_j * s3 + e];
+            if (!(w2 > 0.0f)) continue;
+            const int32_t t = a2_idx[row_j * s3 + e];
+            if (t < 0 || t >= n) { ++*bad; continue; }
+            const float u = w1 * w2;
+            if (u == 0.0f) continue;
+            cand_t[nc] = t;
+            cand_u[nc] = u;
+            cand_src[nc] = a * s3 + e;
+            cand_r2[nc] = row_j * s3 + e;
+            ++nc;
+        }
+    }
+    for (int f = 0; f < sf; ++f) {
+        const float w = f_w[row * sf + f];
+        if (!(w > 0.0f)) continue;
+        const int32_t t = f_idx[row * sf + f];
+        if (t < 0 || t >= n) { ++*bad; continue; }
+        cand_t[nc] = t;
+        cand_u[nc] = w;
+        cand_src[nc] = -(f + 1);
+        cand_r2[nc] = -1;
+        ++nc;
+    }
+    return nc;
+}
+
+int64_t oracle_ser_refresh(const int32_t *a1_idx, const float *a1_w, int s2,
+                           const int32_t *a2_idx, const float *a2_w, int s3,
+                           const int32_t *f_idx, const float *f_w, int sf,
+                           int32_t *out_idx, float *out_w, int s1, int B, int n, int k)
+{
+    const int64_t rows = (int64_t)B * n * k;
+    int64_t bad = 0;
+    if (s2 * s3 + sf > ORACLE_MAX_CAND) return -1;
+
+#pragma omp parallel for schedule(static) reduction(+ : bad)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int h = (int)(row % k);
+        const int64_t b = row / ((int64_t)n * k);
+        int32_t cand_t[ORACLE_MAX_CAND], ut[ORACLE_MAX_CAND];
+        float cand_u[ORACLE_MAX_CAND], uw[ORACLE_MAX_CAND];
+        int cand_src[ORACLE_MAX_CAND];
+        int64_t cand_r2[ORACLE_MAX_CAND];
+        int64_t my_bad = 0;
+        const int nc = ser_refresh_candidates(a1_idx, a1_w, s2, a2_idx, a2_w, s3, f_idx, f_w, sf,
+                                              row, b, h, n, k, cand_t, cand_u, cand_src, cand_r2,
+                                              &my_bad);
+        bad += my_bad;
+        const int nu = merge_and_order(cand_t, cand_u, nc, ut, uw);
+        for (int r = 0; r < s1; ++r) {
+            out_idx[row * s1 + r] = r < nu ? ut[r] : 0;
+            out_w[row * s1 + r] = r < nu ? uw[r] : 0.0f;
+        }
+    }
+    return bad;
+}
+
+/* Backward of oracle_ser_refresh (R9, R13): for every candidate merged into a kept slot r,
+ *     a path (a, e):    dw1[b,i,h,a] += g_r * w2,  dw2[b,j,h,e] += g_r * w1
+ *     a refresh slot f: dfw[b,i,h,f] += g_r
+ * in fp64; g_r as oracle_ser_backward (divided by W_r when grad_is_log). */
+int64_t oracle_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                    const int32_t *a2_idx, const float *a2_w, int s3,
+                                    const int32_t *f_idx, const float *f_w, int sf,
+                                    const float *gout, int s1, int grad_is_log,
+                                    int B, int n, int k, double *dw1, double *dw2, double *dfw)
+{
+    int64_t bad = 0;
+    if (s2 * s3 + sf > ORACLE_MAX_CAND) return -1;
+
+#pragma omp parallel for schedule(dynamic, 1) reduction(+ : bad)
+    for (int64_t plane = 0; plane < (int64_t)B * k; ++plane) {
+        const int64_t b = plane / k;
+        const int h = (int)(plane % k);
+        for (int i = 0; i < n; ++i) {
+            const int64_t row = ((int64_t)b * n + i) * k + h;
+            for (int a = 0; a < s2; ++a) dw1[row * s2 + a] = 0.0;
+            for (int e = 0; e < s3; ++e) dw2[row * s3 + e] = 0.0;
+            for (int f = 0; f < sf; ++f) dfw[row * sf + f] = 0.0;
+        }
+        for (int i = 0; i < n; ++i) {
+            const int64_t row = ((int64_t)b * n + i) * k + h;
+            int32_t cand_t[ORACLE_MAX_CAND], ut[ORACLE_MAX_CAND];
+            float cand_u[ORACLE_MAX_CAND], uw[ORACLE_MAX_CAND];
+            int cand_src[ORACLE_MAX_CAND];
+            int64_t cand_r2[ORACLE_MAX_CAND];
+            int64_t my_bad = 0;
+            const int nc = ser_refresh_candidates(a1_idx, a1_w, s2, a2_idx, a2_w, s3, f_idx, f_w,
+                                                  sf, row, b, h, n, k, cand_t, cand_u, cand_src,
+                                                  cand_r2, &my_bad);
+            bad += my_bad;
+            const int nu = merge_and_order(cand_t, cand_u, nc, ut, uw);
+            const int kept = nu < s1 ? nu : s1;
+            for (int r = 0; r < kept; ++r) {
+                double g = (double)gout[row * s1 + r];
+                if (grad_is_log) g /= (double)uw[r];
+                for (int x = 0; x < nc; ++x) {
+                    if (cand_t[x] != ut[r]) continue;
+                    if (cand_src[x] < 0) {
+                        dfw[row * sf + (-cand_src[x] - 1)] += g;
+                    } else {
+                        const int a = cand_src[x] / s3;
+                        dw1[row * s2 + a] += g * (double)a2_w[cand_r2[x]];
+                        dw2[cand_r2[x]] += g * (double)a1_w[row * s2 + a];
                     }
                 }
             }
