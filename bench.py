@@ -395,7 +395,7 @@ def run_ours(args):
 
     extra = None
     if not args.no_extra:
-        extra = measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak)
+        extra = measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak)
 
     e2e = None
     if not args.no_e2e:
@@ -433,13 +433,15 @@ def run_ours(args):
     return result
 
 
-def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
+def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     """The calls around the step, each timed alone with CUDA events, L2 flushed between reps.
 
     leg_sparsify builds the step's two legs from the workload's stored edges; ser_backward
     takes the step's d ln w back to the legs; leg_backward takes those leg gradients back to
-    the stored weights and the mixing coefficients. Bytes are compulsory: every input read
-    once, every output written once (ser_backward's second-leg rows counted in full).
+    the stored weights and the mixing coefficients; ser_sea_refresh_forward is the fused
+    forward with the stored edges joining the referral as refresh edges. Bytes are
+    compulsory: every input read once, every output written once (ser_backward's second-leg
+    rows counted in full; the refresh forward's gathered rows counted from its own edges).
     """
     le = {k: v.to(dev) for k, v in I.leg_inputs(wl).items()}
     B, n, k = wl.B, wl.n, wl.hkv
@@ -457,6 +459,16 @@ def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     # L2 is evicted by reading a 256 MB buffer (a write would leave dirty lines whose
     # write-back the next timed call would pay for)
     flush = torch.zeros(64 << 20, dtype=torch.int32, device=dev)
+    rf_i = torch.empty_like(ap_i)
+    rf_w = torch.empty_like(ap_w)
+    rf_o = torch.empty_like(g["q"])
+    rf_lse = torch.empty((B, n, wl.hq), dtype=f32, device=dev)
+    gm.gm_ser_sea_refresh_forward(g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], g["a2_idx"],
+                                  g["a2_w"], le["e_idx"], le["e_w"], wl.s1, wl.scale, out_idx=rf_i,
+                                  out_w=rf_w, o=rf_o, lse=rf_lse, stream=stream)
+    torch.cuda.synchronize(dev)
+    rf_bytes = (compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), rf_i.cpu().numpy(),
+                                 rf_w.cpu().numpy())["fused_forward"] + e_b_refresh(wl))
     e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
     leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
     calls = {
@@ -468,6 +480,12 @@ def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
                          lambda: gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"],
                                                     dlw, grad_is_log=True, dw1=dw1, dw2=dw2,
                                                     stream=stream)),
+        "ser_sea_refresh_forward": ("sea_fwd_tile_kernel (fused SER->SEA, refresh candidates)", rf_bytes,
+                                    lambda: gm.gm_ser_sea_refresh_forward(
+                                        g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], g["a2_idx"],
+                                        g["a2_w"], le["e_idx"], le["e_w"], wl.s1, wl.scale,
+                                        out_idx=rf_i, out_w=rf_w, o=rf_o, lse=rf_lse,
+                                        stream=stream)),
         "leg_backward": ("leg_bwd_tile_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
                          lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,
@@ -497,6 +515,11 @@ def measure_extra(gm, wl, g, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     out["note"] = ("timed alone, median of %d reps, L2 flushed (256 MB read) before each; "
                    "not part of the step's value" % reps)
     return out
+
+
+def e_b_refresh(wl: I.Workload) -> int:
+    """Bytes of a refresh edge set [B, n, hkv, s1] (int32 index + fp32 weight per slot)."""
+    return wl.B * wl.n * wl.hkv * wl.s1 * 8
 
 
 def measure_e2e(gm, wl, x, dev, stream, steps, world):

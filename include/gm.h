@@ -189,6 +189,63 @@ gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
                           cudaStream_t stream);
 
 /*
+ * gm_ser_refresh_forward - referral with refresh edges, A' = Sparsify_s1(A1 A2 + F).
+ * Source: ai.info summary, "Methodology in Plain English", referral paragraph (optional refresh
+ * edges pull in the input edges or the top positions of the latest dense attention layer) and
+ * "Main Findings", bullet on refresh and realignment (they help). The pages give no formula;
+ * the reading here: the refresh edges are one more sparse edge set that joins the referral's
+ * candidates before the cut.
+ *
+ * As gm_ser_forward, with sf refresh candidates after the s2*s3 two-hop paths: candidate
+ * s2*s3 + f of row (b,i,h) is (f_idx[b,i,h,f], f_w[b,i,h,f]) with its own weight (weight > 0;
+ * zero weights are dropped). Merge (fp32, ascending candidate order), order and cut as
+ * gm_ser_forward; bit-identical to that definition.
+ *
+ *   f_idx, f_w  device, [B, n, k, sf]   refresh edges (int32 targets, fp32 weights >= 0)
+ *   other arguments as gm_ser_forward
+ *   limits      1 <= sf, s2*s3 + sf <= 32, 1 <= s1 <= 32
+ * An active refresh slot whose index lies outside [0, n) is skipped and raises the device
+ * index-range flag.
+ */
+gm_status gm_ser_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                 const int32_t *a2_idx, const float *a2_w, int s3,
+                                 const int32_t *f_idx, const float *f_w, int sf,
+                                 int32_t *out_idx, float *out_w, int s1,
+                                 int B, int n, int k, cudaStream_t stream);
+
+/*
+ * gm_ser_refresh_backward - gradients of gm_ser_refresh_forward's kept weights with respect to
+ * both legs' weights and the refresh weights.
+ * Source: as gm_ser_refresh_forward; only retained weights get gradients (referral paragraph).
+ *
+ * As gm_ser_backward for the path candidates; a refresh slot f whose target was kept in slot r
+ * receives dfw[b,i,h,f] = g_r (the merged weight is a plain sum of it). Cut targets get nothing.
+ *
+ *   f_idx, f_w, sf   as gm_ser_refresh_forward
+ *   dfw              device fp32 [B, n, k, sf], written (added to if accumulate)
+ *   other arguments as gm_ser_backward
+ */
+gm_status gm_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                  const int32_t *a2_idx, const float *a2_w, int s3,
+                                  const int32_t *f_idx, const float *f_w, int sf,
+                                  const float *gout, int s1, int grad_is_log,
+                                  int B, int n, int k, float *dw1, float *dw2, float *dfw,
+                                  int accumulate, cudaStream_t stream);
+
+/*
+ * gm_ser_sea_refresh_forward - gm_ser_refresh_forward followed by gm_sea_forward on its result,
+ * in one kernel (as gm_ser_sea_forward, with the refresh edges f_idx/f_w/sf of
+ * gm_ser_refresh_forward). Same arguments, limits and results as the two calls in sequence.
+ */
+gm_status gm_ser_sea_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                     const int32_t *a2_idx, const float *a2_w, int s3,
+                                     const int32_t *f_idx, const float *f_w, int sf,
+                                     int32_t *out_idx, float *out_w, int s1,
+                                     const void *q, const void *k, const void *v, gm_dtype dtype,
+                                     int B, int n, int hq, int hkv, int d, float scale,
+                                     void *o, float *lse, cudaStream_t stream);
+
+/*
  * gm_sea_forward - sparse edge attention.
  * Source: ai.info summary, "Key Contributions" item 3 (SEA: edge indices select the K/V
  * positions; node factor = scaled q.k, edge factor = log edge weight, combined as a product

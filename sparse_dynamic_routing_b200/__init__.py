@@ -6,6 +6,8 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_leg_sparsify     both referral legs from the stored edges (mixed, then sparsified)
     gm_leg_backward     gradients of the kept leg weights
     gm_ser_forward      sparse edge referral, A' = Sparsify_s1(A1 A2)
+    gm_ser_refresh_forward / _backward, gm_ser_sea_refresh_forward
+                        the referral with refresh edges, A' = Sparsify_s1(A1 A2 + F)
     gm_sea_forward      sparse edge attention
     gm_ser_sea_forward  both in one kernel
     gm_sea_backward     gradients of sparse edge attention
@@ -26,6 +28,9 @@ from ._binding import (  # noqa: F401
     gm_sea_forward,
     gm_ser_backward,
     gm_ser_forward,
+    gm_ser_refresh_backward,
+    gm_ser_refresh_forward,
+    gm_ser_sea_refresh_forward,
     gm_ser_sea_forward,
     gm_version,
     load_library,

@@ -29,6 +29,12 @@ SIGNATURES = {
     "gm_leg_backward": [_vp, _vp, _ci, _vp, _vp, ctypes.c_int64, _vp, _ci, _vp, _ci, _ci, _ci,
                         _ci, _vp, _vp, _vp, _ci, _vp],
     "gm_ser_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
+    "gm_ser_refresh_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci,
+                               _ci, _vp],
+    "gm_ser_refresh_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci,
+                                _ci, _vp, _vp, _vp, _ci, _vp],
+    "gm_ser_sea_refresh_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp,
+                                   _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp],
     "gm_ser_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _vp, _vp, _ci,
                         _vp],
     "gm_sea_forward": [_vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp,
@@ -219,6 +225,89 @@ def gm_ser_backward(a1_idx, a1_w, a2_idx, a2_w, gout, grad_is_log=False, dw1=Non
         _ptr(dw1, f32, "dw1"), _ptr(dw2, f32, "dw2"), int(bool(accumulate)), _stream(stream))
     _check(st, "gm_ser_backward")
     return dw1, dw2
+
+
+def _refresh_shapes(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w):
+    B, n, k, s2 = a1_idx.shape
+    s3, sf = a2_idx.shape[3], f_idx.shape[3]
+    if a2_idx.shape[:3] != (B, n, k) or f_idx.shape[:3] != (B, n, k):
+        raise ValueError("edge tensor shapes disagree")
+    if a1_w.shape != a1_idx.shape or a2_w.shape != a2_idx.shape or f_w.shape != f_idx.shape:
+        raise ValueError("edge weight shapes disagree with their indices")
+    return B, n, k, s2, s3, sf
+
+
+def gm_ser_refresh_forward(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, s1: int, out_idx=None,
+                           out_w=None, stream=None):
+    """Referral with refresh edges, A' = Sparsify_s1(A1 A2 + F). Returns (out_idx, out_w)."""
+    B, n, k, s2, s3, sf = _refresh_shapes(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w)
+    dev = a1_idx.device
+    i32, f32 = torch.int32, torch.float32
+    out_idx = torch.empty((B, n, k, s1), dtype=i32, device=dev) if out_idx is None else out_idx
+    out_w = torch.empty((B, n, k, s1), dtype=f32, device=dev) if out_w is None else out_w
+    st = load_library().gm_ser_refresh_forward(
+        _ptr(a1_idx, i32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, i32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3,
+        _ptr(f_idx, i32, "f_idx"), _ptr(f_w, f32, "f_w"), sf,
+        _ptr(out_idx, i32, "out_idx"), _ptr(out_w, f32, "out_w"), s1, B, n, k, _stream(stream))
+    _check(st, "gm_ser_refresh_forward")
+    return out_idx, out_w
+
+
+def gm_ser_refresh_backward(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, gout, grad_is_log=False,
+                            dw1=None, dw2=None, dfw=None, accumulate=False, stream=None):
+    """Gradients of the kept weights of the referral with refresh edges. Returns (dw1, dw2, dfw)."""
+    B, n, k, s2, s3, sf = _refresh_shapes(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w)
+    s1 = gout.shape[3]
+    if tuple(gout.shape[:3]) != (B, n, k):
+        raise ValueError("gout must be [B, n, k, s1]")
+    dev = a1_idx.device
+    i32, f32 = torch.int32, torch.float32
+    dw1 = torch.empty((B, n, k, s2), dtype=f32, device=dev) if dw1 is None else dw1
+    dw2 = torch.empty((B, n, k, s3), dtype=f32, device=dev) if dw2 is None else dw2
+    dfw = torch.empty((B, n, k, sf), dtype=f32, device=dev) if dfw is None else dfw
+    st = load_library().gm_ser_refresh_backward(
+        _ptr(a1_idx, i32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, i32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3,
+        _ptr(f_idx, i32, "f_idx"), _ptr(f_w, f32, "f_w"), sf,
+        _ptr(gout, f32, "gout"), s1, int(bool(grad_is_log)), B, n, k,
+        _ptr(dw1, f32, "dw1"), _ptr(dw2, f32, "dw2"), _ptr(dfw, f32, "dfw"),
+        int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_ser_refresh_backward")
+    return dw1, dw2, dfw
+
+
+def gm_ser_sea_refresh_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, s1: int,
+                               scale=None, out_idx=None, out_w=None, o=None, lse=None,
+                               want_edges=True, want_lse=True, stream=None):
+    """Fused referral with refresh edges -> SEA forward. Returns (out_idx, out_w, o, lse)."""
+    B, n, hq, d = q.shape
+    hkv = k.shape[2]
+    _, _, kk, s2, s3, sf = _refresh_shapes(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w)
+    if kk != hkv or tuple(a1_idx.shape[:2]) != (B, n):
+        raise ValueError("edge tensors must be [B, n, hkv, s]")
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape:
+        raise ValueError("k/v shapes disagree with q")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("q, k, v must share a dtype")
+    dev = q.device
+    i32, f32 = torch.int32, torch.float32
+    if want_edges:
+        out_idx = torch.empty((B, n, hkv, s1), dtype=i32, device=dev) if out_idx is None else out_idx
+        out_w = torch.empty((B, n, hkv, s1), dtype=f32, device=dev) if out_w is None else out_w
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty((B, n, hq), dtype=f32, device=dev)
+    st = load_library().gm_ser_sea_refresh_forward(
+        _ptr(a1_idx, i32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, i32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3,
+        _ptr(f_idx, i32, "f_idx"), _ptr(f_w, f32, "f_w"), sf,
+        _ptr(out_idx, i32, "out_idx"), _ptr(out_w, f32, "out_w"), s1,
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _fdtype(q),
+        B, n, hq, hkv, d, _scale(scale, d), _ptr(o, q.dtype, "o"), _ptr(lse, f32, "lse"),
+        _stream(stream))
+    _check(st, "gm_ser_sea_refresh_forward")
+    return out_idx, out_w, o, lse
 
 
 def gm_sea_forward(q, k, v, idx, w, scale=None, o=None, lse=None, want_lse=True, stream=None):

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/gm.h"
 #include "gm_bwd_gather.cuh"
@@ -51,6 +52,14 @@ gm_status check_ser(const int32_t *a1_idx, const float *a1_w, int s2, const int3
     if ((int64_t)B * n == 0) return GM_OK;
     if ((int64_t)B * n * k >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
     if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
+    return GM_OK;
+}
+
+// Refresh edges of the referral: sf slots per row joining the s2*s3 path candidates.
+gm_status check_refresh(const int32_t *f_idx, const float *f_w, int sf, int s2, int s3, int64_t rows)
+{
+    if (sf < 1 || s2 * s3 + sf > MAX_SLOTS) return GM_ERR_INVALID_ARG;
+    if (rows > 0 && (!f_idx || !f_w)) return GM_ERR_INVALID_ARG;
     return GM_OK;
 }
 
@@ -190,11 +199,11 @@ template <typename T, int D, int G> struct TileOK {
     static constexpr bool value = (D == 64 || D == 128) && D / VEC >= 2 && D / VEC <= 16 && VEC * G <= 16;
 };
 
-template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M>
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int SF = 0>
 gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
 {
     using TG = gm::TileGeom<T, D, G, S1M, TILE_CPL>;
-    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL>;
+    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL, SF>;
     const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -211,13 +220,24 @@ template <typename T, int D, int G> struct SerSeaFwd {
         if constexpr (TileOK<T, D, G>::value) {
             const bool aligned = aligned16(sa.a1_idx) && aligned16(sa.a1_w) && aligned16(sa.a2_idx) &&
                                  aligned16(sa.a2_w) && aligned16(sa.out_idx) && aligned16(sa.out_w);
-            if (aligned && sa.s2 == 2 && sa.s3 == 2) {
+            if (aligned && sa.sf == 0 && sa.s2 == 2 && sa.s3 == 2) {
                 if (sa.s1 <= 2) return launch_tile<T, D, G, true, 2, 2, 2>(sa, a, st);
                 if (sa.s1 <= 4) return launch_tile<T, D, G, true, 2, 2, 4>(sa, a, st);
             }
-            if (aligned && sa.s2 == 4 && sa.s3 == 4) {
+            if (aligned && sa.sf == 0 && sa.s2 == 4 && sa.s3 == 4) {
                 if (sa.s1 <= 2) return launch_tile<T, D, G, true, 4, 4, 2>(sa, a, st);
                 if (sa.s1 <= 4) return launch_tile<T, D, G, true, 4, 4, 4>(sa, a, st);
+            }
+            // refresh edges: bf16 features, budgets 2 or 4, s1 <= 4, sf in {2, 4}
+            if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                if (aligned && sa.sf > 0 && aligned16(sa.f_idx) && aligned16(sa.f_w) && sa.s1 <= 4 &&
+                    sa.s2 == sa.s3 && (sa.s2 == 2 || sa.s2 == 4) && (sa.sf == 2 || sa.sf == 4)) {
+                    if (sa.s2 == 2)
+                        return sa.sf == 2 ? launch_tile<T, D, G, true, 2, 2, 4, 2>(sa, a, st)
+                                          : launch_tile<T, D, G, true, 2, 2, 4, 4>(sa, a, st);
+                    return sa.sf == 2 ? launch_tile<T, D, G, true, 4, 4, 4, 2>(sa, a, st)
+                                      : launch_tile<T, D, G, true, 4, 4, 4, 4>(sa, a, st);
+                }
             }
         }
         gm::ser_sea_fwd_kernel<T, D, G, WPB_SEA><<<blocks_for(a.rows, WPB_SEA), WPB_SEA * 32, 0, st>>>(sa, a);
@@ -505,6 +525,73 @@ gm_status gm_leg_backward(const int32_t *e_idx, const float *e_w, int s0,
     if (tile != GM_ERR_UNSUPPORTED) return tile;
     gm::leg_bwd_kernel<WPB_LEG><<<blocks_for(a.tokens, WPB_LEG), WPB_LEG * 32, 0, stream>>>(a);
     return launched();
+}
+
+gm_status gm_ser_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                 const int32_t *a2_idx, const float *a2_w, int s3,
+                                 const int32_t *f_idx, const float *f_w, int sf,
+                                 int32_t *out_idx, float *out_w, int s1,
+                                 int B, int n, int k, cudaStream_t stream)
+{
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, k);
+    if (st != GM_OK) return st;
+    st = check_refresh(f_idx, f_w, sf, s2, s3, (int64_t)B * n);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
+    SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k,
+              (uint32_t)((int64_t)B * n * k), row_map(k, n), f_idx, f_w, sf};
+    gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
+    return launched();
+}
+
+gm_status gm_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                  const int32_t *a2_idx, const float *a2_w, int s3,
+                                  const int32_t *f_idx, const float *f_w, int sf,
+                                  const float *gout, int s1, int grad_is_log,
+                                  int B, int n, int k, float *dw1, float *dw2, float *dfw,
+                                  int accumulate, cudaStream_t stream)
+{
+    if ((grad_is_log != 0 && grad_is_log != 1) || (accumulate != 0 && accumulate != 1)) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, k);
+    if (st != GM_OK) return st;
+    st = check_refresh(f_idx, f_w, sf, s2, s3, (int64_t)B * n);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!gout || !dw1 || !dw2 || !dfw) return GM_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * n * k;
+    if (!accumulate) {
+        gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dw2), rows * s3);
+        if (launched() != GM_OK) return GM_ERR_CUDA;
+    }
+    const SerArgs f{a1_idx, a1_w, a2_idx, a2_w, nullptr, nullptr, s1, s2, s3, n, k, (uint32_t)rows,
+                    row_map(k, n), f_idx, f_w, sf};
+    const gm::SerBwdArgs b{f, gout, grad_is_log, dw1, dw2, accumulate, dfw};
+    gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
+    return launched();
+}
+
+gm_status gm_ser_sea_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                     const int32_t *a2_idx, const float *a2_w, int s3,
+                                     const int32_t *f_idx, const float *f_w, int sf,
+                                     int32_t *out_idx, float *out_w, int s1,
+                                     const void *q, const void *k, const void *v, gm_dtype dtype,
+                                     int B, int n, int hq, int hkv, int d, float scale,
+                                     void *o, float *lse, cudaStream_t stream)
+{
+    if ((out_idx == nullptr) != (out_w == nullptr)) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, hkv);
+    if (st != GM_OK) return st;
+    st = check_refresh(f_idx, f_w, sf, s2, s3, (int64_t)B * n);
+    if (st != GM_OK) return st;
+    const int32_t dummy_idx = 0;
+    const float dummy_w = 0.0f;
+    st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    const uint32_t rows = (uint32_t)((int64_t)B * n * hkv);
+    SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows, row_map(hkv, n),
+               f_idx, f_w, sf};
+    SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows, row_map(hkv, n)};
+    return dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
 }
 
 gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype dtype,

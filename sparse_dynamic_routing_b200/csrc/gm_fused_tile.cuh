@@ -57,29 +57,30 @@ template <int S> __device__ __forceinline__ void ld_vec(const float *p, float (&
 // Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when both
 // are still nonzero and share a target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
 // group's members are thus added to its first occurrence in ascending candidate order.
-// Unrolled by template recursion so the candidate arrays stay in registers.
-template <int C0, int C2, int NC>
+// Unrolled (template recursion over c, an unrolled loop over c2) so the candidate arrays
+// stay in registers.
+template <int C0, int NC>
 __device__ __forceinline__ void merge_pairs(const int32_t (&ct)[NC], float (&cu)[NC])
 {
     if constexpr (C0 < NC - 1) {
-        if constexpr (C2 < NC) {
-            const bool same = cu[C0] != 0.0f && cu[C2] != 0.0f && ct[C2] == ct[C0];
-            cu[C0] = same ? __fadd_rn(cu[C0], cu[C2]) : cu[C0];
-            cu[C2] = same ? 0.0f : cu[C2];
-            merge_pairs<C0, C2 + 1, NC>(ct, cu);
-        } else {
-            merge_pairs<C0 + 1, C0 + 2, NC>(ct, cu);
+#pragma unroll
+        for (int c2 = C0 + 1; c2 < NC; ++c2) {
+            const bool same = cu[C0] != 0.0f && cu[c2] != 0.0f && ct[c2] == ct[C0];
+            cu[C0] = same ? __fadd_rn(cu[C0], cu[c2]) : cu[C0];
+            cu[c2] = same ? 0.0f : cu[c2];
         }
+        merge_pairs<C0 + 1, NC>(ct, cu);
     }
 }
 
 // Referral of one edge row by one thread (exact S2, S3; s1 <= S1M). Slots r >= s1 and slots
-// beyond the number of distinct targets come back as (0, 0.0f).
-template <int S2, int S3, int S1M>
+// beyond the number of distinct targets come back as (0, 0.0f). SF > 0: the row's SF refresh
+// edges (a.sf == SF) join the candidates after the S2*S3 paths, with their own weights.
+template <int S2, int S3, int S1M, int SF = 0>
 __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32_t (&to)[S1M],
                                            float (&wo)[S1M])
 {
-    constexpr int NC = S2 * S3;
+    constexpr int NP2 = S2 * S3, NC = NP2 + SF;
     uint32_t seq_base, h;
     a.map.split(row, seq_base, h);
     int32_t j[S2];
@@ -119,8 +120,24 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
             cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
         }
     }
+    if constexpr (SF > 0) {
+        int32_t tf[SF];
+        float wf[SF];
+        ld_vec<SF>(a.f_idx + (size_t)row * SF, tf);
+        ld_vec<SF>(a.f_w + (size_t)row * SF, wf);
+#pragma unroll
+        for (int f = 0; f < SF; ++f) {
+            bool v = wf[f] > 0.0f;
+            if (v && (tf[f] < 0 || tf[f] >= a.n)) {
+                raise_index_error();
+                v = false;
+            }
+            ct[NP2 + f] = tf[f];
+            cu[NP2 + f] = v ? wf[f] : 0.0f;
+        }
+    }
     // merge: the first occurrence of a target absorbs the later ones, in ascending order
-    merge_pairs<0, 1, NC>(ct, cu);
+    merge_pairs<0, NC>(ct, cu);
     // top-s1: repeated arg-max by (weight desc, index asc); the winner is then removed by
     // value (nonzero targets are distinct after the merge, so the match is unique)
 #pragma unroll
@@ -161,9 +178,11 @@ template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
 };
 
-// REFER = true: fused SER -> SEA (edges from the referral of sa's legs);
+// REFER = true: fused SER -> SEA (edges from the referral of sa's legs, plus SF refresh edges
+// per row when SF > 0);
 // REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
-template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL>
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL,
+          int SF = 0>
 __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
     using TG = TileGeom<T, D, G, S1M, CPL>;
@@ -218,7 +237,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(Se
                     }
                 }
             } else if (row < rows) {
-                ser_thread<S2, S3, S1M>(sa, row, to, wo);
+                ser_thread<S2, S3, S1M, SF>(sa, row, to, wo);
                 if (sa.out_idx != nullptr) {
                     if (sa.s1 == S1M && S1M == 4) {
                         *reinterpret_cast<int4 *>(sa.out_idx + (size_t)row * 4) = make_int4(to[0], to[1], to[2], to[3]);

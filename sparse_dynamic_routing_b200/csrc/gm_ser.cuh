@@ -3,7 +3,9 @@
 // "Graph Machine: Towards Better Pretraining via Edges" (ai.info summary), "Key
 // Contributions" item 3 and "Methodology in Plain English", referral paragraph:
 // A' = Sparsify_s1(A1 A2). Lane c < s2*s3 owns candidate c = a*s3 + e, i.e. the two-hop
-// path i -> j = A1.idx[a] -> t = A2[j].idx[e] with weight fl32(A1.w[a] * A2[j].w[e]).
+// path i -> j = A1.idx[a] -> t = A2[j].idx[e] with weight fl32(A1.w[a] * A2[j].w[e]). With
+// refresh edges F ("Methodology in Plain English", referral paragraph, last sentence), lane
+// s2*s3 + f owns refresh slot f with its own weight: A' = Sparsify_s1(A1 A2 + F).
 // Duplicates are merged with __match_any_sync: the lowest lane of each group of equal
 // targets sums the group's weights in ascending lane (= candidate) order with __fadd_rn.
 // Top-s1 is s1 rounds of a two-stage warp max (REDUX) on the key (weight bits, ~index):
@@ -27,6 +29,10 @@ struct SerArgs {
     int n, k;
     uint32_t rows;  // B * n * k
     RowMap map;     // heads = k
+    // refresh edges [rows, sf] joining the candidates after the two-hop paths (sf = 0: none)
+    const int32_t *f_idx;
+    const float *f_w;
+    int sf;
 };
 
 // Referral of one edge row. On return lane r < s1 holds the r-th kept (t, W); other lanes
@@ -67,6 +73,20 @@ __device__ __forceinline__ void ser_row(const SerArgs &a, uint32_t row, uint32_t
             } else {
                 u = __fmul_rn(w1, w2);
                 t = t2;
+            }
+        }
+    }
+    // refresh lanes nc <= lane < nc + sf: candidate nc + f is refresh slot f with its own weight
+    if (lane >= nc && lane < nc + a.sf) {
+        const size_t rf = (size_t)row * a.sf + (lane - nc);
+        const float wf = __ldg(a.f_w + rf);
+        const int32_t tf = __ldg(a.f_idx + rf);
+        if (wf > 0.0f) {
+            if (tf < 0 || tf >= a.n) {
+                raise_index_error();
+            } else {
+                u = wf;
+                t = tf;
             }
         }
     }

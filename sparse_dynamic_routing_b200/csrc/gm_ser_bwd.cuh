@@ -26,6 +26,7 @@ struct SerBwdArgs {
     float *dw1;          // [rows, s2]
     float *dw2;          // [rows, s3]
     int accumulate;
+    float *dfw;          // [rows, sf] when the forward had refresh edges
 };
 
 template <int WPB>
@@ -67,6 +68,20 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
             } else {
                 u = __fmul_rn(w1, w2);
                 t = t2;
+            }
+        }
+    }
+    const bool refresh = lane >= nc && lane < nc + a.sf;  // refresh slot lane - nc
+    if (refresh) {
+        const size_t rf = (size_t)row * a.sf + (lane - nc);
+        const float wf = __ldg(a.f_w + rf);
+        const int32_t tf = __ldg(a.f_idx + rf);
+        if (wf > 0.0f) {
+            if (tf < 0 || tf >= a.n) {
+                raise_index_error();
+            } else {
+                u = wf;
+                t = tf;
             }
         }
     }
@@ -116,7 +131,12 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
         *p = b.accumulate ? *p + d1 : d1;
     }
     // ---- second leg: scatter to the shared second-leg rows ----------------------------------------
-    if (slot >= 0) atomicAdd(b.dw2 + r2, g * w1);
+    if (slot >= 0 && lane < nc) atomicAdd(b.dw2 + r2, g * w1);
+    // ---- refresh slots: d W / d w_f = 1 -------------------------------------------------------------
+    if (refresh) {
+        float *p = b.dfw + (size_t)row * a.sf + (lane - nc);
+        *p = b.accumulate ? *p + g : g;
+    }
 }
 
 // The same backward, one thread per edge row, for small exact budgets (S2, S3; s1 <= S1M):
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
     bool cand[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) cand[c] = cu[c] != 0.0f;
-    merge_pairs<0, 1, NC>(ct, cu);
+    merge_pairs<0, NC>(ct, cu);
     // selection (weight desc, target asc) and the upstream gradient of each kept slot
     int32_t kt[S1M];
     float kg[S1M];

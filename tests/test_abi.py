@@ -159,3 +159,24 @@ def test_leg_argument_checks(lib):
     assert g(FAKE, FAKE, 4, FAKE, FAKE, 64, FAKE, 4, FAKE, 4, 1, 8, 8, FAKE, FAKE, FAKE, 2, NULL) == bnd.GM_ERR_INVALID_ARG
     assert g(FAKE, FAKE, 9, FAKE, FAKE, 64, FAKE, 4, FAKE, 4, 1, 8, 8, FAKE, FAKE, FAKE, 0, NULL) == bnd.GM_ERR_INVALID_ARG
     assert g(NULL, NULL, 4, NULL, NULL, 0, NULL, 4, NULL, 4, 3, 0, 8, NULL, NULL, NULL, 0, NULL) == bnd.GM_OK
+
+
+def test_refresh_argument_checks(lib):
+    f = lib.gm_ser_refresh_forward
+    # a1_idx, a1_w, s2, a2_idx, a2_w, s3, f_idx, f_w, sf, out_idx, out_w, s1, B, n, k, stream
+    assert f(FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, FAKE, 0, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, FAKE, 17, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, FAKE, FAKE, 4, NULL, FAKE, 4, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, FAKE, FAKE, 4, FAKE, FAKE, 4, NULL, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    g = lib.gm_ser_refresh_backward
+    # ..., f_idx, f_w, sf, gout, s1, grad_is_log, B, n, k, dw1, dw2, dfw, accumulate, stream
+    assert g(FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, 2, 0, 1, 8, 2, FAKE, FAKE, NULL, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, 2, 3, 1, 8, 2, FAKE, FAKE, FAKE, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+    h = lib.gm_ser_sea_refresh_forward
+    base = [FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, FAKE, 2, FAKE, FAKE, FAKE,
+            bnd.GM_BF16, 1, 8, 4, 2, 128, 0.1, FAKE + 1, NULL, NULL]  # o misaligned
+    assert h(*base) == bnd.GM_ERR_INVALID_ARG
+    a = list(base)
+    a[8] = 31  # s2*s3 + sf > 32
+    a[22] = FAKE
+    assert h(*a) == bnd.GM_ERR_INVALID_ARG
