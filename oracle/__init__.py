@@ -253,3 +253,39 @@ def ser_refresh_backward(a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, gout, grad_is_l
     if bad < 0:
         raise ValueError("s2*s3 + sf exceeds the oracle's candidate buffer")
     return dw1, dw2, dfw, int(bad)
+
+
+def ser_chain(a1_idx, a1_w, legs, s_mid: int, s1: int):
+    """Multi-step referral: B_1 = A1, B_{m+1} = Sparsify(B_m A_{m+1}) for the legs A_2..A_l in
+    `legs` (a list of (idx, w) [B, n, k, s3]); every intermediate is cut to s_mid slots, the
+    last to s1. Each step is oracle_ser. Returns (idx, w, bad_refs)."""
+    cur_i, cur_w, bad = a1_idx, a1_w, 0
+    for m, (li, lw) in enumerate(legs):
+        s_out = s1 if m == len(legs) - 1 else s_mid
+        cur_i, cur_w, b = ser(cur_i, cur_w, li, lw, s_out)
+        bad += b
+    return cur_i, cur_w, bad
+
+
+def ser_chain_backward(a1_idx, a1_w, legs, s_mid: int, gout, grad_is_log: bool = False):
+    """Gradients of ser_chain's kept weights w.r.t. A1's weights and every leg's weights.
+
+    The forward is recomputed step by step; the gradient then runs back through the steps,
+    each one oracle_ser_backward (the gradient w.r.t. a step's first leg is the upstream
+    gradient of the previous step's kept weights, rounded to fp32 between steps). Returns
+    (dw1 [B,n,k,s2], [dleg_2, ..., dleg_l], bad_refs), fp64.
+    """
+    firsts = [(_np(a1_idx, np.int32), _np(a1_w, np.float32))]
+    for li, lw in legs[:-1]:
+        oi, ow, _ = ser(firsts[-1][0], firsts[-1][1], li, lw, s_mid)
+        firsts.append((oi, ow))
+    g = _np(gout, np.float32)
+    dlegs = [None] * len(legs)
+    d_first, bad = None, 0
+    for m in range(len(legs) - 1, -1, -1):
+        d_first, d_leg, b = ser_backward(firsts[m][0], firsts[m][1], legs[m][0], legs[m][1], g,
+                                         grad_is_log and m == len(legs) - 1)
+        bad += b
+        dlegs[m] = d_leg
+        g = d_first.astype(np.float32)
+    return d_first, dlegs, bad
