@@ -246,6 +246,65 @@ gm_status gm_ser_sea_refresh_forward(const int32_t *a1_idx, const float *a1_w, i
                                      void *o, float *lse, cudaStream_t stream);
 
 /*
+ * gm_ser_chain_forward - multi-step referral: B_1 = A1, B_{m+1} = Sparsify(B_m A_{m+1}),
+ * A' = B_l, for legs A2 .. Al.
+ * Source: ai.info summary, "Key Contributions" item 2 (the soft sparse adjacency matrix is
+ * raised to the l-th power and the result is sparsified) and "Main Findings", bullet on
+ * referral (models with 3 and 4 legs; more steps do not always help). The pages give no
+ * formula for the intermediate cuts; the reading here: every step is gm_ser_forward's
+ * referral applied to the row's previous result, intermediates cut to s_mid slots, the last
+ * step to s1.
+ *
+ *   a1_idx, a1_w     device, [B, n, k, s2]        first leg
+ *   leg_idx, leg_w   HOST arrays of nlegs device pointers, each [B, n, k, s3]: the legs
+ *                    A2 .. A(nlegs+1) in chain order (they may be the same tensor: A^l)
+ *   nlegs            1 .. 7 (1 is gm_ser_forward)
+ *   s_mid            slots of every intermediate (1 <= s_mid, s_mid*s3 <= 32)
+ *   out_idx, out_w   device, [B, n, k, s1], written
+ *   other limits     as gm_ser_forward
+ * Deterministic and bit-identical to the steps above in sequence; no intermediate is written.
+ */
+gm_status gm_ser_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                               const int32_t *const *leg_idx, const float *const *leg_w, int nlegs,
+                               int s3, int s_mid, int32_t *out_idx, float *out_w, int s1,
+                               int B, int n, int k, cudaStream_t stream);
+
+/*
+ * gm_ser_chain_backward - gradients of gm_ser_chain_forward's kept weights with respect to the
+ * first leg's and every chain leg's weights.
+ * Source: as gm_ser_chain_forward; only retained weights get gradients (referral paragraph).
+ *
+ * The chain is recomputed; the gradient runs back through the steps (each step as
+ * gm_ser_backward, every intermediate's kept set held as the forward chose it).
+ *
+ *   gout, grad_is_log  as gm_ser_backward (grad_is_log applies to the final A')
+ *   dw1                device fp32 [B, n, k, s2], written (added to if accumulate)
+ *   dleg               HOST array of nlegs device pointers, fp32 [B, n, k, s3] each: the
+ *                      legs' gradients, zeroed by library kernels then scatter-added (added to
+ *                      without zeroing if accumulate); pointers may alias when legs do (the
+ *                      contributions then add up)
+ *   other arguments    as gm_ser_chain_forward
+ */
+gm_status gm_ser_chain_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                const int32_t *const *leg_idx, const float *const *leg_w, int nlegs,
+                                int s3, int s_mid, const float *gout, int s1, int grad_is_log,
+                                int B, int n, int k, float *dw1, float *const *dleg, int accumulate,
+                                cudaStream_t stream);
+
+/*
+ * gm_ser_sea_chain_forward - gm_ser_chain_forward followed by gm_sea_forward on its result.
+ * One fused kernel for bf16 features, s2 = s3 = s_mid in {2, 4}, s1 <= 4 and nlegs in {2, 3};
+ * other shapes run the chain into out_idx/out_w and then SEA (GM_ERR_UNSUPPORTED if those are
+ * NULL). Arguments as gm_ser_chain_forward and gm_ser_sea_forward (k = hkv).
+ */
+gm_status gm_ser_sea_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                   const int32_t *const *leg_idx, const float *const *leg_w,
+                                   int nlegs, int s3, int s_mid, int32_t *out_idx, float *out_w,
+                                   int s1, const void *q, const void *k, const void *v,
+                                   gm_dtype dtype, int B, int n, int hq, int hkv, int d,
+                                   float scale, void *o, float *lse, cudaStream_t stream);
+
+/*
  * gm_sea_forward - sparse edge attention.
  * Source: ai.info summary, "Key Contributions" item 3 (SEA: edge indices select the K/V
  * positions; node factor = scaled q.k, edge factor = log edge weight, combined as a product

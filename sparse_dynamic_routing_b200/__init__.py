@@ -6,6 +6,8 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_leg_sparsify     both referral legs from the stored edges (mixed, then sparsified)
     gm_leg_backward     gradients of the kept leg weights
     gm_ser_forward      sparse edge referral, A' = Sparsify_s1(A1 A2)
+    gm_ser_chain_forward / _backward, gm_ser_sea_chain_forward
+                        multi-step referral, B_{m+1} = Sparsify(B_m A_{m+1})
     gm_ser_refresh_forward / _backward, gm_ser_sea_refresh_forward
                         the referral with refresh edges, A' = Sparsify_s1(A1 A2 + F)
     gm_sea_forward      sparse edge attention
@@ -27,9 +29,12 @@ from ._binding import (  # noqa: F401
     gm_sea_backward_workspace_size,
     gm_sea_forward,
     gm_ser_backward,
+    gm_ser_chain_backward,
+    gm_ser_chain_forward,
     gm_ser_forward,
     gm_ser_refresh_backward,
     gm_ser_refresh_forward,
+    gm_ser_sea_chain_forward,
     gm_ser_sea_refresh_forward,
     gm_ser_sea_forward,
     gm_version,

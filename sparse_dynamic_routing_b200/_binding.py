@@ -29,6 +29,11 @@ SIGNATURES = {
     "gm_leg_backward": [_vp, _vp, _ci, _vp, _vp, ctypes.c_int64, _vp, _ci, _vp, _ci, _ci, _ci,
                         _ci, _vp, _vp, _vp, _ci, _vp],
     "gm_ser_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
+    "gm_ser_chain_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _vp],
+    "gm_ser_chain_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _vp,
+                              _vp, _ci, _vp],
+    "gm_ser_sea_chain_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _vp, _vp, _ci, _vp, _vp, _vp,
+                                 _ci, _ci, _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp],
     "gm_ser_refresh_forward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci,
                                _ci, _vp],
     "gm_ser_refresh_backward": [_vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci,
@@ -307,6 +312,82 @@ def gm_ser_sea_refresh_forward(q, k, v, a1_idx, a1_w, a2_idx, a2_w, f_idx, f_w, 
         B, n, hq, hkv, d, _scale(scale, d), _ptr(o, q.dtype, "o"), _ptr(lse, f32, "lse"),
         _stream(stream))
     _check(st, "gm_ser_sea_refresh_forward")
+    return out_idx, out_w, o, lse
+
+
+def _chain_legs(a1_idx, a1_w, legs):
+    B, n, k, s2 = a1_idx.shape
+    if a1_w.shape != a1_idx.shape or not legs:
+        raise ValueError("first leg shapes disagree, or no chain legs")
+    s3 = legs[0][0].shape[3]
+    for li, lw in legs:
+        if tuple(li.shape) != (B, n, k, s3) or lw.shape != li.shape:
+            raise ValueError("every chain leg must be [B, n, k, s3]")
+    pi = (ctypes.c_void_p * len(legs))(*[_ptr(li, torch.int32, "leg_idx") for li, _ in legs])
+    pw = (ctypes.c_void_p * len(legs))(*[_ptr(lw, torch.float32, "leg_w") for _, lw in legs])
+    return B, n, k, s2, s3, pi, pw
+
+
+def gm_ser_chain_forward(a1_idx, a1_w, legs, s_mid: int, s1: int, out_idx=None, out_w=None,
+                         stream=None):
+    """Multi-step referral through `legs` [(idx, w), ...]. Returns (out_idx, out_w) [B,n,k,s1]."""
+    B, n, k, s2, s3, pi, pw = _chain_legs(a1_idx, a1_w, legs)
+    dev = a1_idx.device
+    out_idx = torch.empty((B, n, k, s1), dtype=torch.int32, device=dev) if out_idx is None else out_idx
+    out_w = torch.empty((B, n, k, s1), dtype=torch.float32, device=dev) if out_w is None else out_w
+    st = load_library().gm_ser_chain_forward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, torch.float32, "a1_w"), s2,
+        ctypes.cast(pi, ctypes.c_void_p), ctypes.cast(pw, ctypes.c_void_p), len(legs), s3, s_mid,
+        _ptr(out_idx, torch.int32, "out_idx"), _ptr(out_w, torch.float32, "out_w"), s1, B, n, k,
+        _stream(stream))
+    _check(st, "gm_ser_chain_forward")
+    return out_idx, out_w
+
+
+def gm_ser_chain_backward(a1_idx, a1_w, legs, s_mid: int, gout, grad_is_log=False, dw1=None,
+                          dlegs=None, accumulate=False, stream=None):
+    """Gradients of the multi-step referral's kept weights. Returns (dw1, [dleg, ...])."""
+    B, n, k, s2, s3, pi, pw = _chain_legs(a1_idx, a1_w, legs)
+    s1 = gout.shape[3]
+    dev = a1_idx.device
+    f32 = torch.float32
+    dw1 = torch.empty((B, n, k, s2), dtype=f32, device=dev) if dw1 is None else dw1
+    if dlegs is None:
+        dlegs = [torch.empty((B, n, k, s3), dtype=f32, device=dev) for _ in legs]
+    pd = (ctypes.c_void_p * len(legs))(*[_ptr(d, f32, "dleg") for d in dlegs])
+    st = load_library().gm_ser_chain_backward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        ctypes.cast(pi, ctypes.c_void_p), ctypes.cast(pw, ctypes.c_void_p), len(legs), s3, s_mid,
+        _ptr(gout, f32, "gout"), s1, int(bool(grad_is_log)), B, n, k, _ptr(dw1, f32, "dw1"),
+        ctypes.cast(pd, ctypes.c_void_p), int(bool(accumulate)), _stream(stream))
+    _check(st, "gm_ser_chain_backward")
+    return dw1, dlegs
+
+
+def gm_ser_sea_chain_forward(q, k, v, a1_idx, a1_w, legs, s_mid: int, s1: int, scale=None,
+                             out_idx=None, out_w=None, o=None, lse=None, want_lse=True,
+                             stream=None):
+    """Multi-step referral -> SEA forward. Returns (out_idx, out_w, o, lse)."""
+    B, n, hq, d = q.shape
+    hkv = k.shape[2]
+    _, _, kk, s2, s3, pi, pw = _chain_legs(a1_idx, a1_w, legs)
+    if kk != hkv or tuple(a1_idx.shape[:2]) != (B, n):
+        raise ValueError("edge tensors must be [B, n, hkv, s]")
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape or k.dtype != q.dtype or v.dtype != q.dtype:
+        raise ValueError("k/v must match q")
+    dev = q.device
+    out_idx = torch.empty((B, n, hkv, s1), dtype=torch.int32, device=dev) if out_idx is None else out_idx
+    out_w = torch.empty((B, n, hkv, s1), dtype=torch.float32, device=dev) if out_w is None else out_w
+    o = torch.empty_like(q) if o is None else o
+    if lse is None and want_lse:
+        lse = torch.empty((B, n, hq), dtype=torch.float32, device=dev)
+    st = load_library().gm_ser_sea_chain_forward(
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, torch.float32, "a1_w"), s2,
+        ctypes.cast(pi, ctypes.c_void_p), ctypes.cast(pw, ctypes.c_void_p), len(legs), s3, s_mid,
+        _ptr(out_idx, torch.int32, "out_idx"), _ptr(out_w, torch.float32, "out_w"), s1,
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _fdtype(q), B, n, hq, hkv, d,
+        _scale(scale, d), _ptr(o, q.dtype, "o"), _ptr(lse, torch.float32, "lse"), _stream(stream))
+    _check(st, "gm_ser_sea_chain_forward")
     return out_idx, out_w, o, lse
 
 

@@ -16,6 +16,7 @@
 #include "gm_sea_bwd.cuh"
 #include "gm_ser.cuh"
 #include "gm_ser_bwd.cuh"
+#include "gm_ser_chain.cuh"
 
 namespace {
 
@@ -60,6 +61,38 @@ gm_status check_refresh(const int32_t *f_idx, const float *f_w, int sf, int s2, 
 {
     if (sf < 1 || s2 * s3 + sf > MAX_SLOTS) return GM_ERR_INVALID_ARG;
     if (rows > 0 && (!f_idx || !f_w)) return GM_ERR_INVALID_ARG;
+    return GM_OK;
+}
+
+// Arguments of a multi-step referral: legs[0] is the second leg of the first step, legs[1..]
+// the chain (nlegs in 1..GM_MAX_CHAIN). Fills a SerArgs for the chain kernels.
+gm_status chain_args(const int32_t *a1_idx, const float *a1_w, int s2,
+                     const int32_t *const *leg_idx, const float *const *leg_w, int nlegs, int s3,
+                     int s_mid, int s1, int B, int n, int k, SerArgs &a)
+{
+    if (nlegs < 1 || nlegs > GM_MAX_CHAIN || !leg_idx || !leg_w) return GM_ERR_INVALID_ARG;
+    if (s_mid < 1 || s_mid > MAX_SLOTS || s_mid * s3 > MAX_SLOTS) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, leg_idx[0], leg_w[0], s3, s1, B, n, k);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    for (int m = 0; m < nlegs; ++m)
+        if (!leg_idx[m] || !leg_w[m]) return GM_ERR_INVALID_ARG;
+    a.a1_idx = a1_idx;
+    a.a1_w = a1_w;
+    a.a2_idx = leg_idx[0];
+    a.a2_w = leg_w[0];
+    for (int m = 1; m < nlegs; ++m) {
+        a.chain_idx[m - 1] = leg_idx[m];
+        a.chain_w[m - 1] = leg_w[m];
+    }
+    a.nchain = nlegs - 1;
+    a.s_mid = s_mid;
+    a.s1 = s1;
+    a.s2 = s2;
+    a.s3 = s3;
+    a.n = n;
+    a.k = k;
+    a.rows = (uint32_t)((int64_t)B * n * k);
+    a.map = row_map(k, n);
     return GM_OK;
 }
 
@@ -199,11 +232,11 @@ template <typename T, int D, int G> struct TileOK {
     static constexpr bool value = (D == 64 || D == 128) && D / VEC >= 2 && D / VEC <= 16 && VEC * G <= 16;
 };
 
-template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int SF = 0>
+template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int SF = 0, int NL = 1>
 gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
 {
     using TG = gm::TileGeom<T, D, G, S1M, TILE_CPL>;
-    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL, SF>;
+    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL, SF, NL>;
     const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
@@ -217,9 +250,25 @@ gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
 template <typename T, int D, int G> struct SerSeaFwd {
     static gm_status run(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
     {
+        if (sa.nchain > 0 && !TileOK<T, D, G>::value) return GM_ERR_UNSUPPORTED;  // chains: tile only
         if constexpr (TileOK<T, D, G>::value) {
-            const bool aligned = aligned16(sa.a1_idx) && aligned16(sa.a1_w) && aligned16(sa.a2_idx) &&
-                                 aligned16(sa.a2_w) && aligned16(sa.out_idx) && aligned16(sa.out_w);
+            bool aligned = aligned16(sa.a1_idx) && aligned16(sa.a1_w) && aligned16(sa.a2_idx) &&
+                       aligned16(sa.a2_w) && aligned16(sa.out_idx) && aligned16(sa.out_w);
+        for (int m = 0; m < sa.nchain; ++m) aligned = aligned && aligned16(sa.chain_idx[m]) && aligned16(sa.chain_w[m]);
+        if (sa.nchain > 0) {
+            // multi-step referral: bf16 features, s2 = s3 = s_mid in {2, 4}, s1 <= 4, 3 or 4 legs
+            if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                if (aligned && sa.sf == 0 && sa.s1 <= 4 && sa.s2 == sa.s3 && sa.s_mid == sa.s2 &&
+                    (sa.s2 == 2 || sa.s2 == 4) && (sa.nchain == 1 || sa.nchain == 2)) {
+                    if (sa.s2 == 2)
+                        return sa.nchain == 1 ? launch_tile<T, D, G, true, 2, 2, 4, 0, 2>(sa, a, st)
+                                              : launch_tile<T, D, G, true, 2, 2, 4, 0, 3>(sa, a, st);
+                    return sa.nchain == 1 ? launch_tile<T, D, G, true, 4, 4, 4, 0, 2>(sa, a, st)
+                                          : launch_tile<T, D, G, true, 4, 4, 4, 0, 3>(sa, a, st);
+                }
+            }
+            return GM_ERR_UNSUPPORTED;  // the caller runs the chain, then SEA
+        }
             if (aligned && sa.sf == 0 && sa.s2 == 2 && sa.s3 == 2) {
                 if (sa.s1 <= 2) return launch_tile<T, D, G, true, 2, 2, 2>(sa, a, st);
                 if (sa.s1 <= 4) return launch_tile<T, D, G, true, 2, 2, 4>(sa, a, st);
@@ -592,6 +641,105 @@ gm_status gm_ser_sea_refresh_forward(const int32_t *a1_idx, const float *a1_w, i
                f_idx, f_w, sf};
     SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows, row_map(hkv, n)};
     return dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
+}
+
+gm_status gm_ser_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                               const int32_t *const *leg_idx, const float *const *leg_w, int nlegs,
+                               int s3, int s_mid, int32_t *out_idx, float *out_w, int s1,
+                               int B, int n, int k, cudaStream_t stream)
+{
+    SerArgs a{};
+    gm_status st = chain_args(a1_idx, a1_w, s2, leg_idx, leg_w, nlegs, s3, s_mid, s1, B, n, k, a);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
+    a.out_idx = out_idx;
+    a.out_w = out_w;
+    const unsigned grid = blocks_for(a.rows, WPB_SER);
+    switch (nlegs) {
+    case 1: gm::ser_chain_kernel<1, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    case 2: gm::ser_chain_kernel<2, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    case 3: gm::ser_chain_kernel<3, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    case 4: gm::ser_chain_kernel<4, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    case 5: gm::ser_chain_kernel<5, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    case 6: gm::ser_chain_kernel<6, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    default: gm::ser_chain_kernel<7, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;
+    }
+    return launched();
+}
+
+gm_status gm_ser_chain_backward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                const int32_t *const *leg_idx, const float *const *leg_w, int nlegs,
+                                int s3, int s_mid, const float *gout, int s1, int grad_is_log,
+                                int B, int n, int k, float *dw1, float *const *dleg, int accumulate,
+                                cudaStream_t stream)
+{
+    if ((grad_is_log != 0 && grad_is_log != 1) || (accumulate != 0 && accumulate != 1)) return GM_ERR_INVALID_ARG;
+    SerArgs a{};
+    gm_status st = chain_args(a1_idx, a1_w, s2, leg_idx, leg_w, nlegs, s3, s_mid, s1, B, n, k, a);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!gout || !dw1 || !dleg) return GM_ERR_INVALID_ARG;
+    gm::ChainBwdArgs b{};
+    b.f = a;
+    b.gout = gout;
+    b.grad_is_log = grad_is_log;
+    b.dw1 = dw1;
+    b.accumulate = accumulate;
+    for (int m = 0; m < nlegs; ++m) {
+        if (!dleg[m]) return GM_ERR_INVALID_ARG;
+        b.dleg[m] = dleg[m];
+    }
+    if (!accumulate) {  // every leg gradient is scatter-added: clear them all first
+        for (int m = 0; m < nlegs; ++m) {
+            gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dleg[m]),
+                                                               (int64_t)a.rows * s3);
+            if (launched() != GM_OK) return GM_ERR_CUDA;
+        }
+    }
+    const unsigned grid = blocks_for(a.rows, WPB_SER);
+    switch (nlegs) {
+    case 1: gm::ser_chain_bwd_kernel<1, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    case 2: gm::ser_chain_bwd_kernel<2, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    case 3: gm::ser_chain_bwd_kernel<3, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    case 4: gm::ser_chain_bwd_kernel<4, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    case 5: gm::ser_chain_bwd_kernel<5, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    case 6: gm::ser_chain_bwd_kernel<6, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    default: gm::ser_chain_bwd_kernel<7, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;
+    }
+    return launched();
+}
+
+gm_status gm_ser_sea_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
+                                   const int32_t *const *leg_idx, const float *const *leg_w,
+                                   int nlegs, int s3, int s_mid, int32_t *out_idx, float *out_w,
+                                   int s1, const void *q, const void *k, const void *v,
+                                   gm_dtype dtype, int B, int n, int hq, int hkv, int d,
+                                   float scale, void *o, float *lse, cudaStream_t stream)
+{
+    if ((out_idx == nullptr) != (out_w == nullptr)) return GM_ERR_INVALID_ARG;
+    SerArgs sa{};
+    gm_status st = chain_args(a1_idx, a1_w, s2, leg_idx, leg_w, nlegs, s3, s_mid, s1, B, n, hkv, sa);
+    if (st != GM_OK) return st;
+    const int32_t dummy_idx = 0;
+    const float dummy_w = 0.0f;
+    st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    sa.out_idx = out_idx;
+    sa.out_w = out_w;
+    SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, sa.rows, row_map(hkv, n)};
+    if (nlegs > 1) {
+        st = dispatch<SerSeaFwd>(dtype, d, hq / hkv, sa, a, stream);
+        if (st != GM_ERR_UNSUPPORTED) return st;
+        // no fused kernel for this shape: the chain writes A', then SEA reads it
+        if (!out_idx) return GM_ERR_UNSUPPORTED;
+        st = gm_ser_chain_forward(a1_idx, a1_w, s2, leg_idx, leg_w, nlegs, s3, s_mid, out_idx, out_w,
+                                  s1, B, n, hkv, stream);
+        if (st != GM_OK) return st;
+        return gm_sea_forward(q, k, v, dtype, out_idx, out_w, s1, B, n, hq, hkv, d, scale, o, lse,
+                              stream);
+    }
+    return gm_ser_sea_forward(a1_idx, a1_w, s2, leg_idx[0], leg_w[0], s3, out_idx, out_w, s1, q, k, v,
+                              dtype, B, n, hq, hkv, d, scale, o, lse, stream);
 }
 
 gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype dtype,

@@ -73,25 +73,22 @@ __device__ __forceinline__ void merge_pairs(const int32_t (&ct)[NC], float (&cu)
     }
 }
 
-// Referral of one edge row by one thread (exact S2, S3; s1 <= S1M). Slots r >= s1 and slots
-// beyond the number of distinct targets come back as (0, 0.0f). SF > 0: the row's SF refresh
-// edges (a.sf == SF) join the candidates after the S2*S3 paths, with their own weights.
-template <int S2, int S3, int S1M, int SF = 0>
-__device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32_t (&to)[S1M],
-                                           float (&wo)[S1M])
+// One referral step of one edge row by one thread: first leg (j, w1) of S_IN slots in
+// registers, second leg [rows, S3] at (leg_idx, leg_w); SF > 0 appends the row's SF refresh
+// edges (a.sf == SF) after the S_IN*S3 paths. Keeps the s_keep <= S_OUT heaviest targets;
+// other slots, and slots beyond the number of distinct targets, come back as (0, 0.0f).
+template <int S_IN, int S3, int S_OUT, int SF = 0>
+__device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uint32_t seq_base,
+                                             uint32_t h, const int32_t (&j)[S_IN],
+                                             const float (&w1)[S_IN], const int32_t *leg_idx,
+                                             const float *leg_w, int s_keep,
+                                             int32_t (&to)[S_OUT], float (&wo)[S_OUT])
 {
-    constexpr int NP2 = S2 * S3, NC = NP2 + SF;
-    uint32_t seq_base, h;
-    a.map.split(row, seq_base, h);
-    int32_t j[S2];
-    float w1[S2];
-    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
-    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
-
+    constexpr int NP2 = S_IN * S3, NC = NP2 + SF;
     int32_t ct[NC];
     float cu[NC];
 #pragma unroll
-    for (int x = 0; x < S2; ++x) {
+    for (int x = 0; x < S_IN; ++x) {
         bool act = w1[x] > 0.0f;
         if (act && (j[x] < 0 || j[x] >= a.n)) {
             raise_index_error();
@@ -106,8 +103,8 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
         }
         if (act) {
             const size_t r2 = ((size_t)(seq_base + (uint32_t)j[x]) * a.k + h) * S3;
-            ld_vec<S3>(a.a2_idx + r2, t2);
-            ld_vec<S3>(a.a2_w + r2, w2);
+            ld_vec<S3>(leg_idx + r2, t2);
+            ld_vec<S3>(leg_w + r2, w2);
         }
 #pragma unroll
         for (int e = 0; e < S3; ++e) {
@@ -138,10 +135,10 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
     // merge: the first occurrence of a target absorbs the later ones, in ascending order
     merge_pairs<0, NC>(ct, cu);
-    // top-s1: repeated arg-max by (weight desc, index asc); the winner is then removed by
+    // top-s: repeated arg-max by (weight desc, index asc); the winner is then removed by
     // value (nonzero targets are distinct after the merge, so the match is unique)
 #pragma unroll
-    for (int r = 0; r < S1M; ++r) {
+    for (int r = 0; r < S_OUT; ++r) {
         float bw = 0.0f;
         int32_t bt = 0;
 #pragma unroll
@@ -152,9 +149,43 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
         }
 #pragma unroll
         for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
-        const bool keep = r < a.s1 && bw > 0.0f;
+        const bool keep = r < s_keep && bw > 0.0f;
         to[r] = keep ? bt : 0;
         wo[r] = keep ? bw : 0.0f;
+    }
+}
+
+// Referral of one edge row by one thread (exact S2, S3; s1 <= S1M), with SF refresh edges
+// when SF > 0 and, when NL > 1, NL - 1 further referral steps through the chain legs (every
+// intermediate of S2 = s_mid slots, the row's previous result held in registers).
+template <int S2, int S3, int S1M, int SF = 0, int NL = 1>
+__device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32_t (&to)[S1M],
+                                           float (&wo)[S1M])
+{
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    int32_t j[S2];
+    float w1[S2];
+    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
+    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
+    if constexpr (NL == 1) {
+        refer_thread<S2, S3, S1M, SF>(a, row, seq_base, h, j, w1, a.a2_idx, a.a2_w, a.s1, to, wo);
+    } else {
+        static_assert(SF == 0, "refresh edges join single-step referrals only");
+#pragma unroll
+        for (int m = 0; m + 1 < NL; ++m) {
+            int32_t jn[S2];
+            float wn[S2];
+            refer_thread<S2, S3, S2>(a, row, seq_base, h, j, w1, m == 0 ? a.a2_idx : a.chain_idx[m - 1],
+                                     m == 0 ? a.a2_w : a.chain_w[m - 1], S2, jn, wn);
+#pragma unroll
+            for (int x = 0; x < S2; ++x) {
+                j[x] = jn[x];
+                w1[x] = wn[x];
+            }
+        }
+        refer_thread<S2, S3, S1M>(a, row, seq_base, h, j, w1, a.chain_idx[NL - 2], a.chain_w[NL - 2],
+                                  a.s1, to, wo);
     }
 }
 
@@ -179,10 +210,10 @@ template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
 };
 
 // REFER = true: fused SER -> SEA (edges from the referral of sa's legs, plus SF refresh edges
-// per row when SF > 0);
+// per row when SF > 0, or through NL legs of a multi-step referral when NL > 1);
 // REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
 template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL,
-          int SF = 0>
+          int SF = 0, int NL = 1>
 __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
     using TG = TileGeom<T, D, G, S1M, CPL>;
@@ -237,7 +268,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(Se
                     }
                 }
             } else if (row < rows) {
-                ser_thread<S2, S3, S1M, SF>(sa, row, to, wo);
+                ser_thread<S2, S3, S1M, SF, NL>(sa, row, to, wo);
                 if (sa.out_idx != nullptr) {
                     if (sa.s1 == S1M && S1M == 4) {
                         *reinterpret_cast<int4 *>(sa.out_idx + (size_t)row * 4) = make_int4(to[0], to[1], to[2], to[3]);

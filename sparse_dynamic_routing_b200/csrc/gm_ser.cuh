@@ -16,6 +16,11 @@
 
 #include "gm_common.cuh"
 
+// Legs of a multi-step referral after the first one (the pages' models use 3 or 4 legs).
+#ifndef GM_MAX_CHAIN
+#define GM_MAX_CHAIN 7
+#endif
+
 namespace gm {
 
 struct SerArgs {
@@ -33,85 +38,117 @@ struct SerArgs {
     const int32_t *f_idx;
     const float *f_w;
     int sf;
+    // multi-step referral: legs 3.. of the chain B_{m+1} = Sparsify(B_m A_{m+1}) (leg 2 is
+    // a2), nchain of them; intermediates are cut to s_mid slots, the last step to s1
+    const int32_t *chain_idx[GM_MAX_CHAIN - 1];
+    const float *chain_w[GM_MAX_CHAIN - 1];
+    int nchain;
+    int s_mid;
 };
 
-// Referral of one edge row. On return lane r < s1 holds the r-th kept (t, W); other lanes
-// (and slots beyond the number of distinct targets) hold (0, 0.0f). Must be called by all
-// 32 lanes of the warp. `seq_base` = b*n and `h` = channel of `row`.
-__device__ __forceinline__ void ser_row(const SerArgs &a, uint32_t row, uint32_t seq_base,
-                                        uint32_t h, int lane, int32_t &t_out, float &w_out)
+// ---- one referral step of one row, one candidate per lane ----------------------------------
+//
+// The first leg of the row is held by the warp (lane a < s_in holds slot a: target j_l,
+// weight w1_l); the second leg is [rows, s3] at (leg_idx, leg_w), channel h of the same
+// sequence; lanes s_in*s3 .. s_in*s3 + sf - 1 hold the row's refresh slots, if any.
+
+struct ReferCand {
+    int32_t t;    // candidate target (valid when u != 0)
+    float u;      // candidate weight (0: no candidate)
+    float w1;     // first-leg weight of a path candidate
+    float w2;     // second-leg weight of a path candidate
+    size_t r2;    // second-leg element of a path candidate
+    bool path;    // lane < s_in * s3
+    bool refresh; // refresh slot lane - s_in * s3
+};
+
+__device__ __forceinline__ ReferCand refer_candidates(int32_t j_l, float w1_l, int s_in,
+                                                      const int32_t *leg_idx, const float *leg_w,
+                                                      int s3, const int32_t *f_idx,
+                                                      const float *f_w, int sf, uint32_t row,
+                                                      int n, int k, uint32_t seq_base,
+                                                      uint32_t h, int lane)
 {
-    const int nc = a.s2 * a.s3;
-
-    // first leg: lane a < s2 reads slot a of row i
-    int32_t j_l = 0;
-    float w1_l = 0.0f;
-    if (lane < a.s2) {
-        j_l = __ldg(a.a1_idx + (size_t)row * a.s2 + lane);
-        w1_l = __ldg(a.a1_w + (size_t)row * a.s2 + lane);
-    }
-    const int ca = lane / a.s3;          // first-leg slot of this lane's candidate
-    const int ce = lane - ca * a.s3;     // second-leg slot
+    const int nc = s_in * s3;
+    const int ca = lane / s3;          // first-leg slot of this lane's candidate
+    const int ce = lane - ca * s3;     // second-leg slot
     const int32_t j = __shfl_sync(FULL, j_l, ca);
-    const float w1 = __shfl_sync(FULL, w1_l, ca);
-
-    // second leg: lane c reads slot e of row j (same channel h)
-    float u = 0.0f;
-    int32_t t = 0;
-    bool act = lane < nc && w1 > 0.0f;
-    if (act && (j < 0 || j >= a.n)) {
+    ReferCand c;
+    c.w1 = __shfl_sync(FULL, w1_l, ca);
+    c.u = 0.0f;
+    c.w2 = 0.0f;
+    c.t = 0;
+    c.r2 = 0;
+    c.path = lane < nc;
+    c.refresh = lane >= nc && lane < nc + sf;
+    bool act = c.path && c.w1 > 0.0f;
+    if (act && (j < 0 || j >= n)) {
         if (ce == 0) raise_index_error();  // once per active first-leg slot
         act = false;
     }
     if (act) {
-        const size_t r2 = ((size_t)(seq_base + (uint32_t)j) * a.k + h) * a.s3 + ce;
-        const float w2 = __ldg(a.a2_w + r2);
-        const int32_t t2 = __ldg(a.a2_idx + r2);
-        if (w2 > 0.0f) {
-            if (t2 < 0 || t2 >= a.n) {
+        c.r2 = ((size_t)(seq_base + (uint32_t)j) * k + h) * s3 + ce;
+        c.w2 = __ldg(leg_w + c.r2);
+        const int32_t t2 = __ldg(leg_idx + c.r2);
+        if (c.w2 > 0.0f) {
+            if (t2 < 0 || t2 >= n) {
                 raise_index_error();
             } else {
-                u = __fmul_rn(w1, w2);
-                t = t2;
+                c.u = __fmul_rn(c.w1, c.w2);
+                c.t = t2;
             }
         }
     }
-    // refresh lanes nc <= lane < nc + sf: candidate nc + f is refresh slot f with its own weight
-    if (lane >= nc && lane < nc + a.sf) {
-        const size_t rf = (size_t)row * a.sf + (lane - nc);
-        const float wf = __ldg(a.f_w + rf);
-        const int32_t tf = __ldg(a.f_idx + rf);
+    if (c.refresh) {
+        const size_t rf = (size_t)row * sf + (lane - nc);
+        const float wf = __ldg(f_w + rf);
+        const int32_t tf = __ldg(f_idx + rf);
         if (wf > 0.0f) {
-            if (tf < 0 || tf >= a.n) {
+            if (tf < 0 || tf >= n) {
                 raise_index_error();
             } else {
-                u = wf;
-                t = tf;
+                c.u = wf;
+                c.t = tf;
             }
         }
     }
-    const bool cand = u != 0.0f;
+    return c;
+}
 
-    // merge: equal targets form a group whose lowest lane (the leader) accumulates the
-    // other members in ascending lane order. Only non-leading members need a shuffle.
+// Merge: equal targets form a group whose lowest lane (the leader) accumulates the other
+// members in ascending lane order (only non-leading members need a shuffle). Returns the
+// lane's selection key (weight bits, ~target), nonzero on leaders only.
+__device__ __forceinline__ void refer_merge(const ReferCand &c, int lane, unsigned &key_hi,
+                                            unsigned &key_lo)
+{
+    const bool cand = c.u != 0.0f;
     const unsigned cmask = __ballot_sync(FULL, cand);
-    const unsigned grp = __match_any_sync(FULL, cand ? t : -1) & cmask;
+    const unsigned grp = __match_any_sync(FULL, cand ? c.t : -1) & cmask;
     const bool leader = cand && (__ffs(grp) - 1 == lane);
-    float W = u;
+    float W = c.u;
     unsigned followers = __ballot_sync(FULL, cand && !leader);
     while (followers) {  // warp-uniform loop, usually empty
         const int src = __ffs(followers) - 1;
         followers &= followers - 1;
-        const float v = __shfl_sync(FULL, u, src);
+        const float v = __shfl_sync(FULL, c.u, src);
         if (leader && ((grp >> src) & 1u)) W = __fadd_rn(W, v);
     }
+    key_hi = leader ? __float_as_uint(W) : 0u;
+    key_lo = leader ? ~(unsigned)c.t : 0u;
+}
 
-    // top-s1 by (weight desc, index asc)
-    unsigned key_hi = leader ? __float_as_uint(W) : 0u;
-    unsigned key_lo = leader ? ~(unsigned)t : 0u;
+// Top-s_out by (weight desc, index asc). Lane r < s_out receives the r-th kept (t, W),
+// others (0, 0.0f); every candidate lane whose target was kept receives its slot and W.
+__device__ __forceinline__ void refer_select(const ReferCand &c, unsigned key_hi, unsigned key_lo,
+                                             int s_out, int lane, int32_t &t_out, float &w_out,
+                                             int &slot, float &slot_w)
+{
     t_out = 0;
     w_out = 0.0f;
-    for (int r = 0; r < a.s1; ++r) {
+    slot = -1;
+    slot_w = 0.0f;
+    const bool cand = c.u != 0.0f;
+    for (int r = 0; r < s_out; ++r) {
         const unsigned mh = __reduce_max_sync(FULL, key_hi);
         if (mh == 0u) break;  // warp-uniform: no candidate left, the rest stays padding
         const unsigned ml = __reduce_max_sync(FULL, key_hi == mh ? key_lo : 0u);
@@ -119,8 +156,34 @@ __device__ __forceinline__ void ser_row(const SerArgs &a, uint32_t row, uint32_t
             t_out = (int32_t)~ml;
             w_out = __uint_as_float(mh);
         }
+        if (cand && (int32_t)~ml == c.t) {
+            slot = r;
+            slot_w = __uint_as_float(mh);
+        }
         if (key_hi == mh && key_lo == ml) key_hi = key_lo = 0u;
     }
+}
+
+// Referral of one edge row. On return lane r < s1 holds the r-th kept (t, W); other lanes
+// (and slots beyond the number of distinct targets) hold (0, 0.0f). Must be called by all
+// 32 lanes of the warp. `seq_base` = b*n and `h` = channel of `row`.
+__device__ __forceinline__ void ser_row(const SerArgs &a, uint32_t row, uint32_t seq_base,
+                                        uint32_t h, int lane, int32_t &t_out, float &w_out)
+{
+    // first leg: lane a < s2 reads slot a of row i
+    int32_t j_l = 0;
+    float w1_l = 0.0f;
+    if (lane < a.s2) {
+        j_l = __ldg(a.a1_idx + (size_t)row * a.s2 + lane);
+        w1_l = __ldg(a.a1_w + (size_t)row * a.s2 + lane);
+    }
+    const ReferCand c = refer_candidates(j_l, w1_l, a.s2, a.a2_idx, a.a2_w, a.s3, a.f_idx, a.f_w,
+                                         a.sf, row, a.n, a.k, seq_base, h, lane);
+    unsigned key_hi, key_lo;
+    refer_merge(c, lane, key_hi, key_lo);
+    int slot;
+    float slot_w;
+    refer_select(c, key_hi, key_lo, a.s1, lane, t_out, w_out, slot, slot_w);
 }
 
 template <int WPB>

@@ -29,6 +29,38 @@ struct SerBwdArgs {
     float *dfw;          // [rows, sf] when the forward had refresh edges
 };
 
+// Backward of one referral step of one row (the candidates, merge and selection of
+// refer_candidates / refer_merge / refer_select, recomputed). Lane r < s_out holds g_r, the
+// upstream gradient of kept slot r (of ln W_r when grad_is_log). Returns, on lane a < s_in,
+// the gradient of first-leg slot a (its candidates' terms summed in ascending e), scatter-adds
+// the second-leg gradients into dleg with fp32 atomics, and gives refresh lanes g of their
+// target in g_refresh.
+__device__ __forceinline__ float refer_step_backward(const ReferCand &c, unsigned key_hi,
+                                                     unsigned key_lo, int s_in, int s3, int s_out,
+                                                     float g_l, int grad_is_log, float *dleg,
+                                                     int lane, float &g_refresh)
+{
+    int32_t t_out;
+    float w_out;
+    int slot;
+    float slot_w;
+    refer_select(c, key_hi, key_lo, s_out, lane, t_out, w_out, slot, slot_w);
+    const float gs = __shfl_sync(FULL, g_l, slot >= 0 ? slot : 0);
+    float g = 0.0f;
+    if (slot >= 0) g = grad_is_log ? gs / slot_w : gs;
+    // first leg: lane a sums its s3 candidates in ascending e
+    const float c1 = slot >= 0 ? g * c.w2 : 0.0f;
+    float d1 = 0.0f;
+    for (int e = 0; e < s3; ++e) {
+        const float v = __shfl_sync(FULL, c1, (lane * s3 + e) & 31);
+        d1 += v;
+    }
+    // second leg: scatter to the shared second-leg rows
+    if (slot >= 0 && c.path) atomicAdd(dleg + c.r2, g * c.w1);
+    g_refresh = c.refresh ? g : 0.0f;
+    return lane < s_in ? d1 : 0.0f;
+}
+
 template <int WPB>
 __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
 {
@@ -38,104 +70,28 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
     if (row >= a.rows) return;  // warp-uniform
     uint32_t seq_base, h;
     a.map.split(row, seq_base, h);
-    const int nc = a.s2 * a.s3;
-
-    // ---- forward recompute (ser_row's arithmetic, keeping the per-lane candidate) ----------
     int32_t j_l = 0;
-    float w1_l = 0.0f;
+    float w1_l = 0.0f, g_l = 0.0f;
     if (lane < a.s2) {
         j_l = __ldg(a.a1_idx + (size_t)row * a.s2 + lane);
         w1_l = __ldg(a.a1_w + (size_t)row * a.s2 + lane);
     }
-    const int ca = lane / a.s3, ce = lane - ca * a.s3;
-    const int32_t j = __shfl_sync(FULL, j_l, ca);
-    const float w1 = __shfl_sync(FULL, w1_l, ca);
-    float u = 0.0f, w2 = 0.0f;
-    int32_t t = 0;
-    size_t r2 = 0;
-    bool act = lane < nc && w1 > 0.0f;
-    if (act && (j < 0 || j >= a.n)) {
-        if (ce == 0) raise_index_error();
-        act = false;
-    }
-    if (act) {
-        r2 = ((size_t)(seq_base + (uint32_t)j) * a.k + h) * a.s3 + ce;
-        w2 = __ldg(a.a2_w + r2);
-        const int32_t t2 = __ldg(a.a2_idx + r2);
-        if (w2 > 0.0f) {
-            if (t2 < 0 || t2 >= a.n) {
-                raise_index_error();
-            } else {
-                u = __fmul_rn(w1, w2);
-                t = t2;
-            }
-        }
-    }
-    const bool refresh = lane >= nc && lane < nc + a.sf;  // refresh slot lane - nc
-    if (refresh) {
-        const size_t rf = (size_t)row * a.sf + (lane - nc);
-        const float wf = __ldg(a.f_w + rf);
-        const int32_t tf = __ldg(a.f_idx + rf);
-        if (wf > 0.0f) {
-            if (tf < 0 || tf >= a.n) {
-                raise_index_error();
-            } else {
-                u = wf;
-                t = tf;
-            }
-        }
-    }
-    const bool cand = u != 0.0f;
-    const unsigned cmask = __ballot_sync(FULL, cand);
-    const unsigned grp = __match_any_sync(FULL, cand ? t : -1) & cmask;
-    const bool leader = cand && (__ffs(grp) - 1 == lane);
-    float W = u;
-    unsigned followers = __ballot_sync(FULL, cand && !leader);
-    while (followers) {
-        const int src = __ffs(followers) - 1;
-        followers &= followers - 1;
-        const float v = __shfl_sync(FULL, u, src);
-        if (leader && ((grp >> src) & 1u)) W = __fadd_rn(W, v);
-    }
-    unsigned key_hi = leader ? __float_as_uint(W) : 0u;
-    unsigned key_lo = leader ? ~(unsigned)t : 0u;
-
-    // ---- selection, and each candidate's kept slot ------------------------------------------
-    int slot = -1;       // kept slot of this lane's candidate (-1: not kept)
-    float slot_w = 0.0f;  // its merged weight
-    for (int r = 0; r < a.s1; ++r) {
-        const unsigned mh = __reduce_max_sync(FULL, key_hi);
-        if (mh == 0u) break;  // warp-uniform
-        const unsigned ml = __reduce_max_sync(FULL, key_hi == mh ? key_lo : 0u);
-        if (cand && (int32_t)~ml == t) {
-            slot = r;
-            slot_w = __uint_as_float(mh);
-        }
-        if (key_hi == mh && key_lo == ml) key_hi = key_lo = 0u;
-    }
-    float g = 0.0f;
-    if (slot >= 0) {
-        g = __ldg(b.gout + (size_t)row * a.s1 + slot);
-        if (b.grad_is_log) g = g / slot_w;
-    }
-
-    // ---- first leg: lane a sums its s3 candidates in ascending e --------------------------------
-    const float c1 = slot >= 0 ? g * w2 : 0.0f;
-    float d1 = 0.0f;
-    for (int e = 0; e < a.s3; ++e) {
-        const float v = __shfl_sync(FULL, c1, (lane * a.s3 + e) & 31);
-        d1 += v;
-    }
+    if (lane < a.s1) g_l = __ldg(b.gout + (size_t)row * a.s1 + lane);
+    const ReferCand c = refer_candidates(j_l, w1_l, a.s2, a.a2_idx, a.a2_w, a.s3, a.f_idx, a.f_w,
+                                         a.sf, row, a.n, a.k, seq_base, h, lane);
+    unsigned key_hi, key_lo;
+    refer_merge(c, lane, key_hi, key_lo);
+    float g_refresh;
+    const float d1 = refer_step_backward(c, key_hi, key_lo, a.s2, a.s3, a.s1, g_l, b.grad_is_log,
+                                         b.dw2, lane, g_refresh);
     if (lane < a.s2) {
         float *p = b.dw1 + (size_t)row * a.s2 + lane;
         *p = b.accumulate ? *p + d1 : d1;
     }
-    // ---- second leg: scatter to the shared second-leg rows ----------------------------------------
-    if (slot >= 0 && lane < nc) atomicAdd(b.dw2 + r2, g * w1);
-    // ---- refresh slots: d W / d w_f = 1 -------------------------------------------------------------
-    if (refresh) {
-        float *p = b.dfw + (size_t)row * a.sf + (lane - nc);
-        *p = b.accumulate ? *p + g : g;
+    // refresh slots: d W / d w_f = 1
+    if (c.refresh) {
+        float *p = b.dfw + (size_t)row * a.sf + (lane - a.s2 * a.s3);
+        *p = b.accumulate ? *p + g_refresh : g_refresh;
     }
 }
 

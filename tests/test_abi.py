@@ -180,3 +180,22 @@ def test_refresh_argument_checks(lib):
     a[8] = 31  # s2*s3 + sf > 32
     a[22] = FAKE
     assert h(*a) == bnd.GM_ERR_INVALID_ARG
+
+
+def test_chain_argument_checks(lib):
+    legs_i = (ctypes.c_void_p * 8)(*([FAKE] * 8))
+    legs_w = (ctypes.c_void_p * 8)(*([FAKE] * 8))
+    f = lib.gm_ser_chain_forward
+    # a1_idx, a1_w, s2, leg_idx[], leg_w[], nlegs, s3, s_mid, out_idx, out_w, s1, B, n, k, stream
+    li, lw = ctypes.cast(legs_i, ctypes.c_void_p), ctypes.cast(legs_w, ctypes.c_void_p)
+    assert f(FAKE, FAKE, 4, li, lw, 0, 4, 4, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, li, lw, 8, 4, 4, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, li, lw, 2, 4, 9, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, NULL, lw, 2, 4, 4, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, 4, li, lw, 2, 4, 4, NULL, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    legs_i[1] = None
+    assert f(FAKE, FAKE, 4, li, lw, 2, 4, 4, FAKE, FAKE, 4, 1, 8, 2, NULL) == bnd.GM_ERR_INVALID_ARG
+    g = lib.gm_ser_chain_backward
+    # ..., s_mid, gout, s1, grad_is_log, B, n, k, dw1, dleg[], accumulate, stream
+    assert g(FAKE, FAKE, 4, li, lw, 1, 4, 4, FAKE, 4, 0, 1, 8, 2, FAKE, NULL, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+    assert g(FAKE, FAKE, 4, li, lw, 1, 4, 4, FAKE, 4, 2, 1, 8, 2, FAKE, li, 0, NULL) == bnd.GM_ERR_INVALID_ARG
