@@ -439,9 +439,11 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     leg_sparsify builds the step's two legs from the workload's stored edges; ser_backward
     takes the step's d ln w back to the legs; leg_backward takes those leg gradients back to
     the stored weights and the mixing coefficients; ser_sea_refresh_forward is the fused
-    forward with the stored edges joining the referral as refresh edges. Bytes are
+    forward with the stored edges joining the referral as refresh edges;
+    ser_sea_chain_forward is the fused forward through a three-leg referral chain. Bytes are
     compulsory: every input read once, every output written once (ser_backward's second-leg
-    rows counted in full; the refresh forward's gathered rows counted from its own edges).
+    rows counted in full; the refresh and chain forwards' gathered rows counted from their own
+    edges, the chain's third leg in full).
     """
     le = {k: v.to(dev) for k, v in I.leg_inputs(wl).items()}
     B, n, k = wl.B, wl.n, wl.hkv
@@ -469,6 +471,19 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     torch.cuda.synchronize(dev)
     rf_bytes = (compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), rf_i.cpu().numpy(),
                                  rf_w.cpu().numpy())["fused_forward"] + e_b_refresh(wl))
+    # a three-leg chain (the pages' R3): the step's two legs and one more drawn the same way
+    leg3 = [v.to(dev) for v in I.edges(wl, 2, wl.s3, layer=1)]
+    ch_legs = [(g["a2_idx"], g["a2_w"]), (leg3[0], leg3[1])]
+    ch_i = torch.empty_like(ap_i)
+    ch_w = torch.empty_like(ap_w)
+    ch_o = torch.empty_like(g["q"])
+    ch_lse = torch.empty((B, n, wl.hq), dtype=f32, device=dev)
+    gm.gm_ser_sea_chain_forward(g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], ch_legs, wl.s2,
+                                wl.s1, wl.scale, out_idx=ch_i, out_w=ch_w, o=ch_o, lse=ch_lse,
+                                stream=stream)
+    torch.cuda.synchronize(dev)
+    ch_bytes = (compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ch_i.cpu().numpy(),
+                                 ch_w.cpu().numpy())["fused_forward"] + tok * k * wl.s3 * 8)
     e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
     leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
     calls = {
@@ -486,6 +501,11 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
                                         g["a2_w"], le["e_idx"], le["e_w"], wl.s1, wl.scale,
                                         out_idx=rf_i, out_w=rf_w, o=rf_o, lse=rf_lse,
                                         stream=stream)),
+        "ser_sea_chain_forward": ("sea_fwd_tile_kernel (fused 3-leg referral->SEA)", ch_bytes,
+                                  lambda: gm.gm_ser_sea_chain_forward(
+                                      g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], ch_legs,
+                                      wl.s2, wl.s1, wl.scale, out_idx=ch_i, out_w=ch_w, o=ch_o,
+                                      lse=ch_lse, stream=stream)),
         "leg_backward": ("leg_bwd_tile_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
                          lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,
