@@ -14,9 +14,10 @@
 //    and to a shared-memory tile with log2 weights for phase 2.
 //  Phase 2 - attention, C lanes (one 16-byte chunk each) per row, 32 / C rows per pass. Each
 //    lane handles its chunk for all G query heads of the group, so a K/V chunk is unpacked
-//    once and used G times, with packed fp32x2 FMAs. The lane stages exactly the q/K/V
-//    chunks it will read with 16-byte cp.async, P passes ahead, so every byte in flight sits
-//    in shared memory, and completion needs no spin-wait (cp.async.wait_group).
+//    once and used G times, with packed fp32x2 FMAs. The lane stages exactly the K/V chunks
+//    it will read with 16-byte cp.async, P passes ahead, so every byte in flight sits in
+//    shared memory, and completion needs no spin-wait (cp.async.wait_group); its q chunks
+//    go straight to registers one pass ahead.
 // All shuffles run on all 32 lanes: slots are padded to S1M and inactive ones masked after
 // the reduction, so rows at a ragged tail simply compute on zeros and store nothing.
 #pragma once
@@ -189,11 +190,11 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
-// Resident blocks per SM the forward tile kernel is compiled for (shared memory allows about
-// five at the largest stage): caps registers at 65536 / (32 * WPB * MINB) without forcing
-// spills.
+// Resident blocks per SM the forward tile kernel is compiled for (shared memory allows six
+// 4-warp blocks at the largest stage): caps registers at 65536 / (32 * WPB * MINB) = 85
+// without spills.
 #ifndef GM_TILE_MINB
-#define GM_TILE_MINB 4
+#define GM_TILE_MINB 6
 #endif
 
 template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
@@ -204,7 +205,8 @@ template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static constexpr int ROW = D * (int)sizeof(T); // bytes per feature row
     // per row: q rows of the group, then K and V rows of the S1M slots (chunk-interleaved
     // per lane is not needed: every lane reads back only what it copied)
-    static constexpr int RQ = 0, RK = G * ROW, RV = RK + S1M * ROW, RBYTES = RV + S1M * ROW;
+    // per row: the K and V rows of the S1M slots (q goes straight to registers)
+    static constexpr int RK = 0, RV = S1M * ROW, RBYTES = RV + S1M * ROW;
     static constexpr int STAGE = RPW * RBYTES;
     static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
 };
@@ -303,12 +305,6 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(Se
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
                 if (row < rows) {
-                    const char *qs = reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW);
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int cc = 0; cc < CPL; ++cc)
-                            cp_async16(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16, qs + g * TG::ROW + (c * CPL + cc) * 16);
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
@@ -325,10 +321,31 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(Se
             }
             cp_async_commit();
         };
+        // q chunks of a pass, read into registers one pass ahead (a pass's compute covers the
+        // load; q needs no shared memory, which leaves room for more resident warps)
+        auto load_q = [&](int pass, uint4 (&qv)[G][CPL]) {
+            const uint32_t row = r0 + pass * RPW + rr;
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc)
+                    qv[g][cc] = (pass < NPASS && row < rows)
+                                    ? ld16(reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW) +
+                                           g * TG::ROW + (c * CPL + cc) * 16)
+                                    : make_uint4(0u, 0u, 0u, 0u);
+        };
+        uint4 qnext[G][CPL];
+        load_q(0, qnext);
 #pragma unroll
         for (int pass = 0; pass < P; ++pass) issue(pass);
 
         for (int pass = 0; pass < NPASS; ++pass) {
+            uint4 qcur[G][CPL];
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int cc = 0; cc < CPL; ++cc) qcur[g][cc] = qnext[g][cc];
+            load_q(pass + 1, qnext);
             cp_async_wait<P - 1>();
             const int lr = pass * RPW + rr;
             const uint32_t row = r0 + lr;
@@ -349,9 +366,8 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(Se
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) {
                     float f[VEC];
-                    // an invalid row (ragged tail) computes on whatever the stage holds and
-                    // stores nothing
-                    unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + (c * CPL + cc) * 16), f);
+                    // an invalid row (ragged tail) computes on zeros and stores nothing
+                    unpack<T>(qcur[g][cc], f);
 #pragma unroll
                     for (int x = 0; x < NP; ++x) q2[g][cc * NP + x] = make_float2(f[2 * x], f[2 * x + 1]);
                 }
