@@ -4,8 +4,8 @@
 // forward (gm_fused_tile.cuh): a warp owns tiles of 32 consecutive edge rows; phase 1 loads
 // the tile's edges one thread per row into shared memory; phase 2 processes RPW rows per
 // pass with C lanes per row, each lane owning one 16-byte chunk of every feature row for all
-// G query heads, with q, dO, K and V chunks staged by the lane itself via cp.async P passes
-// ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
+// G query heads, with its K and V chunks staged by the lane itself via cp.async P passes
+// ahead and its q and dO chunks read into registers one pass ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
 // dp_j = dO.v_j, D = sum_j p_j dp_j and dz_j = p_j (dp_j - D):
 //   dq          = scale sum_j dz_j k_j                       (stored)
 //   dK[t_j]    += scale sum_heads dz_j q                     (GATHER = false: 16-byte fp32
@@ -30,20 +30,22 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
     static constexpr int RPW = 32 / C;
     static constexpr int NPASS = 32 / RPW;
     static constexpr int ROW = D * (int)sizeof(T);
-    static constexpr int RQ = 0, RG = G * ROW, RK = 2 * G * ROW, RV = RK + S1M * ROW;
+    // per row: the K and V rows of the S1M slots (q and dO go straight to registers)
+    static constexpr int RK = 0, RV = S1M * ROW;
     static constexpr int RBYTES = RV + S1M * ROW;
     static constexpr int STAGE = RPW * RBYTES;
     static_assert(C >= 2 && C <= 16 && (C & (C - 1)) == 0, "two or more rows per warp pass");
 };
 
-// Resident blocks per SM the tile kernel is compiled for (its shared memory allows about four
-// at the largest stage): caps registers at 65536 / (32 * WPB * MINB) without forcing spills.
+// Resident blocks per SM the tile kernel is compiled for: caps registers at 65536 / (32 * WPB *
+// MINB). The gather row pass fits 102 registers (five blocks; ptxas spills 8 bytes); the
+// atomic row pass needs more and keeps four.
 #ifndef GM_BWD_TILE_MINB
-#define GM_BWD_TILE_MINB 4
+#define GM_BWD_TILE_MINB 5
 #endif
 
 template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER>
-__global__ void __launch_bounds__(WPB * 32, GM_BWD_TILE_MINB) sea_bwd_tile_kernel(SeaBwdArgs a)
+__global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
     using TG = BwdTileGeom<T, D, G, S1M>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
@@ -100,12 +102,6 @@ __global__ void __launch_bounds__(WPB * 32, GM_BWD_TILE_MINB) sea_bwd_tile_kerne
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
                 if (row < rows) {
-                    const size_t qoff = (size_t)row * (G * TG::ROW) + c * 16;
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        cp_async16(st + TG::RQ + g * TG::ROW + c * 16, static_cast<const char *>(a.q) + qoff + g * TG::ROW);
-                        cp_async16(st + TG::RG + g * TG::ROW + c * 16, static_cast<const char *>(a.dout) + qoff + g * TG::ROW);
-                    }
 #pragma unroll
                     for (int jj = 0; jj < S1M; ++jj) {
                         if (tile_lw[lr * S1M + jj] != -INFINITY) {
@@ -119,10 +115,31 @@ __global__ void __launch_bounds__(WPB * 32, GM_BWD_TILE_MINB) sea_bwd_tile_kerne
             }
             cp_async_commit();
         };
+        // q and dO chunks of a pass in registers, read one pass ahead (a pass's compute covers
+        // the loads; without them in shared memory more warps are resident)
+        auto load_qg = [&](int pass, uint4 (&qv)[G], uint4 (&gv)[G]) {
+            const uint32_t row = r0 + pass * RPW + rr;
+            const bool ok = pass < NPASS && row < rows;
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const size_t off = (size_t)row * (G * TG::ROW) + g * TG::ROW + c * 16;
+                qv[g] = ok ? ld16(static_cast<const char *>(a.q) + off) : make_uint4(0u, 0u, 0u, 0u);
+                gv[g] = ok ? ld16(static_cast<const char *>(a.dout) + off) : make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        uint4 qn[G], gn[G];
+        load_qg(0, qn, gn);
 #pragma unroll
         for (int pass = 0; pass < P; ++pass) issue(pass);
 
         for (int pass = 0; pass < NPASS; ++pass) {
+            uint4 qc[G], gc[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                qc[g] = qn[g];
+                gc[g] = gn[g];
+            }
+            load_qg(pass + 1, qn, gn);
             cp_async_wait<P - 1>();
             const int lr = pass * RPW + rr;
             const uint32_t row = r0 + lr;
@@ -140,12 +157,11 @@ __global__ void __launch_bounds__(WPB * 32, GM_BWD_TILE_MINB) sea_bwd_tile_kerne
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 float f[VEC];
-                // an invalid row (ragged tail) computes on whatever the stage holds and stores
-                // nothing
-                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RQ + g * TG::ROW + c * 16), f);
+                // an invalid row (ragged tail) computes on zeros and stores nothing
+                unpack<T>(qc[g], f);
 #pragma unroll
                 for (int x = 0; x < NP; ++x) q2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
-                unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RG + g * TG::ROW + c * 16), f);
+                unpack<T>(gc[g], f);
 #pragma unroll
                 for (int x = 0; x < NP; ++x) g2[g][x] = make_float2(f[2 * x], f[2 * x + 1]);
             }
