@@ -206,9 +206,6 @@ unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int
     return (unsigned)(need < fit ? need : fit);
 }
 
-#ifndef GM_TILE_P
-#define GM_TILE_P 2
-#endif
 #ifndef GM_WPB_TILE
 #define GM_WPB_TILE 4
 #endif
@@ -221,7 +218,10 @@ unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int
 #ifndef GM_TILE_CPL
 #define GM_TILE_CPL 1
 #endif
-constexpr int TILE_P = GM_TILE_P;  // passes of copies in flight per warp
+// Passes of K/V copies in flight per warp in the forward tile kernel: two for budgets of 2
+// (little work per pass to cover the loads), one for budgets of 4 (a pass covers them, and
+// the freed shared memory admits more warps).
+template <int S1M> constexpr int tile_passes() { return S1M >= 4 ? 1 : 2; }
 constexpr int WPB_TILE = GM_WPB_TILE;
 constexpr int TILE_CPL = GM_TILE_CPL;  // 16-byte chunks of a feature row per lane
 
@@ -236,8 +236,9 @@ template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int SF 
 gm_status launch_tile(const SerArgs &sa, const SeaArgs &a, cudaStream_t st)
 {
     using TG = gm::TileGeom<T, D, G, S1M, TILE_CPL>;
-    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, TILE_P, WPB_TILE, TILE_CPL, SF, NL>;
-    const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + TILE_P * TG::STAGE);
+    constexpr int P = tile_passes<S1M>();
+    auto kern = gm::sea_fwd_tile_kernel<T, D, G, REFER, S2, S3, S1M, P, WPB_TILE, TILE_CPL, SF, NL>;
+    const size_t smem = (size_t)WPB_TILE * (32 * S1M * 8 + P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GM_ERR_CUDA;

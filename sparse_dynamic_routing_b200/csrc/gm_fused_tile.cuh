@@ -190,12 +190,10 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
-// Resident blocks per SM the forward tile kernel is compiled for (shared memory allows six
-// 4-warp blocks at the largest stage): caps registers at 65536 / (32 * WPB * MINB) = 85
-// without spills.
-#ifndef GM_TILE_MINB
-#define GM_TILE_MINB 6
-#endif
+// Resident 4-warp blocks per SM the forward tile kernel is compiled for: caps registers at
+// 65536 / (32 * WPB * MINB) without spills. With two stages in flight shared memory admits
+// six; with one, registers (73 at seven blocks) are the limit.
+#define GM_TILE_MINB(P) ((P) == 1 ? 7 : 6)
 
 template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static constexpr int VEC = Vec<T>::N;          // elements per 16-byte chunk
@@ -216,7 +214,7 @@ template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
 // REFER = false: SEA alone on the edges a.idx / a.w (s = a.s <= S1M), sa unused.
 template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, int WPB, int CPL,
           int SF = 0, int NL = 1>
-__global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
+__global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
     using TG = TileGeom<T, D, G, S1M, CPL>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
