@@ -344,7 +344,7 @@ template <typename T, int D, int G> struct SeaBwd {
 #define GM_GATHER_U 4
 #endif
 #ifndef GM_GATHER_P
-#define GM_GATHER_P 3
+#define GM_GATHER_P 2
 #endif
 #ifndef GM_WPB_GATHER
 #define GM_WPB_GATHER 2
