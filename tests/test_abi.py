@@ -199,3 +199,14 @@ def test_chain_argument_checks(lib):
     # ..., s_mid, gout, s1, grad_is_log, B, n, k, dw1, dleg[], accumulate, stream
     assert g(FAKE, FAKE, 4, li, lw, 1, 4, 4, FAKE, 4, 0, 1, 8, 2, FAKE, NULL, 0, NULL) == bnd.GM_ERR_INVALID_ARG
     assert g(FAKE, FAKE, 4, li, lw, 1, 4, 4, FAKE, 4, 2, 1, 8, 2, FAKE, li, 0, NULL) == bnd.GM_ERR_INVALID_ARG
+
+
+def test_binding_signatures_match_the_header():
+    """Every declaration's parameter count equals the ctypes signature's (no GPU needed)."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"\b(gm_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", src, flags=re.S)
+    assert decls
+    for name, params in decls:
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(bnd.SIGNATURES[name]) == n, f"{name}: header has {n} parameters"
