@@ -55,50 +55,22 @@ template <int S> __device__ __forceinline__ void ld_vec(const float *p, float (&
     }
 }
 
-// Target of a candidate that takes no part (zero weight): unique per candidate and negative,
-// so it never equals another candidate's target.
-__device__ __forceinline__ int32_t no_target(int c) { return -2 - c; }
-
-// Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when c is
-// still nonzero and c2 shares its target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
+// Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when both
+// are still nonzero and share a target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
 // group's members are thus added to its first occurrence in ascending candidate order.
-// Candidates with zero weight carry no_target(), so an equal target implies both are live:
-// a c2 already cleared by an earlier c' shares c's target only if c' cleared c as well.
 // Unrolled (template recursion over c, an unrolled loop over c2) so the candidate arrays
 // stay in registers.
 template <int C0, int NC>
 __device__ __forceinline__ void merge_pairs(const int32_t (&ct)[NC], float (&cu)[NC])
 {
     if constexpr (C0 < NC - 1) {
-        const bool live = cu[C0] != 0.0f;  // stays so while c absorbs (weights are positive)
 #pragma unroll
         for (int c2 = C0 + 1; c2 < NC; ++c2) {
-            const bool same = live && ct[c2] == ct[C0];
+            const bool same = cu[C0] != 0.0f && cu[c2] != 0.0f && ct[c2] == ct[C0];
             cu[C0] = same ? __fadd_rn(cu[C0], cu[c2]) : cu[C0];
             cu[c2] = same ? 0.0f : cu[c2];
         }
         merge_pairs<C0 + 1, NC>(ct, cu);
-    }
-}
-
-// Keeps the S heaviest (weight desc, then target asc) of the distinct live targets offered one
-// at a time, as a sorted register list; slots never filled stay (0, 0.0f).
-template <int S>
-__device__ __forceinline__ void top_insert(float W, int32_t t, float (&bw)[S], int32_t (&bt)[S])
-{
-    if (W > bw[S - 1] || (W == bw[S - 1] && W > 0.0f && t < bt[S - 1])) {
-        bw[S - 1] = W;
-        bt[S - 1] = t;
-#pragma unroll
-        for (int x = S - 1; x > 0; --x) {
-            const bool up = bw[x] > bw[x - 1] || (bw[x] == bw[x - 1] && bt[x] < bt[x - 1]);
-            const float fw = bw[x];
-            const int32_t ft = bt[x];
-            bw[x] = up ? bw[x - 1] : bw[x];
-            bt[x] = up ? bt[x - 1] : bt[x];
-            bw[x - 1] = up ? fw : bw[x - 1];
-            bt[x - 1] = up ? ft : bt[x - 1];
-        }
     }
 }
 
@@ -142,9 +114,8 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
                 raise_index_error();
                 v = false;
             }
-            const float u = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
-            ct[x * S3 + e] = u != 0.0f ? t2[e] : no_target(x * S3 + e);
-            cu[x * S3 + e] = u;
+            ct[x * S3 + e] = t2[e];
+            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
         }
     }
     if constexpr (SF > 0) {
@@ -159,29 +130,29 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
                 raise_index_error();
                 v = false;
             }
-            ct[NP2 + f] = v ? tf[f] : no_target(NP2 + f);
+            ct[NP2 + f] = tf[f];
             cu[NP2 + f] = v ? wf[f] : 0.0f;
         }
     }
     // merge: the first occurrence of a target absorbs the later ones, in ascending order
     merge_pairs<0, NC>(ct, cu);
-    // top-s by (weight desc, index asc): the merged targets are distinct, so offering each
-    // live one to a sorted list of S_OUT gives the unique answer
-    float bw[S_OUT];
-    int32_t bt[S_OUT];
+    // top-s: repeated arg-max by (weight desc, index asc); the winner is then removed by
+    // value (nonzero targets are distinct after the merge, so the match is unique)
 #pragma unroll
     for (int r = 0; r < S_OUT; ++r) {
-        bw[r] = 0.0f;
-        bt[r] = 0;
-    }
+        float bw = 0.0f;
+        int32_t bt = 0;
 #pragma unroll
-    for (int c = 0; c < NC; ++c)
-        if (cu[c] > 0.0f) top_insert<S_OUT>(cu[c], ct[c], bw, bt);
+        for (int c = 0; c < NC; ++c) {
+            const bool better = cu[c] > bw || (cu[c] == bw && cu[c] > 0.0f && ct[c] < bt);
+            bw = better ? cu[c] : bw;
+            bt = better ? ct[c] : bt;
+        }
 #pragma unroll
-    for (int r = 0; r < S_OUT; ++r) {
-        const bool keep = r < s_keep && bw[r] > 0.0f;
-        to[r] = keep ? bt[r] : 0;
-        wo[r] = keep ? bw[r] : 0.0f;
+        for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
+        const bool keep = r < s_keep && bw > 0.0f;
+        to[r] = keep ? bt : 0;
+        wo[r] = keep ? bw : 0.0f;
     }
 }
 

@@ -144,9 +144,8 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
                 raise_index_error();
                 v = false;
             }
-            const float u = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
-            ct[x * S3 + e] = u != 0.0f ? t2[e] : no_target(x * S3 + e);
-            cu[x * S3 + e] = u;
+            ct[x * S3 + e] = t2[e];
+            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
             w2c[x * S3 + e] = w2[e];
         }
     }
@@ -154,26 +153,25 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 #pragma unroll
     for (int c = 0; c < NC; ++c) cand[c] = cu[c] != 0.0f;
     merge_pairs<0, NC>(ct, cu);
-    // selection (weight desc, target asc), as the forward's, and the upstream gradient of
-    // each kept slot
-    float bw[S1M];
-    int32_t bt[S1M];
-#pragma unroll
-    for (int r = 0; r < S1M; ++r) {
-        bw[r] = 0.0f;
-        bt[r] = 0;
-    }
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-        if (cu[c] > 0.0f) top_insert<S1M>(cu[c], ct[c], bw, bt);
+    // selection (weight desc, target asc) and the upstream gradient of each kept slot
     int32_t kt[S1M];
     float kg[S1M];
 #pragma unroll
     for (int r = 0; r < S1M; ++r) {
-        const bool keep = r < a.s1 && bw[r] > 0.0f;
+        float bw = 0.0f;
+        int32_t bt = 0;
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+            const bool better = cu[c] > bw || (cu[c] == bw && cu[c] > 0.0f && ct[c] < bt);
+            bw = better ? cu[c] : bw;
+            bt = better ? ct[c] : bt;
+        }
+#pragma unroll
+        for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
+        const bool keep = r < a.s1 && bw > 0.0f;
         float g = keep ? __ldg(b.gout + (size_t)row * a.s1 + r) : 0.0f;
-        if (b.grad_is_log) g = keep ? g / bw[r] : 0.0f;
-        kt[r] = keep ? bt[r] : -1;  // -1 never equals a live target
+        if (b.grad_is_log) g = keep ? g / bw : 0.0f;
+        kt[r] = keep ? bt : -1;  // -1 never equals a valid target
         kg[r] = g;
     }
     // per candidate: the gradient of its kept target (0 if cut)
