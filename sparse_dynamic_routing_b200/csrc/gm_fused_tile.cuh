@@ -55,18 +55,25 @@ template <int S> __device__ __forceinline__ void ld_vec(const float *p, float (&
     }
 }
 
-// Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when both
-// are still nonzero and share a target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
+// Target of a candidate that takes no part (zero weight): unique per candidate and negative,
+// so it never equals another candidate's target.
+__device__ __forceinline__ int32_t no_target(int c) { return -2 - c; }
+
+// Duplicate merge over candidate pairs (c, c2), c < c2, in lexicographic order: when c is
+// still nonzero and c2 shares its target, c absorbs c2 (one __fadd_rn) and c2 is cleared. A
 // group's members are thus added to its first occurrence in ascending candidate order.
+// Zero-weight candidates carry no_target(), so an equal target implies both are live (a c2
+// already cleared by an earlier c' shares c's target only if c' cleared c as well).
 // Unrolled (template recursion over c, an unrolled loop over c2) so the candidate arrays
 // stay in registers.
 template <int C0, int NC>
 __device__ __forceinline__ void merge_pairs(const int32_t (&ct)[NC], float (&cu)[NC])
 {
     if constexpr (C0 < NC - 1) {
+        const bool live = cu[C0] != 0.0f;  // stays so while c absorbs (weights are positive)
 #pragma unroll
         for (int c2 = C0 + 1; c2 < NC; ++c2) {
-            const bool same = cu[C0] != 0.0f && cu[c2] != 0.0f && ct[c2] == ct[C0];
+            const bool same = live && ct[c2] == ct[C0];
             cu[C0] = same ? __fadd_rn(cu[C0], cu[c2]) : cu[C0];
             cu[c2] = same ? 0.0f : cu[c2];
         }
@@ -114,8 +121,9 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
                 raise_index_error();
                 v = false;
             }
-            ct[x * S3 + e] = t2[e];
-            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+            const float u = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+            ct[x * S3 + e] = u != 0.0f ? t2[e] : no_target(x * S3 + e);
+            cu[x * S3 + e] = u;
         }
     }
     if constexpr (SF > 0) {
@@ -130,7 +138,7 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
                 raise_index_error();
                 v = false;
             }
-            ct[NP2 + f] = tf[f];
+            ct[NP2 + f] = v ? tf[f] : no_target(NP2 + f);
             cu[NP2 + f] = v ? wf[f] : 0.0f;
         }
     }

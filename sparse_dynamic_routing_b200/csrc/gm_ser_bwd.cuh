@@ -144,8 +144,9 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
                 raise_index_error();
                 v = false;
             }
-            ct[x * S3 + e] = t2[e];
-            cu[x * S3 + e] = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+            const float u = v ? __fmul_rn(w1[x], w2[e]) : 0.0f;
+            ct[x * S3 + e] = u != 0.0f ? t2[e] : no_target(x * S3 + e);
+            cu[x * S3 + e] = u;
             w2c[x * S3 + e] = w2[e];
         }
     }
