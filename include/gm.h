@@ -11,7 +11,11 @@
  *     shared by the query heads of the GQA group, score = scale * q.k + ln w, softmax over
  *     the entries, weighted sum of V;
  *   - the backward passes of both (SEA: dq, dk, dv, d ln w; SER: gradients of the kept
- *     referral weights with respect to both legs' weights).
+ *     referral weights with respect to both legs' weights);
+ *   - around the referral: the legs built from the stored edges (mixed across the k edge
+ *     channels and sparsified, gm_leg_sparsify) and their backward; refresh edges joining
+ *     the referral's candidates (gm_ser_refresh_*); multi-step referral chains
+ *     (gm_ser_chain_*), each also fused with SEA.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
