@@ -440,7 +440,9 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     takes the step's d ln w back to the legs; leg_backward takes those leg gradients back to
     the stored weights and the mixing coefficients; ser_sea_refresh_forward is the fused
     forward with the stored edges joining the referral as refresh edges;
-    ser_sea_chain_forward is the fused forward through a three-leg referral chain. Bytes are
+    ser_sea_chain_forward is the fused forward through a three-leg referral chain;
+    ser_refresh_backward and ser_chain_backward take the step's d ln w back through the
+    referral with refresh edges and through the three-leg chain. Bytes are
     compulsory: every input read once, every output written once (ser_backward's second-leg
     rows counted in full; the refresh and chain forwards' gathered rows counted from their own
     edges, the chain's third leg in full).
@@ -484,6 +486,11 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     torch.cuda.synchronize(dev)
     ch_bytes = (compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ch_i.cpu().numpy(),
                                  ch_w.cpu().numpy())["fused_forward"] + tok * k * wl.s3 * 8)
+    rf_dw1 = torch.empty((B, n, k, wl.s2), dtype=f32, device=dev)
+    rf_dw2 = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
+    rf_dfw = torch.empty((B, n, k, wl.s1), dtype=f32, device=dev)
+    ch_dw1 = torch.empty((B, n, k, wl.s2), dtype=f32, device=dev)
+    ch_dl = [torch.empty((B, n, k, wl.s3), dtype=f32, device=dev) for _ in ch_legs]
     e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
     leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
     calls = {
@@ -506,6 +513,19 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
                                       g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], ch_legs,
                                       wl.s2, wl.s1, wl.scale, out_idx=ch_i, out_w=ch_w, o=ch_o,
                                       lse=ch_lse, stream=stream)),
+        "ser_refresh_backward": ("zero_i32_kernel + ser_bwd_kernel (warp per row, refresh lanes)",
+                                 leg_b + e_b + tok * k * wl.s1 * 4 + grad_b + tok * k * wl.s1 * 4
+                                 + tok * k * wl.s3 * 4,
+                                 lambda: gm.gm_ser_refresh_backward(
+                                     g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"], le["e_idx"],
+                                     le["e_w"], dlw, grad_is_log=True, dw1=rf_dw1, dw2=rf_dw2,
+                                     dfw=rf_dfw, stream=stream)),
+        "ser_chain_backward": ("zero_i32_kernel x2 + ser_chain_bwd_kernel (3 legs)",
+                               leg_b + tok * k * wl.s3 * 8 + tok * k * wl.s1 * 4
+                               + tok * k * (wl.s2 + 2 * wl.s3) * 4 + 2 * tok * k * wl.s3 * 4,
+                               lambda: gm.gm_ser_chain_backward(
+                                   g["a1_idx"], g["a1_w"], ch_legs, wl.s2, dlw, grad_is_log=True,
+                                   dw1=ch_dw1, dlegs=ch_dl, stream=stream)),
         "leg_backward": ("leg_bwd_tile_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
                          lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,
