@@ -615,6 +615,19 @@ gm_status gm_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int 
     const SerArgs f{a1_idx, a1_w, a2_idx, a2_w, nullptr, nullptr, s1, s2, s3, n, k, (uint32_t)rows,
                     row_map(k, n), f_idx, f_w, sf};
     const gm::SerBwdArgs b{f, gout, grad_is_log, dw1, dw2, accumulate, dfw};
+    // one thread per row for the small budgets (vector loads need 16-byte aligned legs)
+    const bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w) &&
+                         aligned16(f_idx) && aligned16(f_w);
+    const unsigned tblocks = blocks_for(rows, 32 * WPB_SER_THREAD);
+    if (aligned && s2 == s3 && (s2 == 2 || s2 == 4) && s1 <= 4 && (sf == 2 || sf == 4)) {
+        if (s2 == 4)
+            sf == 4 ? gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 4><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b)
+                    : gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 2><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        else
+            sf == 4 ? gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 4><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b)
+                    : gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 2><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        return launched();
+    }
     gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
     return launched();
 }

@@ -101,10 +101,10 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
 // candidate finds the kept slot of its target, the first-leg gradient of slot a is summed
 // in ascending e, and the second-leg gradients are scatter-added with fp32 atomics. It
 // spends a fraction of the warp-per-row kernel's instructions when the budgets are 2 or 4.
-template <int S2, int S3, int S1M, int WPB>
+template <int S2, int S3, int S1M, int WPB, int SF = 0>
 __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 {
-    constexpr int NC = S2 * S3;
+    constexpr int NP2 = S2 * S3, NC = NP2 + SF;  // SF refresh slots after the paths
     const SerArgs &a = b.f;
     const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
     if (row >= a.rows) return;  // no warp-wide operation below
@@ -148,6 +148,22 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
             ct[x * S3 + e] = u != 0.0f ? t2[e] : no_target(x * S3 + e);
             cu[x * S3 + e] = u;
             w2c[x * S3 + e] = w2[e];
+        }
+    }
+    if constexpr (SF > 0) {
+        int32_t tf[SF];
+        float wf[SF];
+        ld_vec<SF>(a.f_idx + (size_t)row * SF, tf);
+        ld_vec<SF>(a.f_w + (size_t)row * SF, wf);
+#pragma unroll
+        for (int f = 0; f < SF; ++f) {
+            bool v = wf[f] > 0.0f;
+            if (v && (tf[f] < 0 || tf[f] >= a.n)) {
+                raise_index_error();
+                v = false;
+            }
+            ct[NP2 + f] = v ? tf[f] : no_target(NP2 + f);
+            cu[NP2 + f] = v ? wf[f] : 0.0f;
         }
     }
     bool cand[NC];
@@ -194,6 +210,13 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 #pragma unroll
         for (int e = 0; e < S3; ++e)
             if (gc[x * S3 + e] != 0.0f) atomicAdd(b.dw2 + r2[x] + e, gc[x * S3 + e] * w1[x]);
+    }
+    if constexpr (SF > 0) {  // refresh slots: d W / d w_f = 1
+#pragma unroll
+        for (int f = 0; f < SF; ++f) {
+            float *p = b.dfw + (size_t)row * SF + f;
+            *p = b.accumulate ? *p + gc[NP2 + f] : gc[NP2 + f];
+        }
     }
 }
 
