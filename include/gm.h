@@ -41,7 +41,7 @@
  * Errors. Argument checks are synchronous and happen before any launch:
  *   GM_ERR_INVALID_ARG  null pointer, negative size, hq % hkv != 0, non-finite scale,
  *                       misaligned feature pointer (16 bytes required), s out of [1, 32];
- *   GM_ERR_UNSUPPORTED  a valid shape this build has no kernel for (see each function);
+ *   GM_ERR_UNSUPPORTED  a valid shape the library has no kernel for (see each function);
  *   GM_ERR_CUDA         the launch failed (cudaGetLastError after the launch);
  *   GM_ERR_INDEX_RANGE  returned by gm_check_device_errors only.
  * B == 0 or n == 0 is an empty problem: GM_OK, nothing launched.

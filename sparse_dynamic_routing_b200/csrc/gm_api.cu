@@ -455,7 +455,7 @@ const char *gm_status_string(gm_status status)
     switch (status) {
     case GM_OK: return "GM_OK";
     case GM_ERR_INVALID_ARG: return "GM_ERR_INVALID_ARG: invalid argument";
-    case GM_ERR_UNSUPPORTED: return "GM_ERR_UNSUPPORTED: shape not supported by this build";
+    case GM_ERR_UNSUPPORTED: return "GM_ERR_UNSUPPORTED: no kernel in this library for the shape";
     case GM_ERR_CUDA: return "GM_ERR_CUDA: CUDA launch or synchronisation failed";
     case GM_ERR_INDEX_RANGE: return "GM_ERR_INDEX_RANGE: an active edge index was outside [0, n)";
     case GM_ERR_SCRATCH_TOO_SMALL:
