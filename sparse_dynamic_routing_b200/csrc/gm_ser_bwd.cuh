@@ -48,15 +48,16 @@ __device__ __forceinline__ float refer_step_backward(const ReferCand &c, unsigne
     const float gs = __shfl_sync(FULL, g_l, slot >= 0 ? slot : 0);
     float g = 0.0f;
     if (slot >= 0) g = grad_is_log ? gs / slot_w : gs;
-    // first leg: lane a sums its s3 candidates in ascending e
-    const float c1 = slot >= 0 ? g * c.w2 : 0.0f;
+    // first leg: lane a sums its s3 candidates in ascending e (each product and add rounded
+    // once, as in ser_bwd_thread_kernel, so both kernels give the same bits)
+    const float c1 = slot >= 0 ? __fmul_rn(g, c.w2) : 0.0f;
     float d1 = 0.0f;
     for (int e = 0; e < s3; ++e) {
         const float v = __shfl_sync(FULL, c1, (lane * s3 + e) & 31);
-        d1 += v;
+        d1 = __fadd_rn(d1, v);
     }
     // second leg: scatter to the shared second-leg rows
-    if (slot >= 0 && c.path) atomicAdd(dleg + c.r2, g * c.w1);
+    if (slot >= 0 && c.path) atomicAdd(dleg + c.r2, __fmul_rn(g, c.w1));
     g_refresh = c.refresh ? g : 0.0f;
     return lane < s_in ? d1 : 0.0f;
 }
@@ -101,6 +102,13 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
 // candidate finds the kept slot of its target, the first-leg gradient of slot a is summed
 // in ascending e, and the second-leg gradients are scatter-added with fp32 atomics. It
 // spends a fraction of the warp-per-row kernel's instructions when the budgets are 2 or 4.
+//
+// The dispatch picks this kernel or ser_bwd_kernel by shape and alignment alone, so the two
+// must agree bit for bit: the candidate products (__fmul_rn), the merge in ascending candidate
+// order (merge_pairs here and refer_thread in gm_fused_tile.cuh; __match_any_sync groups
+// summed from their first lane in refer_merge), the selection (weight descending, then target
+// ascending, zero weights never kept), g / W for a log-weight gradient, and the first-leg sums
+// (g * w2 rounded, then added in ascending e). Only dw2, summed by atomics, varies in order.
 template <int S2, int S3, int S1M, int WPB, int SF = 0>
 __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 {
@@ -204,12 +212,12 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
     for (int x = 0; x < S2; ++x) {
         float d1 = 0.0f;
 #pragma unroll
-        for (int e = 0; e < S3; ++e) d1 += gc[x * S3 + e] * w2c[x * S3 + e];
+        for (int e = 0; e < S3; ++e) d1 = __fadd_rn(d1, __fmul_rn(gc[x * S3 + e], w2c[x * S3 + e]));
         float *p = b.dw1 + (size_t)row * S2 + x;
         *p = b.accumulate ? *p + d1 : d1;
 #pragma unroll
         for (int e = 0; e < S3; ++e)
-            if (gc[x * S3 + e] != 0.0f) atomicAdd(b.dw2 + r2[x] + e, gc[x * S3 + e] * w1[x]);
+            if (gc[x * S3 + e] != 0.0f) atomicAdd(b.dw2 + r2[x] + e, __fmul_rn(gc[x * S3 + e], w1[x]));
     }
     if constexpr (SF > 0) {  // refresh slots: d W / d w_f = 1
 #pragma unroll

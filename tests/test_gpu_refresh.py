@@ -66,8 +66,11 @@ def case(seed, B, n, k, s2, s3, sf, zero_frac=0.1):
     return e(s2), e(s3), e(sf), rng
 
 
+# (2,2,2,2), (4,4,4,4), (2,2,4,3), (4,4,2,2), (4,4,4,1) reach the per-thread backward (s1 < s2
+# leaves slots unkept); the others the warp-per-row kernel
 @pytest.mark.parametrize("s2,s3,sf,s1,n", [(2, 2, 2, 2, 128), (4, 4, 4, 4, 300), (4, 4, 8, 8, 97),
-                                           (2, 2, 1, 3, 61), (1, 1, 6, 4, 33), (3, 3, 5, 8, 45)])
+                                           (2, 2, 1, 3, 61), (1, 1, 6, 4, 33), (3, 3, 5, 8, 45),
+                                           (2, 2, 4, 3, 150), (4, 4, 2, 2, 77), (4, 4, 4, 1, 64)])
 def test_refresh_referral_forward_and_backward(s2, s3, sf, s1, n):
     B, k = 2, 3
     (i1, w1), (i2, w2), (fi, fw), rng = case(s2 * 100 + s3 * 10 + sf, B, n, k, s2, s3, sf)
@@ -152,4 +155,70 @@ def test_fused_refresh_forward_bf16_tile_shapes(s, sf, s1):
     assert_bits(ai, aw, oi, ow)
     assert_close(o, o_ref, 2e-2, "o")
     assert_close(lse, lse_ref, 2e-2, "lse")
+    gm.gm_check_device_errors()
+
+
+def misaligned(a):
+    """`a` copied to the GPU at a data pointer 4 bytes past a 16-byte boundary: the dispatch
+    then takes the warp-per-row kernels instead of the per-thread ones."""
+    src = torch.from_numpy(np.ascontiguousarray(a))
+    flat = torch.empty(src.numel() + 4, dtype=src.dtype, device="cuda")
+    view = flat[1:1 + src.numel()].view(src.shape)
+    view.copy_(src)
+    assert view.data_ptr() % 16 == 4
+    return view
+
+
+def tie_case(seed, n, k, s2, s3, sf):
+    """Targets from {0..3} and weights from {0, 1/8, 1/4, 1/2}: duplicate targets in most rows
+    and exact ties between merged weights, so the tie-break decides the kept set."""
+    rng = np.random.default_rng(seed)
+
+    def e(s):
+        idx = np.minimum(rng.integers(0, 4, (1, n, k, s)), np.arange(n)[None, :, None, None])
+        w = rng.choice(np.float32([0.0, 0.125, 0.25, 0.5]), (1, n, k, s))
+        return idx.astype(np.int32), w.astype(np.float32)
+
+    return e(s2), e(s3), e(sf), rng.standard_normal((1, n, k, 4)).astype(np.float32)
+
+
+@pytest.mark.parametrize("s,sf", [(2, 0), (4, 0), (2, 2), (2, 4), (4, 2), (4, 4)])
+def test_thread_and_warp_backward_agree_bit_for_bit_on_ties(s, sf):
+    """The per-thread and warp-per-row referral backwards are chosen by shape and alignment
+    alone, so they must keep the same slots and give the same first-leg and refresh-slot
+    gradient bits; the second-leg gradient (fp32 atomics) only to rounding order."""
+    n, k, s1 = 96, 2, 4
+    (i1, w1), (i2, w2), (fi, fw), g = tie_case(500 + 10 * s + sf, n, k, s, s, max(sf, 1))
+    if sf:
+        args = (i1, w1, i2, w2, fi, fw)
+        thread = gm.gm_ser_refresh_backward(*[t(a) for a in args], t(g), grad_is_log=True)
+        warp = gm.gm_ser_refresh_backward(*[misaligned(a) for a in args], t(g), grad_is_log=True)
+        ref = oracle.ser_refresh_backward(*args, g, grad_is_log=True)
+        names = ("dw1", "dw2", "dfw")
+    else:
+        args = (i1, w1, i2, w2)
+        thread = gm.gm_ser_backward(*[t(a) for a in args], t(g), grad_is_log=True)
+        warp = gm.gm_ser_backward(*[misaligned(a) for a in args], t(g), grad_is_log=True)
+        ref = oracle.ser_backward(*args, g, grad_is_log=True)
+        names = ("dw1", "dw2")
+    for name, a, b, r in zip(names, thread, warp, ref):
+        assert_rel(a, r, f"thread {name}")
+        assert_rel(b, r, f"warp {name}")
+        if name != "dw2":
+            np.testing.assert_array_equal(host(a).view(np.uint32), host(b).view(np.uint32),
+                                          err_msg=name)
+    # the forward: the fused tile kernel's per-thread referral against the warp kernel
+    gen = torch.Generator().manual_seed(s + sf)
+    q = torch.randn((1, n, 2 * k, 128), generator=gen).to(torch.bfloat16).cuda()
+    kv = torch.randn((1, n, k, 128), generator=gen).to(torch.bfloat16).cuda()
+    if sf:
+        wi, ww = gm.gm_ser_refresh_forward(*[t(a) for a in args], s1)
+        fi_, fw_, _, _ = gm.gm_ser_sea_refresh_forward(q, kv, kv, *[t(a) for a in args], s1)
+        oi, ow, _ = oracle.ser_refresh(*args, s1)
+    else:
+        wi, ww = gm.gm_ser_forward(*[t(a) for a in args], s1)
+        fi_, fw_, _, _ = gm.gm_ser_sea_forward(q, kv, kv, *[t(a) for a in args], s1)
+        oi, ow, _ = oracle.ser(*args, s1)
+    assert_bits(wi, ww, oi, ow)
+    assert_bits(fi_, fw_, oi, ow)
     gm.gm_check_device_errors()

@@ -4,13 +4,15 @@ Such callers (code inside an allocator's own hooks, runtimes whose device memory
 to their own pool, step loops that forbid allocation because it can synchronise the device)
 cannot hand gm_sea_backward a workspace. The no-alloc entry point runs the same gather path
 on a fixed scratch array the library keeps on each device. This file checks, through the C
-ABI, that two calls in a row give what the workspace entry point gives, and that a problem
-too large for the array is refused before anything runs. It is collected last on purpose.
+ABI, that two calls in a row give what the workspace entry point gives and what the fp64
+oracle gives, and that a problem too large for the array is refused before anything runs. It
+is collected last on purpose.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import sparse_dynamic_routing_b200 as gm
 from sparse_dynamic_routing_b200 import _binding as bnd
 from sparse_dynamic_routing_b200 import inputs as I
@@ -33,13 +35,20 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls():
     assert 0 < need <= bnd.load_library().gm_sea_backward_noalloc_max_scratch()
     ref = gm.gm_sea_backward(x["q"], x["k"], x["v"], x["dout"], x["idx"], x["w"], wl.scale,
                              workspace="auto")
+    # both GPU paths are also held to the fp64 oracle on the same bf16 inputs
+    host = I.make(wl, grad=True)
+    want = oracle.sea_backward(host["q"], host["k"], host["v"], host["dout"], host["idx"],
+                               host["w"], wl.scale)[:4]
     for call in range(2):
         got = gm.gm_sea_backward_noalloc(x["q"], x["k"], x["v"], x["dout"], x["idx"], x["w"],
                                          wl.scale)
         gm.gm_check_device_errors()
-        for name, a, b in zip(("dq", "dk", "dv", "dlogw"), got, ref):
+        for name, a, b, w in zip(("dq", "dk", "dv", "dlogw"), got, ref, want):
             err = _max_abs(a, b)
             assert np.isfinite(err) and err <= TOL, f"call {call}: {name} differs by {err}"
+            w = torch.from_numpy(w).reshape(a.shape)
+            err = _max_abs(a.cpu(), w)
+            assert np.isfinite(err) and err <= TOL, f"call {call}: {name} vs oracle: {err}"
         # dq and d ln w come from the same row pass in the same order: identical bits
         assert torch.equal(got[0], ref[0]) and torch.equal(got[3], ref[3])
 
