@@ -1,4 +1,5 @@
-"""CPU oracle of the Graph Machine sparse layer (leg sparsification, SER, SEA, and their backward passes).
+"""CPU oracle of the Graph Machine sparse layer (leg sparsification, SER, SEA, their backward
+passes, and refresh edges from a dense attention layer).
 
 TEST INFRASTRUCTURE. Only the tests, the package smoke check and the benchmark's CPU-baseline
 leg import this module. It wraps the plain C library built from gm_oracle.c (compiled on
@@ -54,6 +55,14 @@ def _load():
         lib.oracle_ser_refresh_backward.restype = ctypes.c_int64
         lib.oracle_ser_refresh_backward.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci,
                                                     f32p, ci, ci, ci, ci, ci, f64p, f64p, f64p]
+        lib.oracle_dense_lse.restype = None
+        lib.oracle_dense_lse.argtypes = [f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double, f64p]
+        lib.oracle_dense_mass.restype = None
+        lib.oracle_dense_mass.argtypes = [f32p, f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double,
+                                          ctypes.c_void_p, ctypes.c_int64, f64p]
+        lib.oracle_dense_refresh.restype = None
+        lib.oracle_dense_refresh.argtypes = [f32p, f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double,
+                                             ci, ctypes.c_void_p, ctypes.c_int64, i32p, f32p]
         _lib = lib
     return _lib
 
@@ -289,3 +298,53 @@ def ser_chain_backward(a1_idx, a1_w, legs, s_mid: int, gout, grad_is_log: bool =
         dlegs[m] = d_leg
         g = d_first.astype(np.float32)
     return d_first, dlegs, bad
+
+
+def _rows(rows):
+    if rows is None:
+        return None, None, 0
+    r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    return r, r.ctypes.data_as(ctypes.c_void_p), int(r.size)
+
+
+def dense_lse(q, k, scale: float | None = None):
+    """Normaliser of causal softmax attention per (b, i, hq), fp64 [B, n, hq]: the lse a dense
+    attention layer's forward returns."""
+    qf, kf = _np(q, np.float32), _np(k, np.float32)
+    B, n, hq, d = qf.shape
+    hkv = kf.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    out = np.zeros((B, n, hq), np.float64)
+    _load().oracle_dense_lse(qf, kf, B, n, hq, hkv, d, scale, out)
+    return out
+
+
+def dense_mass(q, k, lse, scale: float | None = None, rows=None):
+    """Attention mass of each KV head at every position, the mean over its query heads of the
+    causal softmax probabilities, fp64 [nrows, hkv, n] (zero for t > i). rows: flat b*n + i."""
+    qf, kf, lf = _np(q, np.float32), _np(k, np.float32), _np(lse, np.float32)
+    B, n, hq, d = qf.shape
+    hkv = kf.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    r, rp, nr = _rows(rows)
+    nrows = B * n if r is None else nr
+    out = np.zeros((nrows, hkv, n), np.float64)
+    _load().oracle_dense_mass(qf, kf, lf, B, n, hq, hkv, d, scale, rp, nr, out)
+    return out
+
+
+def dense_refresh(q, k, lse, sf: int, scale: float | None = None, rows=None):
+    """Refresh edges from a dense attention layer: per (b, i, h) the sf positions t <= i with
+    the largest attention mass of KV head h (ties: smaller t), weights = that mass in fp32,
+    padded with (0, 0.0). lse is the dense layer's fp32 normaliser [B, n, hq]. Returns
+    (idx int32, w fp32), [B, n, hkv, sf], or [nrows, hkv, sf] for a list of flat rows."""
+    qf, kf, lf = _np(q, np.float32), _np(k, np.float32), _np(lse, np.float32)
+    B, n, hq, d = qf.shape
+    hkv = kf.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    r, rp, nr = _rows(rows)
+    shape = (B, n, hkv, sf) if r is None else (nr, hkv, sf)
+    oi = np.zeros(shape, np.int32)
+    ow = np.zeros(shape, np.float32)
+    _load().oracle_dense_refresh(qf, kf, lf, B, n, hq, hkv, d, scale, sf, rp, nr, oi, ow)
+    return oi, ow

@@ -68,6 +68,16 @@
  *       Sparsify_s1(A1 A2 + F). Candidate order: the paths in ascending c = a*s3 + e, then
  *       the refresh slots in ascending f; merge, order and cut as R2-R5. A kept target's
  *       merged weight passes its gradient unchanged to every refresh slot that reaches it.
+ *   R14 the dense layer whose top positions give refresh edges is plain causal softmax
+ *       attention: query head hq of token i gives position t <= i the probability
+ *       P[hq](i, t) = exp(scale <q[i,hq], k[t,h]> - lse[i,hq]), h = hq / (Hq / Hkv), where
+ *       lse[i,hq] is the natural-log normaliser of that row, as the dense layer's forward
+ *       returns it (oracle_dense_lse computes it from the definition).
+ *   R15 the refresh edges of (b, i, h) are the sf positions t <= i with the largest attention
+ *       mass of KV head h: the mean of P[hq](i, t) over the query heads hq of its group. The
+ *       edge weight is that mean (computed in fp64, rounded to fp32); ties go to the smaller
+ *       position; rows with fewer than sf positions (i + 1 < sf) are padded with (index 0,
+ *       weight 0.0f); the slots are ordered by mass descending, then position ascending.
  *
  * Layouts are contiguous row-major: features [B, n, H, d], edges [B, n, k, s].
  */
@@ -754,4 +764,117 @@ int64_t oracle_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, in
         }
     }
     return bad;
+}
+
+/* ------------------------------------------------------------------------------------------
+ * Refresh edges from the latest dense attention layer   [MF5], and the last sentence of the
+ * referral paragraph of "Methodology in Plain English": refresh edges are the input edges or
+ * the top positions of the most recent dense attention layer. Readings R14, R15.
+ * ---------------------------------------------------------------------------------------- */
+
+/* <q[b,i,hq], k[b,t,h]> in fp64 on inputs widened exactly from fp32 / bf16. */
+static double dense_dot(const float *q, const float *kk, int64_t b, int i, int t, int hqi, int h,
+                        int n, int hq, int hkv, int d)
+{
+    const float *qrow = q + (((int64_t)b * n + i) * hq + hqi) * d;
+    const float *krow = kk + (((int64_t)b * n + t) * hkv + h) * d;
+    double dot = 0.0;
+    for (int x = 0; x < d; ++x) dot += (double)qrow[x] * (double)krow[x];
+    return dot;
+}
+
+/* lse [B, n, hq]: log of sum over t <= i of exp(scale <q[b,i,hq], k[b,t,h]>), the normaliser
+ * of causal softmax attention (R14). */
+void oracle_dense_lse(const float *q, const float *kk, int B, int n, int hq, int hkv, int d,
+                      double scale, double *lse)
+{
+    const int G = hq / hkv;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t bi = 0; bi < (int64_t)B * n; ++bi) {
+        const int64_t b = bi / n;
+        const int i = (int)(bi % n);
+        double *z = (double *)malloc(sizeof(double) * (size_t)(i + 1));
+        for (int hqi = 0; hqi < hq; ++hqi) {
+            const int h = hqi / G;
+            double m = -INFINITY;
+            for (int t = 0; t <= i; ++t) {
+                z[t] = scale * dense_dot(q, kk, b, i, t, hqi, h, n, hq, hkv, d);
+                m = z[t] > m ? z[t] : m;
+            }
+            double l = 0.0;
+            for (int t = 0; t <= i; ++t) l += exp(z[t] - m);
+            lse[bi * hq + hqi] = m + log(l);
+        }
+        free(z);
+    }
+}
+
+/* Attention mass of KV head h at every position (R14, R15): mass[r, h, t] = mean over the
+ * group's query heads of exp(scale <q, k[t]> - lse) for t <= i, 0 for t > i, for the flat
+ * positions rows[r] = b*n + i (NULL: all B*n in order). */
+void oracle_dense_mass(const float *q, const float *kk, const float *lse, int B, int n, int hq,
+                       int hkv, int d, double scale, const int64_t *rows, int64_t nrows,
+                       double *mass)
+{
+    const int G = hq / hkv;
+    if (rows == NULL) nrows = (int64_t)B * n;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t bi = rows ? rows[r] : r;
+        const int64_t b = bi / n;
+        const int i = (int)(bi % n);
+        for (int h = 0; h < hkv; ++h) {
+            double *mrow = mass + (r * hkv + h) * (int64_t)n;
+            for (int t = 0; t < n; ++t) mrow[t] = 0.0;
+            for (int hqi = h * G; hqi < (h + 1) * G; ++hqi) {
+                const double l = (double)lse[bi * hq + hqi];
+                for (int t = 0; t <= i; ++t)
+                    mrow[t] += exp(scale * dense_dot(q, kk, b, i, t, hqi, h, n, hq, hkv, d) - l);
+            }
+            for (int t = 0; t <= i; ++t) mrow[t] /= (double)G;
+        }
+    }
+}
+
+typedef struct {
+    double mass;
+    int32_t t;
+} dense_entry;
+
+/* mass descending, then position ascending (R15) */
+static int dense_entry_order(const void *pa, const void *pb)
+{
+    const dense_entry *a = (const dense_entry *)pa, *b = (const dense_entry *)pb;
+    if (a->mass != b->mass) return a->mass > b->mass ? -1 : 1;
+    return (a->t > b->t) - (a->t < b->t);
+}
+
+/* Refresh edges [nrows, hkv, sf] (R15) from the masses of oracle_dense_mass: all positions
+ * t <= i sorted by (mass desc, t asc), the first sf kept, the rest padded with (0, 0.0f). */
+void oracle_dense_refresh(const float *q, const float *kk, const float *lse, int B, int n,
+                          int hq, int hkv, int d, double scale, int sf, const int64_t *rows,
+                          int64_t nrows, int32_t *out_idx, float *out_w)
+{
+    if (rows == NULL) nrows = (int64_t)B * n;
+    double *mass = (double *)malloc(sizeof(double) * (size_t)nrows * hkv * n);
+    oracle_dense_mass(q, kk, lse, B, n, hq, hkv, d, scale, rows, nrows, mass);
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t bi = rows ? rows[r] : r;
+        const int i = (int)(bi % n);
+        dense_entry *e = (dense_entry *)malloc(sizeof(dense_entry) * (size_t)(i + 1));
+        for (int h = 0; h < hkv; ++h) {
+            for (int t = 0; t <= i; ++t) {
+                e[t].mass = mass[(r * hkv + h) * (int64_t)n + t];
+                e[t].t = t;
+            }
+            qsort(e, (size_t)(i + 1), sizeof(dense_entry), dense_entry_order);
+            for (int f = 0; f < sf; ++f) {
+                out_idx[(r * hkv + h) * sf + f] = f <= i ? e[f].t : 0;
+                out_w[(r * hkv + h) * sf + f] = f <= i ? (float)e[f].mass : 0.0f;
+            }
+        }
+        free(e);
+    }
+    free(mass);
 }
