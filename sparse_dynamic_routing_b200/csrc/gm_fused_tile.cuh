@@ -10,14 +10,17 @@
 //    the s3 second-leg slots behind each (vector loads), forms the s2*s3 candidates in
 //    registers, merges duplicates in ascending candidate order (the first occurrence
 //    accumulates the later ones with __fadd_rn), and selects the s1 heaviest (weight desc,
-//    index asc) by repeated arg-max. Results: A' to global memory (once, for the next layer)
-//    and to a shared-memory tile with log2 weights for phase 2.
+//    index asc) through a compare-exchange chain on 64-bit (weight, ~index) keys. Results: A'
+//    to global memory (once, for the next layer) and to a shared-memory tile with log2
+//    weights for phase 2.
 //  Phase 2 - attention, C lanes (one 16-byte chunk each) per row, 32 / C rows per pass. Each
 //    lane handles its chunk for all G query heads of the group, so a K/V chunk is unpacked
 //    once and used G times, with packed fp32x2 FMAs. The lane stages exactly the K/V chunks
 //    it will read with 16-byte cp.async, P passes ahead, so every byte in flight sits in
-//    shared memory, and completion needs no spin-wait (cp.async.wait_group); its q chunks
-//    go straight to registers one pass ahead.
+//    shared memory, and completion needs no spin-wait (cp.async.wait_group); an inactive
+//    slot's copy reads nothing and fills zeros, so every slot is computed without a branch.
+//    Its q chunks go straight to registers one pass ahead. The softmax normalises the
+//    probabilities before the weighted sum of V, so the output needs no division.
 // All shuffles run on all 32 lanes: slots are padded to S1M and inactive ones masked after
 // the reduction, so rows at a ragged tail simply compute on zeros and store nothing.
 #pragma once
@@ -98,7 +101,7 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
 #pragma unroll
     for (int x = 0; x < S_IN; ++x) {
         bool act = w1[x] > 0.0f;
-        if (act && (j[x] < 0 || j[x] >= a.n)) {
+        if (act && (uint32_t)j[x] >= (uint32_t)a.n) {
             raise_index_error();
             act = false;
         }
@@ -117,7 +120,7 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
 #pragma unroll
         for (int e = 0; e < S3; ++e) {
             bool v = w2[e] > 0.0f;
-            if (v && (t2[e] < 0 || t2[e] >= a.n)) {
+            if (v && (uint32_t)t2[e] >= (uint32_t)a.n) {
                 raise_index_error();
                 v = false;
             }
@@ -134,7 +137,7 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
 #pragma unroll
         for (int f = 0; f < SF; ++f) {
             bool v = wf[f] > 0.0f;
-            if (v && (tf[f] < 0 || tf[f] >= a.n)) {
+            if (v && (uint32_t)tf[f] >= (uint32_t)a.n) {
                 raise_index_error();
                 v = false;
             }
@@ -144,23 +147,30 @@ __device__ __forceinline__ void refer_thread(const SerArgs &a, uint32_t row, uin
     }
     // merge: the first occurrence of a target absorbs the later ones, in ascending order
     merge_pairs<0, NC>(ct, cu);
-    // top-s: repeated arg-max by (weight desc, index asc); the winner is then removed by
-    // value (nonzero targets are distinct after the merge, so the match is unique)
+    // top-s: each merged candidate enters a sorted list of S_OUT 64-bit keys (weight bits,
+    // then the complemented target: positive fp32 weights order as their bit patterns, so
+    // the larger key is the heavier target, the smaller index on equal weights; a zero
+    // weight is key 0 and never enters) by a chain of compare-exchanges, no branches
+    unsigned long long key[S_OUT];
+#pragma unroll
+    for (int r = 0; r < S_OUT; ++r) key[r] = 0ull;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+        unsigned long long kc = cu[c] > 0.0f
+                                    ? ((unsigned long long)__float_as_uint(cu[c]) << 32) | (uint32_t)~ct[c]
+                                    : 0ull;
+#pragma unroll
+        for (int r = 0; r < S_OUT; ++r) {
+            const unsigned long long hi = kc > key[r] ? kc : key[r];
+            kc = kc > key[r] ? key[r] : kc;
+            key[r] = hi;
+        }
+    }
 #pragma unroll
     for (int r = 0; r < S_OUT; ++r) {
-        float bw = 0.0f;
-        int32_t bt = 0;
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-            const bool better = cu[c] > bw || (cu[c] == bw && cu[c] > 0.0f && ct[c] < bt);
-            bw = better ? cu[c] : bw;
-            bt = better ? ct[c] : bt;
-        }
-#pragma unroll
-        for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
-        const bool keep = r < s_keep && bw > 0.0f;
-        to[r] = keep ? bt : 0;
-        wo[r] = keep ? bw : 0.0f;
+        const bool keep = r < s_keep && key[r] != 0ull;
+        to[r] = keep ? (int32_t)~(uint32_t)key[r] : 0;
+        wo[r] = keep ? __uint_as_float((uint32_t)(key[r] >> 32)) : 0.0f;
     }
 }
 
@@ -198,10 +208,33 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
+// The S entries of one row of a warp's shared-memory edge tile (16-byte aligned for S = 4,
+// 8-byte for S = 2), read as one vector.
+template <int S, typename V> __device__ __forceinline__ void ld_tile(const V *p, V (&o)[S])
+{
+    static_assert(sizeof(V) == 4, "32-bit tile entries");
+    if constexpr (S == 4) {
+        const uint4 u = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) o[x] = *reinterpret_cast<const V *>(&w[x]);
+    } else if constexpr (S == 2) {
+        const uint2 u = *reinterpret_cast<const uint2 *>(p);
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int x = 0; x < 2; ++x) o[x] = *reinterpret_cast<const V *>(&w[x]);
+    } else {
+#pragma unroll
+        for (int x = 0; x < S; ++x) o[x] = p[x];
+    }
+}
+
 // Resident 4-warp blocks per SM the forward tile kernel is compiled for: caps registers at
 // 65536 / (32 * WPB * MINB) without spills. With two stages in flight shared memory admits
 // six; with one, registers (73 at seven blocks) are the limit.
+#ifndef GM_TILE_MINB
 #define GM_TILE_MINB(P) ((P) == 1 ? 7 : 6)
+#endif
 
 template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {
     static constexpr int VEC = Vec<T>::N;          // elements per 16-byte chunk
@@ -243,6 +276,9 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
     const float sl2 = a.scale * LOG2E;
     const T *Qg = static_cast<const T *>(a.q);
     T *O = static_cast<T *>(a.o);
+    // this lane's first chunk of K/V row 0: a gathered row's chunk is one wide multiply-add away
+    const char *kbase = static_cast<const char *>(a.k) + (size_t)(c * CPL) * 16;
+    const char *vbase = static_cast<const char *>(a.v) + (size_t)(c * CPL) * 16;
 
     for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
         const uint32_t r0 = tile * 32;
@@ -310,18 +346,21 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                 const int lr = pass * RPW + rr;  // row within the tile
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
-                if (row < rows) {
+                // every slot of a valid row is copied; an inactive one (or a row past the end)
+                // reads nothing and gets zeros, so no branch and no stale data
+                float lwv[S1M];
+                int32_t tv[S1M];
+                ld_tile<S1M>(tile_lw + lr * S1M, lwv);
+                ld_tile<S1M>(tile_t + lr * S1M, tv);
 #pragma unroll
-                    for (int jj = 0; jj < S1M; ++jj) {
-                        if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const uint32_t kvrow = (uint32_t)tile_t[lr * S1M + jj];
+                for (int jj = 0; jj < S1M; ++jj) {
+                    const bool live = row < rows && lwv[jj] != -INFINITY;
+                    const uint32_t kvrow = live ? (uint32_t)tv[jj] : 0u;
 #pragma unroll
-                            for (int cc = 0; cc < CPL; ++cc) {
-                                const size_t off = (size_t)kvrow * TG::ROW + (c * CPL + cc) * 16;
-                                cp_async16(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16, static_cast<const char *>(a.k) + off);
-                                cp_async16(st + TG::RV + jj * TG::ROW + (c * CPL + cc) * 16, static_cast<const char *>(a.v) + off);
-                            }
-                        }
+                    for (int cc = 0; cc < CPL; ++cc) {
+                        const size_t off = (size_t)kvrow * TG::ROW + cc * 16;
+                        cp_async16_zfill(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16, kbase + off, live);
+                        cp_async16_zfill(st + TG::RV + jj * TG::ROW + (c * CPL + cc) * 16, vbase + off, live);
                     }
                 }
             }
@@ -360,11 +399,9 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
 
             float lw[S1M];
             bool act[S1M];
+            ld_tile<S1M>(tile_lw + lr * S1M, lw);
 #pragma unroll
-            for (int jj = 0; jj < S1M; ++jj) {
-                lw[jj] = tile_lw[lr * S1M + jj];
-                act[jj] = valid && lw[jj] != -INFINITY;
-            }
+            for (int jj = 0; jj < S1M; ++jj) act[jj] = valid && lw[jj] != -INFINITY;
             // q chunks of the G heads as fp32 pairs
             float2 q2[G][CPL * NP];
 #pragma unroll
@@ -379,12 +416,14 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                 }
             }
             float2 acc[G][CPL * NP];
-            float m[G], l[G];
-#pragma unroll
-            for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int x = 0; x < CPL * NP; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
+            float m[G] = {}, l[G] = {};
             constexpr int NV = G * S1M;  // (slot, head) scores per row
+            if (NV > C) {  // the distributed softmax's first slot product initialises it
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int x = 0; x < CPL * NP; ++x) acc[g][x] = make_float2(0.0f, 0.0f);
+            }
             if constexpr (NV <= C) {
                 // Distributed softmax. The NV partial dots are reduced across the row's C lanes
                 // by a transposed butterfly: each step sends half of the remaining values to
@@ -400,7 +439,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) {
                         float f[VEC];
-                        // an inactive slot's stage holds stale data: its score is masked below
+                        // an inactive slot's stage holds zeros: its score is masked below
                         unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16), f);
 #pragma unroll
                         for (int x = 0; x < VEC; ++x) kf[cc * VEC + x] = f[x];
@@ -432,20 +471,21 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                 float lz = p;
 #pragma unroll
                 for (int off = G * SPREAD; off < C; off <<= 1) lz += __shfl_xor_sync(FULL, lz, off);
+                // normalised probability (the sum is >= 1 when the head has an active slot: its
+                // largest term is exp2(0)); the lane of slot 0 of each head stores its lse
+                const float pn = lz > 0.0f ? p * rcp_fast(lz) : 0.0f;
+                if (valid && a.lse != nullptr && vi < G && (lane & (SPREAD - 1)) == 0)
+                    a.lse[(size_t)row * G + vi] = lz > 0.0f ? (mz + lg2(lz)) * LN2 : -INFINITY;
                 const int seg = lane & ~(C - 1);
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    m[g] = __shfl_sync(FULL, mz, seg + g * SPREAD);
-                    l[g] = __shfl_sync(FULL, lz, seg + g * SPREAD);
-                }
                 float pp[S1M][G];
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj)
 #pragma unroll
-                    for (int g = 0; g < G; ++g) pp[jj][g] = __shfl_sync(FULL, p, seg + (jj * G + g) * SPREAD);
+                    for (int g = 0; g < G; ++g) pp[jj][g] = __shfl_sync(FULL, pn, seg + (jj * G + g) * SPREAD);
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj) {
-                    if (!act[jj]) continue;  // per lane; no shuffles below
+                    // zero-filled stages: an inactive slot has p = 0 and V = 0, so every slot is
+                    // accumulated without a branch, the first one by a multiply
                     float vf[CPL * VEC];
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) {
@@ -458,8 +498,13 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                     for (int g = 0; g < G; ++g) {
                         const float2 p2 = make_float2(pp[jj][g], pp[jj][g]);
 #pragma unroll
-                        for (int x2 = 0; x2 < CPL * NP; ++x2)
-                            acc[g][x2] = __ffma2_rn(p2, make_float2(vf[2 * x2], vf[2 * x2 + 1]), acc[g][x2]);
+                        for (int x2 = 0; x2 < CPL * NP; ++x2) {
+                            const float2 v2 = make_float2(vf[2 * x2], vf[2 * x2 + 1]);
+                            if (jj == 0)
+                                acc[g][x2] = __fmul2_rn(p2, v2);
+                            else
+                                acc[g][x2] = __ffma2_rn(p2, v2, acc[g][x2]);
+                        }
                     }
                 }
             } else {
@@ -471,7 +516,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc) {
                     float f[VEC];
-                    // an inactive slot's stage holds stale data: its score is masked below
+                    // an inactive slot's stage holds zeros: its score is masked below
                     unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + (c * CPL + cc) * 16), f);
 #pragma unroll
                     for (int x = 0; x < VEC; ++x) kf[cc * VEC + x] = f[x];
@@ -523,19 +568,20 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
             if (valid) {
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const bool nonempty = l[g] > 0.0f;
-                    const float inv = nonempty ? __frcp_rn(l[g]) : 0.0f;
+                    // the distributed softmax accumulated normalised probabilities already
+                    const bool nonempty = NV <= C || l[g] > 0.0f;
+                    const float inv = NV <= C ? 1.0f : (nonempty ? __frcp_rn(l[g]) : 0.0f);
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) {
                         float of[VEC];
 #pragma unroll
                         for (int x = 0; x < NP; ++x) {
-                            of[2 * x] = acc[g][cc * NP + x].x * inv;
-                            of[2 * x + 1] = acc[g][cc * NP + x].y * inv;
+                            of[2 * x] = NV <= C ? acc[g][cc * NP + x].x : acc[g][cc * NP + x].x * inv;
+                            of[2 * x + 1] = NV <= C ? acc[g][cc * NP + x].y : acc[g][cc * NP + x].y * inv;
                         }
                         *reinterpret_cast<uint4 *>(O + ((size_t)row * G + g) * D + (c * CPL + cc) * VEC) = pack<T>(of);
                     }
-                    if (a.lse != nullptr && c == 0)
+                    if (NV > C && a.lse != nullptr && c == 0)
                         a.lse[(size_t)row * G + g] = nonempty ? (m[g] + lg2(l[g])) * LN2 : -INFINITY;
                 }
             }
