@@ -65,7 +65,8 @@ typedef enum gm_status {
     GM_ERR_UNSUPPORTED = 2,
     GM_ERR_CUDA = 3,
     GM_ERR_INDEX_RANGE = 4,
-    GM_ERR_SCRATCH_TOO_SMALL = 5  /* gm_sea_backward_noalloc only */
+    GM_ERR_SCRATCH_TOO_SMALL = 5, /* gm_sea_backward_noalloc only */
+    GM_ERR_WAIT_TIMEOUT = 6       /* from gm_check_device_errors: a kernel gave up on a wait */
 } gm_status;
 
 /* Element type of q, k, v, o and dout. */
@@ -435,10 +436,43 @@ gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, c
 size_t gm_sea_backward_noalloc_max_scratch(void);
 
 /*
+ * gm_dense_refresh_edges - refresh edges from a dense attention layer: for every (b, i, KV
+ * head h), the sf positions t <= i that the dense layer's attention weights most heavily.
+ * Source: ai.info summary, "Methodology in Plain English", referral paragraph (refresh edges
+ * are the input edges or the top positions of the most recent dense attention layer); "Main
+ * Findings", bullet on refresh and realignment. Reading of the pages (they give no formula):
+ * the dense layer is causal softmax attention, P_hq(i, t) = exp(scale <q[i,hq], k[t,h]> -
+ * lse[i,hq]) for t <= i, h = hq / (hq_count / hkv); the attention mass of KV head h at t is
+ * the mean of P_hq(i, t) over the query heads of its group; the sf positions of largest mass
+ * are kept, ties to the smaller position, ordered by mass descending; the edge weight is the
+ * mass. Rows with i + 1 < sf are padded with (index 0, weight 0.0f). The result [B, n, hkv, sf]
+ * is an edge set for gm_ser_refresh_forward / gm_ser_sea_refresh_forward (k = hkv).
+ *
+ *   q         [B, n, hq, d]  bf16, the dense layer's queries
+ *   k         [B, n, hkv, d] bf16, the dense layer's keys
+ *   dtype     GM_BF16 (fp32 features: GM_ERR_UNSUPPORTED)
+ *   lse       [B, n, hq] fp32: the dense layer's per-row normaliser (natural log), as its
+ *             forward returns it
+ *   scale     the dense layer's score scale (1/sqrt(d) for standard attention)
+ *   sf        1..8 positions kept per (b, i, h)
+ *   out_idx, out_w  [B, n, hkv, sf] int32 / fp32, written in full
+ * Limits: d in {64, 128}; hq / hkv in {1, 2, 4}; q and k 16-byte aligned; B * n * hq < 2^31.
+ * The scores run on the tensor cores (bf16 products, fp32 sums), the masses in fp32: a
+ * position whose mass lies within fp32 rounding of the sf-th largest may be exchanged for
+ * another at the same mass.
+ * Errors: GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED as above; GM_ERR_CUDA if the tensor-map
+ * encoder of the driver is unavailable or the launch fails.
+ */
+gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, const float *lse,
+                                 int B, int n, int hq, int hkv, int d, float scale, int sf,
+                                 int32_t *out_idx, float *out_w, cudaStream_t stream);
+
+/*
  * gm_check_device_errors - synchronise `stream`, then read and clear this device's error
  * flag. Returns GM_ERR_INDEX_RANGE if any kernel of this library on the current device met
- * an active slot whose index lay outside [0, n) since the last check, GM_ERR_CUDA if the
- * synchronisation failed, else GM_OK.
+ * an active slot whose index lay outside [0, n) since the last check, GM_ERR_WAIT_TIMEOUT if a
+ * kernel gave up on a bounded wait for an asynchronous copy or tensor-core operation (its
+ * outputs are then incomplete), GM_ERR_CUDA if the synchronisation failed, else GM_OK.
  */
 gm_status gm_check_device_errors(cudaStream_t stream);
 

@@ -56,7 +56,8 @@ def _load():
         lib.oracle_ser_refresh_backward.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci,
                                                     f32p, ci, ci, ci, ci, ci, f64p, f64p, f64p]
         lib.oracle_dense_lse.restype = None
-        lib.oracle_dense_lse.argtypes = [f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double, f64p]
+        lib.oracle_dense_lse.argtypes = [f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double,
+                                         ctypes.c_void_p, ctypes.c_int64, f64p]
         lib.oracle_dense_mass.restype = None
         lib.oracle_dense_mass.argtypes = [f32p, f32p, f32p, ci, ci, ci, ci, ci, ctypes.c_double,
                                           ctypes.c_void_p, ctypes.c_int64, f64p]
@@ -307,15 +308,16 @@ def _rows(rows):
     return r, r.ctypes.data_as(ctypes.c_void_p), int(r.size)
 
 
-def dense_lse(q, k, scale: float | None = None):
-    """Normaliser of causal softmax attention per (b, i, hq), fp64 [B, n, hq]: the lse a dense
-    attention layer's forward returns."""
+def dense_lse(q, k, scale: float | None = None, rows=None):
+    """Normaliser of causal softmax attention per (b, i, hq), fp64 [B, n, hq] (or [nrows, hq]
+    for a list of flat rows b*n + i): the lse a dense attention layer's forward returns."""
     qf, kf = _np(q, np.float32), _np(k, np.float32)
     B, n, hq, d = qf.shape
     hkv = kf.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    out = np.zeros((B, n, hq), np.float64)
-    _load().oracle_dense_lse(qf, kf, B, n, hq, hkv, d, scale, out)
+    r, rp, nr = _rows(rows)
+    out = np.zeros((B, n, hq) if r is None else (nr, hq), np.float64)
+    _load().oracle_dense_lse(qf, kf, B, n, hq, hkv, d, scale, rp, nr, out)
     return out
 
 

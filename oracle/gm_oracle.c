@@ -783,14 +783,17 @@ static double dense_dot(const float *q, const float *kk, int64_t b, int i, int t
     return dot;
 }
 
-/* lse [B, n, hq]: log of sum over t <= i of exp(scale <q[b,i,hq], k[b,t,h]>), the normaliser
- * of causal softmax attention (R14). */
+/* lse [nrows, hq]: log of sum over t <= i of exp(scale <q[b,i,hq], k[b,t,h]>), the normaliser
+ * of causal softmax attention (R14), for the flat positions rows[r] = b*n + i (NULL: all B*n
+ * in order). */
 void oracle_dense_lse(const float *q, const float *kk, int B, int n, int hq, int hkv, int d,
-                      double scale, double *lse)
+                      double scale, const int64_t *rows, int64_t nrows, double *lse)
 {
     const int G = hq / hkv;
+    if (rows == NULL) nrows = (int64_t)B * n;
 #pragma omp parallel for schedule(dynamic, 4)
-    for (int64_t bi = 0; bi < (int64_t)B * n; ++bi) {
+    for (int64_t r = 0; r < nrows; ++r) {
+        const int64_t bi = rows ? rows[r] : r;
         const int64_t b = bi / n;
         const int i = (int)(bi % n);
         double *z = (double *)malloc(sizeof(double) * (size_t)(i + 1));
@@ -803,7 +806,7 @@ void oracle_dense_lse(const float *q, const float *kk, int B, int n, int hq, int
             }
             double l = 0.0;
             for (int t = 0; t <= i; ++t) l += exp(z[t] - m);
-            lse[bi * hq + hqi] = m + log(l);
+            lse[r * hq + hqi] = m + log(l);
         }
         free(z);
     }

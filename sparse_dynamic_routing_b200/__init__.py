@@ -14,6 +14,8 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_ser_sea_forward  both in one kernel
     gm_sea_backward     gradients of sparse edge attention
     gm_ser_backward     gradients of the kept referral weights
+    gm_dense_refresh_edges
+                        refresh edges from a dense attention layer (its top positions)
 """
 from ._binding import (  # noqa: F401
     GM_BF16,
@@ -22,6 +24,7 @@ from ._binding import (  # noqa: F401
     GMIndexRangeError,
     LIB_PATH,
     gm_check_device_errors,
+    gm_dense_refresh_edges,
     gm_leg_backward,
     gm_leg_sparsify,
     gm_sea_backward,

@@ -18,7 +18,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgm_b200.so")
 
 (GM_OK, GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED, GM_ERR_CUDA, GM_ERR_INDEX_RANGE,
- GM_ERR_SCRATCH_TOO_SMALL) = range(6)
+ GM_ERR_SCRATCH_TOO_SMALL, GM_ERR_WAIT_TIMEOUT) = range(7)
 GM_F32, GM_BF16 = 0, 1
 
 # Entry points of include/gm.h with their ctypes signatures.
@@ -52,6 +52,7 @@ SIGNATURES = {
     "gm_sea_backward_noalloc": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci,
                                 _cf, _vp, _vp, _vp, _vp, _ci, _vp],
     "gm_sea_backward_noalloc_max_scratch": [],
+    "gm_dense_refresh_edges": [_vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp, _vp, _vp],
     "gm_check_device_errors": [_vp],
     "gm_status_string": [_ci],
     "gm_version": [],
@@ -524,8 +525,32 @@ def gm_sea_backward_noalloc(q, k, v, dout, idx, w, scale=None, dq=None, dk=None,
     return dq, dk, dv, dlogw
 
 
+def gm_dense_refresh_edges(q, k, lse, sf: int, scale=None, out_idx=None, out_w=None, stream=None):
+    """Refresh edges from a dense attention layer: per (b, i, KV head) the sf positions t <= i of
+    largest attention mass (mean over the head's query group), weighted by that mass.
+    q [B, n, hq, d], k [B, n, hkv, d] bf16; lse [B, n, hq] fp32. Returns (idx, w) [B, n, hkv, sf]."""
+    B, n, hq, d = q.shape
+    hkv = k.shape[2]
+    if tuple(k.shape) != (B, n, hkv, d) or k.dtype != q.dtype:
+        raise ValueError("k must be [B, n, hkv, d] with q's dtype")
+    if tuple(lse.shape) != (B, n, hq):
+        raise ValueError("lse must be [B, n, hq]")
+    dev = q.device
+    if out_idx is None:
+        out_idx = torch.empty((B, n, hkv, sf), dtype=torch.int32, device=dev)
+    if out_w is None:
+        out_w = torch.empty((B, n, hkv, sf), dtype=torch.float32, device=dev)
+    st = load_library().gm_dense_refresh_edges(
+        _ptr(q, name="q"), _ptr(k, name="k"), _fdtype(q), _ptr(lse, torch.float32, "lse"),
+        B, n, hq, hkv, d, _scale(scale, d), sf, _ptr(out_idx, torch.int32, "out_idx"),
+        _ptr(out_w, torch.float32, "out_w"), _stream(stream))
+    _check(st, "gm_dense_refresh_edges")
+    return out_idx, out_w
+
+
 def gm_check_device_errors(stream=None):
-    """Synchronise the stream and raise GMIndexRangeError if a kernel met a bad index."""
+    """Synchronise the stream; raise GMIndexRangeError if a kernel met a bad index, GMError if a
+    kernel gave up on a bounded wait (GM_ERR_WAIT_TIMEOUT)."""
     _check(load_library().gm_check_device_errors(_stream(stream)), "gm_check_device_errors")
 
 

@@ -9,6 +9,7 @@
 #include "gm_bwd_gather.cuh"
 #include "gm_bwd_tile.cuh"
 #include "gm_common.cuh"
+#include "gm_dense_refresh.cuh"
 #include "gm_fused_tile.cuh"
 #include "gm_leg.cuh"
 #include "gm_leg_tile.cuh"
@@ -221,7 +222,10 @@ unsigned persistent_blocks(K kernel, int threads, size_t smem, int64_t rows, int
 // Passes of K/V copies in flight per warp in the forward tile kernel: two for budgets of 2
 // (little work per pass to cover the loads), one for budgets of 4 (a pass covers them, and
 // the freed shared memory admits more warps).
-template <int S1M> constexpr int tile_passes() { return S1M >= 4 ? 1 : 2; }
+#ifndef GM_TILE_P4
+#define GM_TILE_P4 1
+#endif
+template <int S1M> constexpr int tile_passes() { return S1M >= 4 ? GM_TILE_P4 : 2; }
 constexpr int WPB_TILE = GM_WPB_TILE;
 constexpr int TILE_CPL = GM_TILE_CPL;  // 16-byte chunks of a feature row per lane
 
@@ -414,6 +418,79 @@ template <typename T, int D, int G> struct SeaBwdGather {
     }
 };
 
+// ---- refresh edges from a dense attention layer ----------------------------------------------
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the library does not link
+// the driver library itself).
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// A bf16 feature tensor [rows, heads, d] as a 3-d TMA map whose boxes are 64 elements of d
+// (128 bytes, the swizzle width) x 1 head x box_rows rows, in the 128-byte swizzle layout.
+bool feature_tmap(CUtensorMap &m, const void *ptr, int64_t rows, int heads, int d, int box_rows)
+{
+    const EncodeTiledFn f = encode_tiled();
+    if (f == nullptr) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows};
+    const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)heads * d * 2};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return f(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G, int SFM>
+gm_status launch_dense_refresh(const void *q, const void *k, int64_t tokens, const gm::DenseRefreshArgs &a,
+                               cudaStream_t st)
+{
+    constexpr int BN = G == 4 ? 64 : 128;  // G accumulators x BN columns x 2 sets <= 512 TMEM columns
+    using Geo = gm::DenseGeom<D, G, BN>;
+    CUtensorMap tq, tk;
+    if (!feature_tmap(tq, q, tokens, a.hq, D, Geo::BM) || !feature_tmap(tk, k, tokens, a.hkv, D, BN))
+        return GM_ERR_CUDA;
+    auto kern = gm::dense_refresh_kernel<D, G, BN, SFM>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM_BYTES) != cudaSuccess)
+        return GM_ERR_CUDA;
+    kern<<<(unsigned)((int64_t)a.BH * a.nblk), 192, Geo::SMEM_BYTES, st>>>(tq, tk, a);
+    return launched();
+}
+
+template <int D, int G>
+gm_status dense_refresh_sf(const void *q, const void *k, int64_t tokens, const gm::DenseRefreshArgs &a,
+                           cudaStream_t st)
+{
+    if (a.sf <= 2) return launch_dense_refresh<D, G, 2>(q, k, tokens, a, st);
+    if (a.sf <= 4) return launch_dense_refresh<D, G, 4>(q, k, tokens, a, st);
+    return launch_dense_refresh<D, G, 8>(q, k, tokens, a, st);
+}
+
+template <int D>
+gm_status dense_refresh_g(const void *q, const void *k, int64_t tokens, int G, const gm::DenseRefreshArgs &a,
+                          cudaStream_t st)
+{
+    if (G == 1) return dense_refresh_sf<D, 1>(q, k, tokens, a, st);
+    if (G == 2) return dense_refresh_sf<D, 2>(q, k, tokens, a, st);
+    if (G == 4) return dense_refresh_sf<D, 4>(q, k, tokens, a, st);
+    return GM_ERR_UNSUPPORTED;
+}
+
 // ---- scratch for callers that cannot allocate ------------------------------------------------
 //
 // gm_sea_backward_noalloc runs the gather path of gm_sea_backward on this fixed, file-scope
@@ -461,6 +538,9 @@ const char *gm_status_string(gm_status status)
     case GM_ERR_SCRATCH_TOO_SMALL:
         return "GM_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than the library's fixed "
                "array holds (see gm_sea_backward_noalloc_max_scratch)";
+    case GM_ERR_WAIT_TIMEOUT:
+        return "GM_ERR_WAIT_TIMEOUT: a kernel gave up on a bounded wait for an asynchronous copy or "
+               "tensor-core operation; its outputs are incomplete";
     default: return "unknown gm_status";
     }
 }
@@ -858,6 +938,34 @@ gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, c
 
 size_t gm_sea_backward_noalloc_max_scratch(void) { return NOALLOC_SCRATCH_BYTES; }
 
+gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, const float *lse,
+                                 int B, int n, int hq, int hkv, int d, float scale, int sf,
+                                 int32_t *out_idx, float *out_w, cudaStream_t stream)
+{
+    if (B < 0 || n < 0 || hq < 1 || hkv < 1 || d < 1 || sf < 1 || sf > 8) return GM_ERR_INVALID_ARG;
+    if (hq % hkv != 0 || !std::isfinite(scale)) return GM_ERR_INVALID_ARG;
+    if (dtype != GM_F32 && dtype != GM_BF16) return GM_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (dtype != GM_BF16 || (d != 64 && d != 128) || (G != 1 && G != 2 && G != 4)) return GM_ERR_UNSUPPORTED;
+    if ((int64_t)B * n == 0) return GM_OK;
+    if ((int64_t)B * n * hq >= MAX_ROWS) return GM_ERR_UNSUPPORTED;
+    if (!q || !k || !lse || !out_idx || !out_w) return GM_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k)) return GM_ERR_INVALID_ARG;
+    gm::DenseRefreshArgs a{};
+    a.lse = lse;
+    a.out_idx = out_idx;
+    a.out_w = out_w;
+    a.n = n;
+    a.hq = hq;
+    a.hkv = hkv;
+    a.sf = sf;
+    a.nblk = (n + 127) / 128;
+    a.BH = B * hkv;
+    a.sl2 = scale * gm::LOG2E;
+    const int64_t tokens = (int64_t)B * n;
+    return d == 64 ? dense_refresh_g<64>(q, k, tokens, G, a, stream) : dense_refresh_g<128>(q, k, tokens, G, a, stream);
+}
+
 gm_status gm_check_device_errors(cudaStream_t stream)
 {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return GM_ERR_CUDA;
@@ -866,7 +974,7 @@ gm_status gm_check_device_errors(cudaStream_t stream)
     if (flag == 0) return GM_OK;
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(gm::g_error_flag, &zero, sizeof(zero)) != cudaSuccess) return GM_ERR_CUDA;
-    return GM_ERR_INDEX_RANGE;
+    return (flag & gm::ERR_WAIT_TIMEOUT) ? GM_ERR_WAIT_TIMEOUT : GM_ERR_INDEX_RANGE;
 }
 
 }  // extern "C"

@@ -35,8 +35,11 @@ constexpr float LN2 = 0.6931471805599453f;
 
 // Device error word of this library (one per device). Bit 0: an active slot indexed
 // outside [0, n). Kernels set it with atomicOr and carry on; the host reads and clears it.
+// Bit 1: a bounded wait on an asynchronous copy or tensor-core operation ran out of time (the
+// kernel gave up on its remaining work).
 __device__ unsigned int g_error_flag;
 constexpr unsigned ERR_INDEX_RANGE = 1u;
+constexpr unsigned ERR_WAIT_TIMEOUT = 2u;
 
 __device__ __forceinline__ void raise_index_error() { atomicOr(&g_error_flag, ERR_INDEX_RANGE); }
 
@@ -93,6 +96,14 @@ __device__ __forceinline__ float lg2(float x)
 {
     float y;
     asm("lg2.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Fast reciprocal (MUFU; relative error ~2^-23). Used only on softmax sums, which are >= 1.
+__device__ __forceinline__ float rcp_fast(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
 }
 
@@ -154,10 +165,81 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
     const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem) : "memory");
 }
+// The same copy with a source size of 0 or 16 bytes: 0 reads nothing and writes 16 zero bytes
+// (an inactive slot's stage then holds zeros, so it can be computed on like an active one).
+__device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, bool copy)
+{
+    const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(copy ? 16 : 0)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N> __device__ __forceinline__ void cp_async_wait()
 {
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+// ---- shared-memory barriers (mbarrier) with bounded waits --------------------------------
+//
+// Completion of asynchronous copies (TMA) and tensor-core operations is counted on 64-bit
+// shared-memory barriers. Every wait is bounded: after WAIT_LIMIT_NS without completion the
+// waiting thread sets ERR_WAIT_TIMEOUT and reports failure, so a lost completion cannot hang
+// the device.
+
+constexpr unsigned long long WAIT_LIMIT_NS = 1000000000ull;  // one second
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+// Makes barrier initialisation visible to the asynchronous proxy (copy engine, tensor cores).
+__device__ __forceinline__ void mbar_init_fence() { asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+{
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}\n" ::"r"(bar) : "memory");
+}
+// Announces `bytes` of incoming asynchronous copies and arrives once.
+__device__ __forceinline__ void mbar_arrive_expect(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n}\n" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns()
+{
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;\n" : "=l"(t));
+    return t;
+}
+
+// Waits for the completion of the barrier phase with the given parity. Returns false, with
+// ERR_WAIT_TIMEOUT set, if that takes longer than WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > WAIT_LIMIT_NS) {
+            atomicOr(&g_error_flag, ERR_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
 }
 
 // Dot product of a 16-byte chunk of q (as fp32 pairs) with a chunk of k: even and odd

@@ -79,6 +79,8 @@ def test_mass_is_group_mean_of_softmax(hq, hkv):
     rows = [5, 0, B * n - 1, 31]
     np.testing.assert_allclose(oracle.dense_mass(q, k, lse, scale, rows=rows), got[rows], rtol=0,
                                atol=0)
+    np.testing.assert_allclose(oracle.dense_lse(q, k, scale, rows=rows),
+                               oracle.dense_lse(q, k, scale).reshape(B * n, hq)[rows], rtol=0, atol=0)
 
 
 @pytest.mark.parametrize("sf", [1, 2, 4, 8])
