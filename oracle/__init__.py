@@ -31,6 +31,8 @@ def _load():
         f64p = np.ctypeslib.ndpointer(np.float64, flags="C_CONTIGUOUS")
         ci = ctypes.c_int
         lib.oracle_num_threads.restype = ci
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [ci]
         lib.oracle_ser.restype = ctypes.c_int64
         lib.oracle_ser.argtypes = [i32p, f32p, ci, i32p, f32p, ci, i32p, f32p, ci, ci, ci, ci]
         lib.oracle_ser_backward.restype = ctypes.c_int64
@@ -71,6 +73,11 @@ def _load():
 def num_threads() -> int:
     """Threads the oracle's parallel loops use (OMP_NUM_THREADS or all cores)."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's parallel loops from now on."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def _np(x, dtype):

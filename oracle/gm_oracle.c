@@ -100,6 +100,17 @@ int oracle_num_threads(void)
 #endif
 }
 
+/* Threads of the parallel loops from now on (the benchmark times the oracle on one core and on
+ * all of them). */
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    omp_set_num_threads(n > 0 ? n : 1);
+#else
+    (void)n;
+#endif
+}
+
 /* ------------------------------------------------------------------------------------------
  * SER: A' = Sparsify_s1(A1 A2)   [KC3], [MPE2]; readings R1-R5, R8.
  *

@@ -404,7 +404,7 @@ template <typename T, int D, int G> struct SeaBwdGather {
             const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
             if (rs != GM_OK) return rs;
             auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
-            const size_t smem = (size_t)WPB_GATHER * GATHER_P * GATHER_U * G * 32 * 16;
+            const size_t smem = (size_t)WPB_GATHER * gm::gather_warp_bytes<G>(GATHER_U, GATHER_P);
             if (smem > 48 * 1024 &&
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return GM_ERR_CUDA;
@@ -468,7 +468,7 @@ gm_status launch_dense_refresh(const void *q, const void *k, int64_t tokens, con
     auto kern = gm::dense_refresh_kernel<D, G, BN, SFM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM_BYTES) != cudaSuccess)
         return GM_ERR_CUDA;
-    kern<<<(unsigned)((int64_t)a.BH * a.nblk), 192, Geo::SMEM_BYTES, st>>>(tq, tk, a);
+    kern<<<(unsigned)((int64_t)a.BH * a.nblk), 320, Geo::SMEM_BYTES, st>>>(tq, tk, a);
     return launched();
 }
 

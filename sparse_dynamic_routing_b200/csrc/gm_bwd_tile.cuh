@@ -38,10 +38,10 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
 };
 
 // Resident blocks per SM the tile kernel is compiled for: caps registers at 65536 / (32 * WPB *
-// MINB). The gather row pass fits 102 registers (five blocks; ptxas spills 8 bytes); the
-// atomic row pass needs more and keeps four.
+// MINB). Four blocks (128 registers, no spills) measured faster than five (96 registers with
+// spills) for the gather row pass; the atomic row pass keeps four too.
 #ifndef GM_BWD_TILE_MINB
-#define GM_BWD_TILE_MINB 5
+#define GM_BWD_TILE_MINB 4
 #endif
 
 template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER>
@@ -62,6 +62,9 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
     const uint32_t W = gridDim.x * WPB;
     const int rr = lane / C, c = lane % C;
     const float sl2 = a.scale * LOG2E;
+    // this lane's chunk of K/V row 0: a gathered row's chunk is one wide multiply-add away
+    const char *kbase = static_cast<const char *>(a.k) + (size_t)c * 16;
+    const char *vbase = static_cast<const char *>(a.v) + (size_t)c * 16;
 
     for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
         const uint32_t r0 = tile * 32;
@@ -81,7 +84,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                     const float w = __ldg(a.w + (size_t)row * a.s + r);
                     const int32_t ti = __ldg(a.idx + (size_t)row * a.s + r);
                     if (w > 0.0f) {
-                        if (ti < 0 || ti >= a.n) {
+                        if ((uint32_t)ti >= (uint32_t)a.n) {
                             raise_index_error();
                         } else {
                             t = ti;
@@ -101,16 +104,18 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 const int lr = pass * RPW + rr;
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
-                if (row < rows) {
+                // every slot is copied; an inactive one (or a row past the end) reads nothing
+                // and gets zeros, so no branch and no stale data
+                float lwv[S1M];
+                int32_t tv[S1M];
+                ld_tile<S1M>(tile_lw + lr * S1M, lwv);
+                ld_tile<S1M>(tile_t + lr * S1M, tv);
 #pragma unroll
-                    for (int jj = 0; jj < S1M; ++jj) {
-                        if (tile_lw[lr * S1M + jj] != -INFINITY) {
-                            const uint32_t kvrow = (uint32_t)tile_t[lr * S1M + jj];
-                            const size_t off = (size_t)kvrow * TG::ROW + c * 16;
-                            cp_async16(st + TG::RK + jj * TG::ROW + c * 16, static_cast<const char *>(a.k) + off);
-                            cp_async16(st + TG::RV + jj * TG::ROW + c * 16, static_cast<const char *>(a.v) + off);
-                        }
-                    }
+                for (int jj = 0; jj < S1M; ++jj) {
+                    const bool live = row < rows && lwv[jj] != -INFINITY;
+                    const size_t off = (size_t)(live ? (uint32_t)tv[jj] : 0u) * TG::ROW;
+                    cp_async16_zfill(st + TG::RK + jj * TG::ROW + c * 16, kbase + off, live);
+                    cp_async16_zfill(st + TG::RV + jj * TG::ROW + c * 16, vbase + off, live);
                 }
             }
             cp_async_commit();
@@ -148,11 +153,9 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
 
             float lw[S1M];
             bool act[S1M];
+            ld_tile<S1M>(tile_lw + lr * S1M, lw);
 #pragma unroll
-            for (int jj = 0; jj < S1M; ++jj) {
-                lw[jj] = tile_lw[lr * S1M + jj];
-                act[jj] = valid && lw[jj] != -INFINITY;
-            }
+            for (int jj = 0; jj < S1M; ++jj) act[jj] = valid && lw[jj] != -INFINITY;
             float2 q2[G][NP], g2[G][NP];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj) {
                     float kf[VEC], vf[VEC];
-                    // an inactive slot's stage holds stale data: its values are masked below
+                    // an inactive slot's stage holds zeros: its values are masked below
                     unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
                     unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
 #pragma unroll
@@ -217,7 +220,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                     l += __shfl_xor_sync(FULL, l, off);
                     sdp += __shfl_xor_sync(FULL, sdp, off);
                 }
-                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                const float inv = l > 0.0f ? rcp_fast(l) : 0.0f;  // l >= 1: its largest term is 1
                 const float pj = e * inv;
                 const float dzj = pj * ((myact ? dpv : 0.0f) - sdp * inv);
                 const int seg = lane & ~(C - 1);
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
                 float kf[VEC], vf[VEC];
-                // an inactive slot's stage holds stale data: its score and dO.V are masked below
+                // an inactive slot's stage holds zeros: its score and dO.V are masked below
                 unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
                 unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RV + jj * TG::ROW + c * 16), vf);
 #pragma unroll
@@ -268,7 +271,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                     l += p[g][jj];
                     sdp = fmaf(p[g][jj], dp[g][jj], sdp);
                 }
-                const float inv = l > 0.0f ? __frcp_rn(l) : 0.0f;
+                const float inv = l > 0.0f ? rcp_fast(l) : 0.0f;
                 const float Dd = sdp * inv;
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj) {
@@ -285,7 +288,9 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 for (int x = 0; x < NP; ++x) dq2[g][x] = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int jj = 0; jj < S1M; ++jj) {
-                if (!act[jj]) continue;  // per lane; no shuffles below
+                // zero-filled stages: an inactive slot has dz = p = 0 and K = 0 (no branch); the
+                // atomic path still skips its scatter
+                if (!GATHER && !act[jj]) continue;  // per lane; no shuffles below
                 float kf[VEC];
                 unpack<T>(*reinterpret_cast<const uint4 *>(st + TG::RK + jj * TG::ROW + c * 16), kf);
                 float2 pk[NP], pv[NP];

@@ -13,17 +13,19 @@
 // prefix run on the tensor cores: tcgen05.mma with bf16 operands staged by TMA in the
 // 128-byte swizzle layout and fp32 accumulators in tensor memory (TMEM), two key stages and
 // two accumulator sets, so the MMAs of key block j + 1 overlap the selection over block j.
-// Warp roles: warps 0-3 select (thread = query row = TMEM lane), warp 4 loads (TMA), warp 5
-// issues the MMAs. Every wait is bounded (gm_common.cuh, mbar_wait).
+// Warp roles: warps 0-7 select (two threads per query row = TMEM lane, each taking every other
+// 32-column chunk of a key block), warp 8 loads (TMA), warp 9 issues the MMAs. Every wait is
+// bounded (gm_common.cuh, mbar_wait).
 //
-// Selection per row, streaming over ascending t: a sorted register list of the SFM heaviest
+// Selection per thread, streaming over ascending t: a sorted register list of the SFM heaviest
 // (mass, t) so far (SFM = sf rounded up to 2, 4 or 8; the first sf of the top SFM are the top
 // sf). With x_g = scale log2(e) S_g - log2(e) lse_g the mass is mean_g 2^x_g <= 2^max_g x_g, so
-// a position whose max_g x_g lies below log2 of the list's smallest mass cannot enter: it
-// costs G FMAs, a max and a compare. The others (the first SFM, then few) get their mass
-// computed (G exponentials) and are appended to a per-thread shared-memory list; after each
-// 32-column chunk every lane merges its list into the register list, so the lanes of a warp
-// insert in lockstep instead of one divergent branch per column.
+// a position whose max_g x_g lies below log2 of the list's smallest mass cannot enter. The scan
+// is branch-free: per column G FMAs, a max, a compare that sets a bit of a candidate mask, and
+// a store of the x_g to a per-thread shared-memory slot; then each lane walks its own mask
+// (computing the few candidates' masses with G exponentials and inserting those that beat the
+// list), so the lanes of a warp never diverge per column. At the end the two threads of a row
+// merge their lists.
 #pragma once
 
 #include <cuda.h>
@@ -51,10 +53,11 @@ template <int D, int G, int BN> struct DenseGeom {
     static constexpr int K_ATOM = BN * 128;
     static constexpr int QBYTES = G * NA * Q_ATOM;
     static constexpr int KBYTES = NST * NA * K_ATOM;
-    static constexpr int LIST = 32;                 // per-thread candidate list (one chunk)
+    static constexpr int NSEL = 2 * BM;             // selection threads (two per row)
+    static constexpr int SUB = G == 4 ? 8 : 16;     // columns scanned per candidate mask
     static constexpr int OFF_K = QBYTES;
-    static constexpr int OFF_LIST = QBYTES + KBYTES;
-    static constexpr int OFF_BAR = OFF_LIST + LIST * BM * 8;
+    static constexpr int OFF_LIST = QBYTES + KBYTES;  // x values [SUB][NSEL][G]
+    static constexpr int OFF_BAR = OFF_LIST + SUB * NSEL * G * 4;
     static constexpr int NBAR = 2 + 2 * NST + 2 * NACC;  // q_full, k_full/empty, acc_full/empty, mma_done
     static constexpr int TMEM_COLS = NACC * G * BN;
     // + TMEM slot and 1 KB of alignment; a CTA that takes more than half of the 512 TMEM columns
@@ -83,6 +86,13 @@ template <int SFM> __device__ __forceinline__ void list_insert(float (&kw)[SFM],
     }
 }
 
+// Barrier over the first `count` threads of the CTA (the selection warps), id 1 (id 0 is the
+// CTA-wide __syncthreads).
+__device__ __forceinline__ void named_barrier_sync(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(count) : "memory");
+}
+
 // log2 of the list's smallest mass less a margin larger than lg2.approx's error (so the skip
 // test never drops a position that could enter), or -inf while the list has room.
 template <int SFM> __device__ __forceinline__ float skip_bound(const float (&kw)[SFM])
@@ -91,7 +101,7 @@ template <int SFM> __device__ __forceinline__ float skip_bound(const float (&kw)
 }
 
 template <int D, int G, int BN, int SFM>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      DenseRefreshArgs a)
 {
@@ -107,7 +117,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     const uint32_t acc_full = k_empty + 8 * NST, acc_empty = acc_full + 8 * NACC;
     const uint32_t mma_done = acc_empty + 8 * NACC, tslot = mma_done + 8;
     const uint32_t *tslot_p = reinterpret_cast<const uint32_t *>(sm + Geo::OFF_BAR + Geo::NBAR * 8);
-    float2 *list = reinterpret_cast<float2 *>(sm + Geo::OFF_LIST);  // [LIST][BM] (mass, t bits)
+    float *listx = reinterpret_cast<float *>(sm + Geo::OFF_LIST);  // [SUB][NSEL][G] x values
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ib = a.nblk - 1 - (int)(blockIdx.x / (unsigned)a.BH);  // longest prefixes first
@@ -128,7 +138,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
 #pragma unroll
         for (int s = 0; s < NACC; ++s) {
             mbar_init(acc_full + 8 * s, 1);
-            mbar_init(acc_empty + 8 * s, Geo::BM);
+            mbar_init(acc_empty + 8 * s, Geo::NSEL);
         }
         mbar_init(mma_done, 1);
         mbar_init_fence();
@@ -139,7 +149,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     umma::fence_after_sync();
     const uint32_t tmem = *tslot_p;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ---- loads: the query tile once, then the key blocks through NST stages ----------
         if (lane == 0) {
             mbar_arrive_expect(q_full, Geo::QBYTES);
@@ -163,7 +173,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
                 for (int j = max(0, issued - NST); j < issued; ++j) mbar_wait(k_full + 8 * (j % NST), (j / NST) & 1);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ---- MMAs: S_g = Q_g K^T into accumulator set j % NACC ------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc = umma::idesc_bf16_f32(Geo::BM, BN);
@@ -191,8 +201,11 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
             mbar_wait(mma_done, 0);
         }
     } else {
-        // ---- selection: thread = query row i = TMEM lane -----------------------------------
-        const int r = warp * 32 + lane;
+        // ---- selection: two threads per query row i = TMEM lane (warp w reads lane quarter
+        // w % 4), the thread of half w / 4 scanning the chunks cc with cc % 2 == w / 4 ---------
+        const int quarter = warp & 3, half = warp >> 2;
+        const int r = quarter * 32 + lane;
+        const int tid = threadIdx.x;  // 0 .. NSEL-1
         const int i = i0 + r;
         const bool valid = i < a.n;
         float nl[G];  // -log2(e) * lse of the row's query heads
@@ -208,62 +221,92 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
         }
         float L = -INFINITY;
         const float sl2 = a.sl2;
-        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
+        float *myx = listx + tid * G;  // slot c of this thread at myx[c * NSEL * G]
+        bool ok = true;
         for (int j = 0; j < nt; ++j) {
             const int as = j % NACC;
-            if (!__all_sync(FULL, mbar_wait(acc_full + 8 * as, (j / NACC) & 1))) break;
+            ok = __all_sync(FULL, mbar_wait(acc_full + 8 * as, (j / NACC) & 1));
+            if (!ok) break;
             umma::fence_after_sync();
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
+            for (int cc = half; cc < BN / 32; cc += 2) {
                 uint32_t sv[G][32];
 #pragma unroll
                 for (int g = 0; g < G; ++g) umma::tmem_ld32(tlane + (as * G + g) * BN + cc * 32, sv[g]);
                 umma::tmem_wait_ld();
-                const int t0 = j * BN + cc * 32;
-                const int lim = valid ? i - t0 : -1;  // column c is causal for this row iff c <= lim
-                int cnt = 0;
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    float x[G];
-                    float mx = -INFINITY;
+                for (int sub = 0; sub < 32; sub += Geo::SUB) {
+                    const int t0 = j * BN + cc * 32 + sub;
+                    // columns c < SUB of this piece that are causal for the row: c <= i - t0
+                    const int lim = valid ? i - t0 : -1;
+                    const uint32_t causal = lim >= Geo::SUB - 1 ? (1u << Geo::SUB) - 1u
+                                                                : (lim < 0 ? 0u : (2u << lim) - 1u);
+                    uint32_t mask = 0;
 #pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        x[g] = fmaf(__uint_as_float(sv[g][c]), sl2, nl[g]);
-                        mx = fmaxf(mx, x[g]);
+                    for (int c = 0; c < Geo::SUB; ++c) {
+                        float mx = -INFINITY;
+#pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            const float x = fmaf(__uint_as_float(sv[g][sub + c]), sl2, nl[g]);
+                            myx[c * Geo::NSEL * G + g] = x;
+                            mx = fmaxf(mx, x);
+                        }
+                        mask |= (mx > L ? 1u : 0u) << c;
                     }
-                    if (mx > L && c <= lim) {
+                    mask &= causal;
+                    // each lane walks its own candidates (ascending t); the warp loops as long
+                    // as its busiest lane
+                    while (mask) {
+                        const int c = __ffs(mask) - 1;
+                        mask &= mask - 1;
                         float sum = 0.0f;
 #pragma unroll
-                        for (int g = 0; g < G; ++g) sum += ex2(x[g]);
-                        list[cnt * Geo::BM + r] = make_float2(sum * (1.0f / G), __int_as_float(t0 + c));
-                        ++cnt;
+                        for (int g = 0; g < G; ++g) sum += ex2(myx[c * Geo::NSEL * G + g]);
+                        const float m = sum * (1.0f / G);
+                        if (m > kw[SFM - 1]) list_insert<SFM>(kw, kt, m, t0 + c);
                     }
+                    L = skip_bound<SFM>(kw);
                 }
-                // merge this chunk's candidates (ascending t) into the register list
-                for (int e = 0; e < cnt; ++e) {
-                    const float2 v = list[e * Geo::BM + r];
-                    if (v.x > kw[SFM - 1]) list_insert<SFM>(kw, kt, v.x, __float_as_int(v.y));
-                }
-                L = skip_bound<SFM>(kw);
             }
             umma::fence_before_sync();
             mbar_arrive(acc_empty + 8 * as);
         }
-        if (valid) {
-            const size_t o = ((size_t)(row0 + i) * a.hkv + h) * a.sf;
-            for (int f = 0; f < a.sf; ++f) {
-                // f < sf <= SFM; select by unrolled compare so the list stays in registers
-                float w = 0.0f;
-                int t = 0;
+        // the two threads of a row merge their lists: the second half hands its list over in
+        // shared memory (the x-value slots, free now), the first inserts it and writes the row
+        float *hand = listx;  // [BM][SFM] masses, then [BM][SFM] positions
+        named_barrier_sync(1, Geo::NSEL);  // every scan is done with the slots
+        if (half == 1) {
 #pragma unroll
-                for (int x = 0; x < SFM; ++x)
-                    if (x == f) {
-                        w = kw[x];
-                        t = kt[x];
-                    }
-                const bool kept = w >= 0.0f;
-                a.out_idx[o + f] = kept ? t : 0;
-                a.out_w[o + f] = kept ? w : 0.0f;
+            for (int x = 0; x < SFM; ++x) {
+                hand[r * SFM + x] = kw[x];
+                hand[Geo::BM * SFM + r * SFM + x] = __int_as_float(kt[x]);
+            }
+        }
+        named_barrier_sync(1, Geo::NSEL);
+        if (half == 0 && ok) {
+#pragma unroll
+            for (int x = 0; x < SFM; ++x) {
+                const float m = hand[r * SFM + x];
+                if (m > kw[SFM - 1] || (m == kw[SFM - 1] && m >= 0.0f))
+                    list_insert<SFM>(kw, kt, m, __float_as_int(hand[Geo::BM * SFM + r * SFM + x]));
+            }
+            if (valid) {
+                const size_t o = ((size_t)(row0 + i) * a.hkv + h) * a.sf;
+                for (int f = 0; f < a.sf; ++f) {
+                    // f < sf <= SFM; select by unrolled compare so the list stays in registers
+                    float w = 0.0f;
+                    int t = 0;
+#pragma unroll
+                    for (int x = 0; x < SFM; ++x)
+                        if (x == f) {
+                            w = kw[x];
+                            t = kt[x];
+                        }
+                    const bool kept = w >= 0.0f;
+                    a.out_idx[o + f] = kept ? t : 0;
+                    a.out_w[o + f] = kept ? w : 0.0f;
+                }
             }
         }
     }
