@@ -30,8 +30,8 @@
  * Edge semantics. A slot (index, weight) is active iff weight > 0. Inactive slots are never
  * dereferenced. An active slot whose index lies outside [0, n) is treated as inactive and
  * raises the device error flag (see gm_check_device_errors); kernels never trap. Weights are
- * expected finite and >= 0; indices are expected causal (<= the row's own position) but
- * this is not checked. Position 0 of each sequence is the padding token: SER pads missing
+ * expected finite and >= 0; indices are expected causal (<= the row's own position); the
+ * regular build does not check this, the checked build does (gm_checked_build). Position 0 of each sequence is the padding token: SER pads missing
  * output slots with (index 0, weight 0.0f).
  *
  * Ownership and synchrony. The caller allocates and owns every buffer. Entry points allocate
@@ -43,7 +43,8 @@
  *                       misaligned feature pointer (16 bytes required), s out of [1, 32];
  *   GM_ERR_UNSUPPORTED  a valid shape the library has no kernel for (see each function);
  *   GM_ERR_CUDA         the launch failed (cudaGetLastError after the launch);
- *   GM_ERR_INDEX_RANGE  returned by gm_check_device_errors only.
+ *   GM_ERR_INDEX_RANGE, GM_ERR_EDGE_INVALID, GM_ERR_WAIT_TIMEOUT
+ *                       returned by gm_check_device_errors only.
  * B == 0 or n == 0 is an empty problem: GM_OK, nothing launched.
  */
 #ifndef GM_H
@@ -66,7 +67,8 @@ typedef enum gm_status {
     GM_ERR_CUDA = 3,
     GM_ERR_INDEX_RANGE = 4,
     GM_ERR_SCRATCH_TOO_SMALL = 5, /* gm_sea_backward_noalloc only */
-    GM_ERR_WAIT_TIMEOUT = 6       /* from gm_check_device_errors: a kernel gave up on a wait */
+    GM_ERR_WAIT_TIMEOUT = 6,      /* from gm_check_device_errors: a kernel gave up on a wait */
+    GM_ERR_EDGE_INVALID = 7       /* from gm_check_device_errors, checked builds only */
 } gm_status;
 
 /* Element type of q, k, v, o and dout. */
@@ -470,7 +472,9 @@ gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, c
 /*
  * gm_check_device_errors - synchronise `stream`, then read and clear this device's error
  * flag. Returns GM_ERR_INDEX_RANGE if any kernel of this library on the current device met
- * an active slot whose index lay outside [0, n) since the last check, GM_ERR_WAIT_TIMEOUT if a
+ * an active slot whose index lay outside [0, n) since the last check, GM_ERR_EDGE_INVALID if
+ * (checked build) an input edge broke the edge invariants (see gm_checked_build),
+ * GM_ERR_WAIT_TIMEOUT if a
  * kernel gave up on a bounded wait for an asynchronous copy or tensor-core operation (its
  * outputs are then incomplete), GM_ERR_CUDA if the synchronisation failed, else GM_OK.
  */
@@ -481,6 +485,17 @@ const char *gm_status_string(gm_status status);
 
 /* Library ABI version (major * 10000 + minor * 100 + patch). */
 int gm_version(void);
+
+/*
+ * gm_checked_build - 1 for the checked build of this library (libgm_b200_checked.so), 0 for
+ * the regular one. The checked build runs every entry point exactly as the regular build does,
+ * after verifying each edge tensor the call reads (first and second legs, refresh edges, chain
+ * legs, stored edges, SEA edges): every weight finite and >= 0, every active index (weight > 0,
+ * index >= 0) no later than its own row's position i (edges are causal; position 0 is the
+ * padding token). A violation is reported by gm_check_device_errors as GM_ERR_EDGE_INVALID.
+ * The checks cost one extra pass over each edge tensor.
+ */
+int gm_checked_build(void);
 
 #ifdef __cplusplus
 }

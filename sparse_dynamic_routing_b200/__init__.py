@@ -20,8 +20,10 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
 from ._binding import (  # noqa: F401
     GM_BF16,
     GM_F32,
+    GMEdgeInvalidError,
     GMError,
     GMIndexRangeError,
+    CHECKED_LIB_PATH,
     LIB_PATH,
     gm_check_device_errors,
     gm_dense_refresh_edges,

@@ -16,9 +16,10 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgm_b200.so")
+CHECKED_LIB_PATH = os.path.join(_HERE, "libgm_b200_checked.so")  # verifies input edges
 
 (GM_OK, GM_ERR_INVALID_ARG, GM_ERR_UNSUPPORTED, GM_ERR_CUDA, GM_ERR_INDEX_RANGE,
- GM_ERR_SCRATCH_TOO_SMALL, GM_ERR_WAIT_TIMEOUT) = range(7)
+ GM_ERR_SCRATCH_TOO_SMALL, GM_ERR_WAIT_TIMEOUT, GM_ERR_EDGE_INVALID) = range(8)
 GM_F32, GM_BF16 = 0, 1
 
 # Entry points of include/gm.h with their ctypes signatures.
@@ -56,6 +57,7 @@ SIGNATURES = {
     "gm_check_device_errors": [_vp],
     "gm_status_string": [_ci],
     "gm_version": [],
+    "gm_checked_build": [],
 }
 
 
@@ -71,24 +73,36 @@ class GMIndexRangeError(GMError):
     """A kernel met an active edge slot whose index was outside [0, n)."""
 
 
+class GMEdgeInvalidError(GMError):
+    """(Checked build) an input edge had a bad weight or a non-causal index."""
+
+
 _lib = None
 
 
+def open_library(path: str) -> ctypes.CDLL:
+    """A library built from csrc/ (regular or checked) with the ctypes signatures set."""
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m sparse_dynamic_routing_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, args in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = {"gm_status_string": ctypes.c_char_p,
+                      "gm_sea_backward_workspace_size": ctypes.c_size_t,
+                      "gm_sea_backward_noalloc_max_scratch": ctypes.c_size_t}.get(name, ctypes.c_int)
+    return lib
+
+
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
-    """Load libgm_b200.so (once). Raises if it has not been built."""
+    """Load the library the wrappers below call (once; libgm_b200.so unless the environment
+    variable GM_CHECKED=1 selects the checked build). Raises if it has not been built."""
     global _lib
     if _lib is None:
-        if not os.path.exists(path):
-            raise RuntimeError(
-                f"{path} is missing: build it with `python -m sparse_dynamic_routing_b200.build`")
-        lib = ctypes.CDLL(path)
-        for name, args in SIGNATURES.items():
-            fn = getattr(lib, name)
-            fn.argtypes = args
-            fn.restype = {"gm_status_string": ctypes.c_char_p,
-                          "gm_sea_backward_workspace_size": ctypes.c_size_t,
-                          "gm_sea_backward_noalloc_max_scratch": ctypes.c_size_t}.get(name, ctypes.c_int)
-        _lib = lib
+        if path == LIB_PATH and os.environ.get("GM_CHECKED") == "1":
+            path = CHECKED_LIB_PATH
+        _lib = open_library(path)
     return _lib
 
 
@@ -98,7 +112,7 @@ def status_string(status: int) -> str:
 
 def _check(status: int, what: str):
     if status != GM_OK:
-        cls = GMIndexRangeError if status == GM_ERR_INDEX_RANGE else GMError
+        cls = {GM_ERR_INDEX_RANGE: GMIndexRangeError, GM_ERR_EDGE_INVALID: GMEdgeInvalidError}.get(status, GMError)
         raise cls(status, f"{what}: {status_string(status)}")
 
 

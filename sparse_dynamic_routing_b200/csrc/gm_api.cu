@@ -161,6 +161,52 @@ gm_status check_sea(const void *q, const void *k, const void *v, gm_dtype dtype,
     return GM_OK;
 }
 
+// ---- checked builds ----------------------------------------------------------------------------
+//
+// Built with GM_CHECKED=1 (libgm_b200_checked.so), every entry point first verifies each edge
+// tensor it reads: weights finite and >= 0, and every active index causal (no later than the
+// position of its own row; position 0 is the padding token). A violation sets ERR_EDGE_INVALID
+// in the device error word (gm_check_device_errors then returns GM_ERR_EDGE_INVALID); the call
+// itself runs as in the regular build. In the regular build the check compiles to nothing.
+#ifndef GM_CHECKED
+#define GM_CHECKED 0
+#endif
+
+__global__ void check_edges_kernel(const int32_t *idx, const float *w, int64_t E, gm::FastDiv sdiv, gm::RowMap map)
+{
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < E; e += (int64_t)gridDim.x * blockDim.x) {
+        const float we = w[e];
+        const int32_t t = idx[e];
+        const uint32_t row = sdiv.div((uint32_t)e);
+        const uint32_t bi = map.heads.div(row);
+        const uint32_t pos = bi - map.n.div(bi) * map.n.d;
+        const bool bad_w = !(we >= 0.0f) || isinf(we);
+        const bool noncausal = we > 0.0f && t >= 0 && (uint32_t)t > pos;
+        if (bad_w || noncausal) atomicOr(&gm::g_error_flag, gm::ERR_EDGE_INVALID);
+    }
+}
+
+// Edge tensor [B, n, k, s] (nothing in a regular build).
+void check_edges(const int32_t *idx, const float *w, int s, int64_t B, int n, int k, cudaStream_t st)
+{
+    if (!GM_CHECKED || idx == nullptr || w == nullptr) return;
+    const int64_t E = B * n * k * s;
+    if (E == 0) return;
+    const int64_t want = (E + 255) / 256;
+    check_edges_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
+        idx, w, E, gm::FastDiv((uint32_t)s), row_map(k, n));
+}
+
+// The first leg and every leg of a referral chain (arguments filled by chain_args).
+void check_chain_edges(const SerArgs &a, cudaStream_t st)
+{
+    if (!GM_CHECKED) return;
+    const int64_t B = (int64_t)a.rows / ((int64_t)a.n * a.k);
+    check_edges(a.a1_idx, a.a1_w, a.s2, B, a.n, a.k, st);
+    check_edges(a.a2_idx, a.a2_w, a.s3, B, a.n, a.k, st);
+    for (int m = 0; m < a.nchain; ++m) check_edges(a.chain_idx[m], a.chain_w[m], a.s3, B, a.n, a.k, st);
+}
+
 // ---- dispatch over (dtype, d, G) ----------------------------------------------------------
 
 template <template <typename, int, int> class F, typename... Args>
@@ -527,6 +573,8 @@ extern "C" {
 
 int gm_version(void) { return 100; }
 
+int gm_checked_build(void) { return GM_CHECKED ? 1 : 0; }
+
 const char *gm_status_string(gm_status status)
 {
     switch (status) {
@@ -538,6 +586,9 @@ const char *gm_status_string(gm_status status)
     case GM_ERR_SCRATCH_TOO_SMALL:
         return "GM_ERR_SCRATCH_TOO_SMALL: the problem needs more scratch than the library's fixed "
                "array holds (see gm_sea_backward_noalloc_max_scratch)";
+    case GM_ERR_EDGE_INVALID:
+        return "GM_ERR_EDGE_INVALID: (checked build) an input edge had a negative or non-finite "
+               "weight, or an active index beyond its own row's position";
     case GM_ERR_WAIT_TIMEOUT:
         return "GM_ERR_WAIT_TIMEOUT: a kernel gave up on a bounded wait for an asynchronous copy or "
                "tensor-core operation; its outputs are incomplete";
@@ -555,6 +606,8 @@ gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
     SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k,
               (uint32_t)((int64_t)B * n * k), row_map(k, n)};
+    check_edges(a1_idx, a1_w, s2, B, n, k, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, k, stream);
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
     return launched();
 }
@@ -570,6 +623,8 @@ gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!gout || !dw1 || !dw2) return GM_ERR_INVALID_ARG;
     const int64_t rows = (int64_t)B * n * k;
+    check_edges(a1_idx, a1_w, s2, B, n, k, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, k, stream);
     if (!accumulate) {
         gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dw2), rows * s3);
         if (launched() != GM_OK) return GM_ERR_CUDA;
@@ -602,6 +657,7 @@ gm_status gm_leg_sparsify(const int32_t *e_idx, const float *e_w, int s0,
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!a1_idx || !a1_w || !a2_idx || !a2_w) return GM_ERR_INVALID_ARG;
     gm::LegArgs a{};
+    check_edges(e_idx, e_w, s0, B, n, k, stream);
     a.e_idx = e_idx;
     a.e_w = e_w;
     a.mix1 = mix1;
@@ -634,6 +690,7 @@ gm_status gm_leg_backward(const int32_t *e_idx, const float *e_w, int s0,
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!g1 || !g2 || !dew || !dmix1 || !dmix2) return GM_ERR_INVALID_ARG;
     gm::LegArgs a{};
+    check_edges(e_idx, e_w, s0, B, n, k, stream);
     a.e_idx = e_idx;
     a.e_w = e_w;
     a.mix1 = mix1;
@@ -670,6 +727,9 @@ gm_status gm_ser_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s
     if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
     SerArgs a{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, k,
               (uint32_t)((int64_t)B * n * k), row_map(k, n), f_idx, f_w, sf};
+    check_edges(a1_idx, a1_w, s2, B, n, k, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, k, stream);
+    check_edges(f_idx, f_w, sf, B, n, k, stream);
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
     return launched();
 }
@@ -688,6 +748,9 @@ gm_status gm_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int 
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!gout || !dw1 || !dw2 || !dfw) return GM_ERR_INVALID_ARG;
     const int64_t rows = (int64_t)B * n * k;
+    check_edges(a1_idx, a1_w, s2, B, n, k, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, k, stream);
+    check_edges(f_idx, f_w, sf, B, n, k, stream);
     if (!accumulate) {
         gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dw2), rows * s3);
         if (launched() != GM_OK) return GM_ERR_CUDA;
@@ -730,6 +793,9 @@ gm_status gm_ser_sea_refresh_forward(const int32_t *a1_idx, const float *a1_w, i
     st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    check_edges(a1_idx, a1_w, s2, B, n, hkv, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, hkv, stream);
+    check_edges(f_idx, f_w, sf, B, n, hkv, stream);
     const uint32_t rows = (uint32_t)((int64_t)B * n * hkv);
     SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows, row_map(hkv, n),
                f_idx, f_w, sf};
@@ -747,6 +813,7 @@ gm_status gm_ser_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!out_idx || !out_w) return GM_ERR_INVALID_ARG;
     a.out_idx = out_idx;
+    check_chain_edges(a, stream);
     a.out_w = out_w;
     const unsigned grid = blocks_for(a.rows, WPB_SER);
     switch (nlegs) {
@@ -773,6 +840,7 @@ gm_status gm_ser_chain_backward(const int32_t *a1_idx, const float *a1_w, int s2
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!gout || !dw1 || !dleg) return GM_ERR_INVALID_ARG;
     gm::ChainBwdArgs b{};
+    check_chain_edges(a, stream);
     b.f = a;
     b.gout = gout;
     b.grad_is_log = grad_is_log;
@@ -818,6 +886,7 @@ gm_status gm_ser_sea_chain_forward(const int32_t *a1_idx, const float *a1_w, int
     st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    check_chain_edges(sa, stream);
     sa.out_idx = out_idx;
     sa.out_w = out_w;
     SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, sa.rows, row_map(hkv, n)};
@@ -844,6 +913,7 @@ gm_status gm_sea_forward(const void *q, const void *k, const void *v, gm_dtype d
     gm_status st = check_sea(q, k, v, dtype, idx, w, s, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    check_edges(idx, w, s, B, n, hkv, stream);
     SeaArgs a{q, k, v, idx, w, o, lse, s, n, hkv, scale, (uint32_t)((int64_t)B * n * hkv),
               row_map(hkv, n)};
     return dispatch<SeaFwd>(dtype, d, hq / hkv, a, stream);
@@ -865,6 +935,8 @@ gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     st = check_sea(q, k, v, dtype, &dummy_idx, &dummy_w, s1, B, n, hq, hkv, d, scale);
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!o || !aligned16(o)) return GM_ERR_INVALID_ARG;
+    check_edges(a1_idx, a1_w, s2, B, n, hkv, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, hkv, stream);
     const uint32_t rows = (uint32_t)((int64_t)B * n * hkv);
     SerArgs sa{a1_idx, a1_w, a2_idx, a2_w, out_idx, out_w, s1, s2, s3, n, hkv, rows, row_map(hkv, n)};
     SeaArgs a{q, k, v, nullptr, nullptr, o, lse, s1, n, hkv, scale, rows, row_map(hkv, n)};
@@ -890,6 +962,7 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     if (st != GM_OK || (int64_t)B * n == 0) return st;
     if (!dout || !dq || !dk || !dv || !dlogw) return GM_ERR_INVALID_ARG;
     if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
+    check_edges(idx, w, s, B, n, hkv, stream);
     const int64_t rows = (int64_t)B * n * hkv;
     SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, nullptr,
                  s, n, hkv, scale, accumulate, (uint32_t)rows, row_map(hkv, n)};
@@ -974,7 +1047,8 @@ gm_status gm_check_device_errors(cudaStream_t stream)
     if (flag == 0) return GM_OK;
     const unsigned zero = 0;
     if (cudaMemcpyToSymbol(gm::g_error_flag, &zero, sizeof(zero)) != cudaSuccess) return GM_ERR_CUDA;
-    return (flag & gm::ERR_WAIT_TIMEOUT) ? GM_ERR_WAIT_TIMEOUT : GM_ERR_INDEX_RANGE;
+    if (flag & gm::ERR_WAIT_TIMEOUT) return GM_ERR_WAIT_TIMEOUT;
+    return (flag & gm::ERR_EDGE_INVALID) ? GM_ERR_EDGE_INVALID : GM_ERR_INDEX_RANGE;
 }
 
 }  // extern "C"

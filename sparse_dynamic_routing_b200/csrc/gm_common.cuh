@@ -36,10 +36,13 @@ constexpr float LN2 = 0.6931471805599453f;
 // Device error word of this library (one per device). Bit 0: an active slot indexed
 // outside [0, n). Kernels set it with atomicOr and carry on; the host reads and clears it.
 // Bit 1: a bounded wait on an asynchronous copy or tensor-core operation ran out of time (the
-// kernel gave up on its remaining work).
+// kernel gave up on its remaining work). Bit 2: see ERR_EDGE_INVALID.
 __device__ unsigned int g_error_flag;
 constexpr unsigned ERR_INDEX_RANGE = 1u;
 constexpr unsigned ERR_WAIT_TIMEOUT = 2u;
+// Bit 2 (checked builds only): an input edge had a negative or non-finite weight, or an
+// active index beyond its row's own position.
+constexpr unsigned ERR_EDGE_INVALID = 4u;
 
 __device__ __forceinline__ void raise_index_error() { atomicOr(&g_error_flag, ERR_INDEX_RANGE); }
 

@@ -51,7 +51,7 @@ def test_workspace_size(lib):
 
 
 def test_status_strings(lib):
-    for st in range(5):
+    for st in range(8):
         assert bnd.status_string(st).startswith("GM_")
     assert "unknown" in bnd.status_string(99)
     assert lib.gm_version() >= 100
@@ -210,3 +210,14 @@ def test_binding_signatures_match_the_header():
         params = params.strip()
         n = 0 if params in ("", "void") else params.count(",") + 1
         assert len(bnd.SIGNATURES[name]) == n, f"{name}: header has {n} parameters"
+
+
+def test_checked_build_exports_the_same_symbols(lib):
+    """The checked build (input edges verified before every call) is the same ABI."""
+    build.build(checked=True)
+    checked = bnd.open_library(bnd.CHECKED_LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(checked, name), name
+    assert checked.gm_checked_build() == 1
+    assert lib.gm_checked_build() == 0
+    assert "checked" in checked.gm_status_string(bnd.GM_ERR_EDGE_INVALID).decode()

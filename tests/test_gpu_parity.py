@@ -109,13 +109,20 @@ def test_stack_of_21_layers_carries_edges():
         e_idx, e_w, bad = oracle.ser(e_idx, e_w, e_idx, e_w, wl.s1)
         assert bad == 0
         assert_ser_equal(ni, nw, e_idx, e_w)
-        rows = np.sort(rng.choice(wl.B * wl.n, size=512, replace=False))
-        rows[:2] = [0, wl.B * wl.n - 1]
-        o_ref, lse_ref, _ = oracle.sea_forward(f["q"], f["k"], f["v"], e_idx, e_w, wl.scale,
-                                               rows=rows)
-        sel = torch.from_numpy(rows).cuda()
-        assert_close(o.reshape(wl.B * wl.n, wl.hq, wl.d)[sel], o_ref, TOL["bf16"], f"o L{layer}")
-        assert_close(lse.reshape(wl.B * wl.n, wl.hq)[sel], lse_ref, TOL["bf16"], f"lse L{layer}")
+        if layer in (0, wl.layers - 1):
+            # the first layer and the last (edges collapsed toward the first positions: hot
+            # rows, heavy merges) on every row
+            o_ref, lse_ref, _ = oracle.sea_forward(f["q"], f["k"], f["v"], e_idx, e_w, wl.scale)
+            assert_close(o, o_ref, TOL["bf16"], f"o L{layer}")
+            assert_close(lse, lse_ref, TOL["bf16"], f"lse L{layer}")
+        else:
+            rows = np.sort(rng.choice(wl.B * wl.n, size=512, replace=False))
+            rows[:2] = [0, wl.B * wl.n - 1]
+            o_ref, lse_ref, _ = oracle.sea_forward(f["q"], f["k"], f["v"], e_idx, e_w, wl.scale,
+                                                   rows=rows)
+            sel = torch.from_numpy(rows).cuda()
+            assert_close(o.reshape(wl.B * wl.n, wl.hq, wl.d)[sel], o_ref, TOL["bf16"], f"o L{layer}")
+            assert_close(lse.reshape(wl.B * wl.n, wl.hq)[sel], lse_ref, TOL["bf16"], f"lse L{layer}")
         g_idx, g_w = ni, nw
     gm.gm_check_device_errors()
 
