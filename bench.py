@@ -521,6 +521,18 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     ch_dl = [torch.empty((B, n, k, wl.s3), dtype=f32, device=dev) for _ in ch_legs]
     e_b, mix_b = tok * k * wl.s1 * 8, 2 * tok * k * k * 4
     leg_b, grad_b = tok * k * (wl.s2 + wl.s3) * 8, tok * k * (wl.s2 + wl.s3) * 4
+    # the fused backward of the referral and the attention (its bytes: the attention backward's
+    # plus the legs read, their gradients written, dw2 read-modify-written)
+    bwd_b = compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ap_i.cpu().numpy(),
+                             ap_w.cpu().numpy())["backward"]
+    f_dq = torch.empty((B, n, wl.hq, wl.d), dtype=f32, device=dev)
+    f_dk = torch.empty((B, n, k, wl.d), dtype=f32, device=dev)
+    f_dv = torch.empty_like(f_dk)
+    f_dlw = torch.empty((B, n, k, wl.s1), dtype=f32, device=dev)
+    f_dw1 = torch.empty((B, n, k, wl.s2), dtype=f32, device=dev)
+    f_dw2 = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
+    f_ws = torch.empty(gm.gm_sea_backward_workspace_size(g["q"].dtype, wl.s1, B, n, wl.hq, k, wl.d),
+                       dtype=torch.uint8, device=dev)
     calls = {
         "leg_sparsify": ("leg_fwd_tile_kernel", e_b + mix_b + leg_b,
                          lambda: gm.gm_leg_sparsify(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
@@ -554,6 +566,21 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
                                lambda: gm.gm_ser_chain_backward(
                                    g["a1_idx"], g["a1_w"], ch_legs, wl.s2, dlw, grad_is_log=True,
                                    dw1=ch_dw1, dlegs=ch_dl, stream=stream)),
+        "ser_sea_backward": ("count + scan + sea_bwd_tile_kernel with the referral backward + gather",
+                             bwd_b + leg_b + grad_b + tok * k * wl.s3 * 4,
+                             lambda: gm.gm_ser_sea_backward(
+                                 g["q"], g["k"], g["v"], g["dout"], g["a1_idx"], g["a1_w"], g["a2_idx"],
+                                 g["a2_w"], ap_i, ap_w, wl.scale, dq=f_dq, dk=f_dk, dv=f_dv, dlogw=f_dlw,
+                                 dw1=f_dw1, dw2=f_dw2, workspace=f_ws, stream=stream)),
+        "sea_backward_then_ser_backward": ("the unfused pair of the row above",
+                                           bwd_b + leg_b + grad_b + tok * k * wl.s3 * 4,
+                                           lambda: (gm.gm_sea_backward(
+                                               g["q"], g["k"], g["v"], g["dout"], ap_i, ap_w, wl.scale,
+                                               dq=f_dq, dk=f_dk, dv=f_dv, dlogw=f_dlw, workspace=f_ws,
+                                               stream=stream),
+                                               gm.gm_ser_backward(g["a1_idx"], g["a1_w"], g["a2_idx"],
+                                                                  g["a2_w"], f_dlw, grad_is_log=True,
+                                                                  dw1=f_dw1, dw2=f_dw2, stream=stream))),
         "leg_backward": ("leg_bwd_tile_kernel", e_b + mix_b + grad_b + tok * k * wl.s1 * 4 + mix_b,
                          lambda: gm.gm_leg_backward(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     dw1, dw2, dew=dew, dmix1=dm1, dmix2=dm2,

@@ -438,6 +438,37 @@ gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, c
 size_t gm_sea_backward_noalloc_max_scratch(void);
 
 /*
+ * gm_ser_sea_backward - the backward of one sparse layer's referral and attention in one call:
+ * gm_sea_backward on A' (the referral's output edges), and the referral backward of the d ln w
+ * it computes, to both legs' weights. Sources: ai.info summary, "Key Contributions" item 3
+ * (SEA on the referral's edges) and "Methodology in Plain English", referral paragraph (only
+ * the retained referral weights receive gradient).
+ *
+ *   q, k, v, dout, dtype, scale, B, n, hq, hkv, d   as gm_sea_backward
+ *   a1_idx/a1_w [B, n, hkv, s2], a2_idx/a2_w [B, n, hkv, s3]   the referral's legs
+ *   idx/w [B, n, hkv, s1]   A' = Sparsify_s1(A1 A2), exactly as gm_ser_sea_forward returned it
+ *                           (its kept set decides which paths receive gradient)
+ *   dq, dk, dv, dlogw       as gm_sea_backward (dlogw is required)
+ *   dw1 [B, n, hkv, s2], dw2 [B, n, hkv, s3]   gradients of the legs' weights, as
+ *                           gm_ser_backward with grad_is_log = 1 and gout = dlogw
+ *   workspace, workspace_bytes   as gm_sea_backward (gm_sea_backward_workspace_size(..., s1, ...))
+ *   accumulate              0: overwrite every output; 1: add to them (fused shapes only)
+ * With a workspace, s2 = s3 in {2, 4}, s1 <= 4, 16-byte aligned legs and a shape the gather
+ * path covers, the referral backward runs inside the attention backward's row pass (the d ln w
+ * of a tile stays in shared memory, A' is read once); otherwise the call runs gm_sea_backward
+ * and then gm_ser_backward (accumulate must then be 0: GM_ERR_UNSUPPORTED otherwise). dw2 is
+ * summed with fp32 atomics (order varies run to run); everything else is deterministic.
+ * Errors: as gm_sea_backward and gm_ser_backward.
+ */
+gm_status gm_ser_sea_backward(const void *q, const void *k, const void *v, const void *dout, gm_dtype dtype,
+                              const int32_t *a1_idx, const float *a1_w, int s2,
+                              const int32_t *a2_idx, const float *a2_w, int s3,
+                              const int32_t *idx, const float *w, int s1,
+                              int B, int n, int hq, int hkv, int d, float scale,
+                              float *dq, float *dk, float *dv, float *dlogw, float *dw1, float *dw2,
+                              void *workspace, size_t workspace_bytes, int accumulate, cudaStream_t stream);
+
+/*
  * gm_dense_refresh_edges - refresh edges from a dense attention layer: for every (b, i, KV
  * head h), the sf positions t <= i that the dense layer's attention weights most heavily.
  * Source: ai.info summary, "Methodology in Plain English", referral paragraph (refresh edges

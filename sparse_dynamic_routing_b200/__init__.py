@@ -14,6 +14,7 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_ser_sea_forward  both in one kernel
     gm_sea_backward     gradients of sparse edge attention
     gm_ser_backward     gradients of the kept referral weights
+    gm_ser_sea_backward both backward passes in one call (the referral's inside the attention's)
     gm_dense_refresh_edges
                         refresh edges from a dense attention layer (its top positions)
 """
@@ -41,6 +42,7 @@ from ._binding import (  # noqa: F401
     gm_ser_refresh_forward,
     gm_ser_sea_chain_forward,
     gm_ser_sea_refresh_forward,
+    gm_ser_sea_backward,
     gm_ser_sea_forward,
     gm_version,
     load_library,

@@ -53,6 +53,9 @@ SIGNATURES = {
     "gm_sea_backward_noalloc": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _ci, _ci, _ci, _ci, _ci,
                                 _cf, _vp, _vp, _vp, _vp, _ci, _vp],
     "gm_sea_backward_noalloc_max_scratch": [],
+    "gm_ser_sea_backward": [_vp, _vp, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _vp, _vp, _ci, _ci,
+                            _ci, _ci, _ci, _ci, _cf, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                            _ci, _vp],
     "gm_dense_refresh_edges": [_vp, _vp, _ci, _vp, _ci, _ci, _ci, _ci, _ci, _cf, _ci, _vp, _vp, _vp],
     "gm_check_device_errors": [_vp],
     "gm_status_string": [_ci],
@@ -537,6 +540,47 @@ def gm_sea_backward_noalloc(q, k, v, dout, idx, w, scale=None, dq=None, dk=None,
         _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"), int(bool(accumulate)), _stream(stream))
     _check(st, "gm_sea_backward_noalloc")
     return dq, dk, dv, dlogw
+
+
+def gm_ser_sea_backward(q, k, v, dout, a1_idx, a1_w, a2_idx, a2_w, idx, w, scale=None, dq=None,
+                        dk=None, dv=None, dlogw=None, dw1=None, dw2=None, accumulate=False,
+                        workspace="auto", stream=None):
+    """Backward of the referral and the attention in one call (A' = idx/w as the forward
+    returned it). Returns (dq, dk, dv, dlogw, dw1, dw2), all fp32."""
+    B, n, hq, d = q.shape
+    hkv, s1 = idx.shape[2], idx.shape[3]
+    s2, s3 = a1_idx.shape[3], a2_idx.shape[3]
+    if tuple(a1_idx.shape[:3]) != (B, n, hkv) or tuple(a2_idx.shape[:3]) != (B, n, hkv):
+        raise ValueError("legs must be [B, n, hkv, s]")
+    if a1_w.shape != a1_idx.shape or a2_w.shape != a2_idx.shape or w.shape != idx.shape:
+        raise ValueError("edge weight shapes disagree with their indices")
+    if k.shape != (B, n, hkv, d) or v.shape != k.shape or dout.shape != q.shape or dout.dtype != q.dtype:
+        raise ValueError("feature shapes disagree")
+    dev = q.device
+    f32 = torch.float32
+    dq = torch.empty((B, n, hq, d), dtype=f32, device=dev) if dq is None else dq
+    dk = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dk is None else dk
+    dv = torch.empty((B, n, hkv, d), dtype=f32, device=dev) if dv is None else dv
+    dlogw = torch.empty((B, n, hkv, s1), dtype=f32, device=dev) if dlogw is None else dlogw
+    dw1 = torch.empty((B, n, hkv, s2), dtype=f32, device=dev) if dw1 is None else dw1
+    dw2 = torch.empty((B, n, hkv, s3), dtype=f32, device=dev) if dw2 is None else dw2
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a CUDA tensor")
+        nbytes = gm_sea_backward_workspace_size(q.dtype, s1, B, n, hq, hkv, d)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (
+        _ptr(workspace, name="workspace"), workspace.numel() * workspace.element_size())
+    st = load_library().gm_ser_sea_backward(
+        _ptr(q, name="q"), _ptr(k, name="k"), _ptr(v, name="v"), _ptr(dout, name="dout"), _fdtype(q),
+        _ptr(a1_idx, torch.int32, "a1_idx"), _ptr(a1_w, f32, "a1_w"), s2,
+        _ptr(a2_idx, torch.int32, "a2_idx"), _ptr(a2_w, f32, "a2_w"), s3,
+        _ptr(idx, torch.int32, "idx"), _ptr(w, f32, "w"), s1, B, n, hq, hkv, d, _scale(scale, d),
+        _ptr(dq, f32, "dq"), _ptr(dk, f32, "dk"), _ptr(dv, f32, "dv"), _ptr(dlogw, f32, "dlogw"),
+        _ptr(dw1, f32, "dw1"), _ptr(dw2, f32, "dw2"), ws_ptr, ws_bytes, int(bool(accumulate)),
+        _stream(stream))
+    _check(st, "gm_ser_sea_backward")
+    return dq, dk, dv, dlogw, dw1, dw2
 
 
 def gm_dense_refresh_edges(q, k, lse, sf: int, scale=None, out_idx=None, out_w=None, stream=None):

@@ -361,12 +361,12 @@ template <typename T, int D, int G> struct SeaFwd {
 constexpr int BWD_TILE_P = GM_BWD_TILE_P;
 constexpr int WPB_BWD_TILE = GM_WPB_BWD_TILE;
 
-template <typename T, int D, int G, int S1M, bool GATHER>
+template <typename T, int D, int G, int S1M, bool GATHER, int SB = 0>
 gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
 {
     using TG = gm::BwdTileGeom<T, D, G, S1M>;
-    auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE, GATHER>;
-    const size_t smem = (size_t)WPB_BWD_TILE * (32 * S1M * 8 + BWD_TILE_P * TG::STAGE);
+    auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE, GATHER, SB>;
+    const size_t smem = (size_t)WPB_BWD_TILE * (gm::bwd_tile_bytes<S1M, SB>() + BWD_TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GM_ERR_CUDA;
@@ -431,7 +431,10 @@ WsLayout ws_layout(int64_t R, int64_t E, int G)
 }
 
 template <typename T, int D, int G> struct SeaBwdGather {
-    static gm_status run(SeaBwdArgs a, gm::GatherWs ws, const int32_t *idx, const float *w, cudaStream_t st)
+    // sb > 0: the row pass also runs the referral backward of A' = Sparsify(A1 A2) with
+    // budgets s2 = s3 = sb (a.a1_idx ... a.dw2 set; the caller checked the shapes)
+    static gm_status run(SeaBwdArgs a, gm::GatherWs ws, const int32_t *idx, const float *w, cudaStream_t st,
+                         int sb = 0)
     {
         if constexpr (TileOK<T, D, G>::value && 2 * (D / gm::Vec<T>::N) <= 32 && 2 * G <= 8) {
             const int64_t R = a.rows, E = R * a.s;
@@ -447,7 +450,13 @@ template <typename T, int D, int G> struct SeaBwdGather {
             a.cnt = ws.cnt;
             a.off = ws.off;
             a.srec = ws.srec;
-            const gm_status rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
+            gm_status rs;
+            if (sb == 2)
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 2>(a, st) : launch_bwd_tile<T, D, G, 4, true, 2>(a, st);
+            else if (sb == 4)
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 4>(a, st) : launch_bwd_tile<T, D, G, 4, true, 4>(a, st);
+            else
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
             if (rs != GM_OK) return rs;
             auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
             const size_t smem = (size_t)WPB_GATHER * gm::gather_warp_bytes<G>(GATHER_U, GATHER_P);
@@ -1010,6 +1019,54 @@ gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, c
 }
 
 size_t gm_sea_backward_noalloc_max_scratch(void) { return NOALLOC_SCRATCH_BYTES; }
+
+gm_status gm_ser_sea_backward(const void *q, const void *k, const void *v, const void *dout, gm_dtype dtype,
+                              const int32_t *a1_idx, const float *a1_w, int s2,
+                              const int32_t *a2_idx, const float *a2_w, int s3,
+                              const int32_t *idx, const float *w, int s1,
+                              int B, int n, int hq, int hkv, int d, float scale,
+                              float *dq, float *dk, float *dv, float *dlogw, float *dw1, float *dw2,
+                              void *workspace, size_t workspace_bytes, int accumulate, cudaStream_t stream)
+{
+    if (accumulate != 0 && accumulate != 1) return GM_ERR_INVALID_ARG;
+    gm_status st = check_ser(a1_idx, a1_w, s2, a2_idx, a2_w, s3, s1, B, n, hkv);
+    if (st != GM_OK) return st;
+    st = check_sea(q, k, v, dtype, idx, w, s1, B, n, hq, hkv, d, scale);
+    if (st != GM_OK || (int64_t)B * n == 0) return st;
+    if (!dout || !dq || !dk || !dv || !dlogw || !dw1 || !dw2) return GM_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return GM_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)B * n * hkv;
+    const size_t need = gm_sea_backward_workspace_size(dtype, s1, B, n, hq, hkv, d);
+    const bool legs_aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w);
+    const bool fused = workspace != nullptr && need > 0 && legs_aligned && s2 == s3 && (s2 == 2 || s2 == 4) && s1 <= 4;
+    if (!fused) {
+        // the unfused pair: attention backward, then the referral backward of its d ln w (which
+        // needs this call's d ln w alone: no accumulation into the caller's)
+        if (accumulate) return GM_ERR_UNSUPPORTED;
+        st = gm_sea_backward(q, k, v, dout, dtype, idx, w, s1, B, n, hq, hkv, d, scale, dq, dk, dv, dlogw,
+                             workspace, workspace_bytes, 0, stream);
+        if (st != GM_OK) return st;
+        return gm_ser_backward(a1_idx, a1_w, s2, a2_idx, a2_w, s3, dlogw, s1, 1, B, n, hkv, dw1, dw2, 0,
+                               stream);
+    }
+    if (workspace_bytes < need || !aligned16(workspace)) return GM_ERR_INVALID_ARG;
+    check_edges(a1_idx, a1_w, s2, B, n, hkv, stream);
+    check_edges(a2_idx, a2_w, s3, B, n, hkv, stream);
+    check_edges(idx, w, s1, B, n, hkv, stream);
+    if (!accumulate) {
+        gm::zero_i32_kernel<<<148 * 4, 256, 0, stream>>>(reinterpret_cast<int32_t *>(dw2), rows * s3);
+        if (launched() != GM_OK) return GM_ERR_CUDA;
+    }
+    SeaBwdArgs a{q, k, v, dout, idx, w, dq, dk, dv, dlogw, nullptr, nullptr, nullptr,
+                 s1, n, hkv, scale, accumulate, (uint32_t)rows, row_map(hkv, n),
+                 a1_idx, a2_idx, a1_w, a2_w, dw1, dw2};
+    const WsLayout L = ws_layout(rows, rows * s1, hq / hkv);
+    char *base = static_cast<char *>(workspace);
+    const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
+                          reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.srec),
+                          L.nblk};
+    return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream, s2);
+}
 
 gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, const float *lse,
                                  int B, int n, int hq, int hkv, int d, float scale, int sf,

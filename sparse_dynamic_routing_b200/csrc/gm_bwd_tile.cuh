@@ -44,17 +44,86 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
 #define GM_BWD_TILE_MINB 4
 #endif
 
-template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER>
+// Shared memory per warp of the tile row pass: the edge tile (K/V row, log2 w per slot), with
+// the fused referral backward (SB > 0) also each slot's target, weight and d ln w, then the
+// P stages.
+template <int S1M, int SB> __host__ __device__ constexpr int bwd_tile_bytes()
+{
+    return 32 * S1M * (SB > 0 ? 20 : 8);
+}
+
+// Referral backward of one edge row by one thread, fused after the attention backward of its
+// tile: the forward kept (kt[r], kw[r]) (index, weight > 0) of A' = Sparsify(A1 A2); g[r] is
+// the gradient of ln kw[r]. Each two-hop candidate (a, e) whose product fl32(w1 w2) is nonzero
+// and whose target was kept passes g / W to dw1[a] (times w2, summed in ascending e, each
+// product and add rounded once, as ser_bwd_thread_kernel) and to dw2 of its second-leg slot
+// (times w1, fp32 atomics).
+template <int SB, int S1M>
+__device__ __forceinline__ void ser_backward_row(const SeaBwdArgs &a, uint32_t row, uint32_t seq_base, uint32_t h,
+                                                 const int32_t (&kt)[S1M], const float (&kw)[S1M],
+                                                 const float (&gl)[S1M])
+{
+    float kg[S1M];
+#pragma unroll
+    for (int r = 0; r < S1M; ++r) kg[r] = kw[r] > 0.0f ? gl[r] / kw[r] : 0.0f;
+    int32_t j[SB];
+    float w1[SB];
+    ld_vec<SB>(a.a1_idx + (size_t)row * SB, j);
+    ld_vec<SB>(a.a1_w + (size_t)row * SB, w1);
+#pragma unroll
+    for (int x = 0; x < SB; ++x) {
+        bool act = w1[x] > 0.0f;
+        if (act && (uint32_t)j[x] >= (uint32_t)a.n) {
+            raise_index_error();
+            act = false;
+        }
+        int32_t t2[SB];
+        float w2[SB];
+#pragma unroll
+        for (int e = 0; e < SB; ++e) {
+            t2[e] = 0;
+            w2[e] = 0.0f;
+        }
+        const size_t r2 = act ? ((size_t)(seq_base + (uint32_t)j[x]) * a.hkv + h) * SB : 0;
+        if (act) {
+            ld_vec<SB>(a.a2_idx + r2, t2);
+            ld_vec<SB>(a.a2_w + r2, w2);
+        }
+        float d1 = 0.0f;
+#pragma unroll
+        for (int e = 0; e < SB; ++e) {
+            bool v = w2[e] > 0.0f;
+            if (v && (uint32_t)t2[e] >= (uint32_t)a.n) {
+                raise_index_error();
+                v = false;
+            }
+            const bool cand = v && __fmul_rn(w1[x], w2[e]) != 0.0f;
+            float g = 0.0f;
+#pragma unroll
+            for (int r = 0; r < S1M; ++r) g = (cand && t2[e] == kt[r] && kw[r] > 0.0f) ? kg[r] : g;
+            d1 = __fadd_rn(d1, __fmul_rn(g, w2[e]));
+            if (g != 0.0f) atomicAdd(a.dw2 + r2 + e, __fmul_rn(g, w1[x]));
+        }
+        float *p = a.dw1 + (size_t)row * SB + x;
+        *p = a.accumulate ? *p + d1 : d1;
+    }
+}
+
+template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER, int SB = 0>
 __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
     using TG = BwdTileGeom<T, D, G, S1M>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    constexpr int TILE_BYTES = 32 * S1M * 8;
+    constexpr int TILE_BYTES = bwd_tile_bytes<S1M, SB>();
     char *wbase = smem + (size_t)wid * (TILE_BYTES + P * TG::STAGE);
     int32_t *tile_t = reinterpret_cast<int32_t *>(wbase);
     float *tile_lw = reinterpret_cast<float *>(wbase + 32 * S1M * 4);
+    // fused referral backward: raw targets, weights and d ln w of the tile's slots
+    int32_t *tile_tt = reinterpret_cast<int32_t *>(wbase + 32 * S1M * 8);
+    float *tile_w = reinterpret_cast<float *>(wbase + 32 * S1M * 12);
+    float *tile_g = reinterpret_cast<float *>(wbase + 32 * S1M * 16);
     char *stages = wbase + TILE_BYTES;
 
     const uint32_t rows = a.rows;
@@ -94,6 +163,11 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 }
                 tile_t[lane * S1M + r] = (int32_t)((seq_base + (uint32_t)t) * (uint32_t)a.hkv + h);
                 tile_lw[lane * S1M + r] = lw;
+                if constexpr (SB > 0) {
+                    tile_tt[lane * S1M + r] = t;
+                    tile_w[lane * S1M + r] = lw == -INFINITY ? 0.0f : __ldg(a.w + (size_t)row * a.s + r);
+                    tile_g[lane * S1M + r] = 0.0f;
+                }
             }
         }
         __syncwarp();
@@ -369,12 +443,28 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                     }
                     float *pd = a.dlogw + (size_t)row * a.s + c;
                     *pd = a.accumulate ? *pd + dl : dl;
+                    if constexpr (SB > 0) tile_g[lr * S1M + c] = dl;  // this call's gradient only
                 }
             }
             issue(pass + P);
         }
         cp_async_wait<0>();
         __syncwarp();
+        if constexpr (SB > 0) {
+            // ---- phase 3: the referral backward of the tile's rows, one thread per row ------
+            const uint32_t row = r0 + lane;
+            if (row < rows) {
+                uint32_t seq_base, h;
+                a.map.split(row, seq_base, h);
+                int32_t kt[S1M];
+                float kw[S1M], gl[S1M];
+                ld_tile<S1M>(tile_tt + lane * S1M, kt);
+                ld_tile<S1M>(tile_w + lane * S1M, kw);
+                ld_tile<S1M>(tile_g + lane * S1M, gl);
+                ser_backward_row<SB, S1M>(a, row, seq_base, h, kt, kw, gl);
+            }
+            __syncwarp();  // the tile arrays are rewritten by the next tile's phase 1
+        }
     }
 }
 

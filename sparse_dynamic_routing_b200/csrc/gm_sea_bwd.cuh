@@ -40,6 +40,12 @@ struct SeaBwdArgs {
     int accumulate;
     uint32_t rows;  // B * n * hkv
     RowMap map;     // heads = hkv
+    // fused referral backward (tile row pass with SB > 0): A' = Sparsify_s(A1 A2) was the
+    // referral's output; the gradient of ln A'.w that this backward computes flows on to the
+    // legs' weights (dw1 [rows, SB] stored, dw2 [rows, SB] scatter-added)
+    const int32_t *a1_idx, *a2_idx;
+    const float *a1_w, *a2_w;
+    float *dw1, *dw2;
 };
 
 __device__ __forceinline__ void red_add4(float *p, float a, float b, float c, float d)
