@@ -866,6 +866,29 @@ gm_status gm_ser_chain_backward(const int32_t *a1_idx, const float *a1_w, int s2
             if (launched() != GM_OK) return GM_ERR_CUDA;
         }
     }
+    // one thread per row for budgets 2 or 4 (vector loads need 16-byte aligned legs)
+    bool aligned = aligned16(a1_idx) && aligned16(a1_w);
+    for (int m = 0; m < nlegs; ++m) aligned = aligned && aligned16(leg_idx[m]) && aligned16(leg_w[m]);
+    if (aligned && s2 == s3 && s_mid == s2 && (s2 == 2 || s2 == 4) && s1 <= 4 && nlegs <= 4) {
+        const unsigned tgrid = blocks_for(a.rows, 32 * WPB_SER_THREAD);
+        constexpr int W = WPB_SER_THREAD;
+        if (s2 == 2) {
+            switch (nlegs) {
+            case 1: gm::ser_chain_bwd_thread_kernel<2, 1, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            case 2: gm::ser_chain_bwd_thread_kernel<2, 2, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            case 3: gm::ser_chain_bwd_thread_kernel<2, 3, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            default: gm::ser_chain_bwd_thread_kernel<2, 4, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            }
+        } else {
+            switch (nlegs) {
+            case 1: gm::ser_chain_bwd_thread_kernel<4, 1, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            case 2: gm::ser_chain_bwd_thread_kernel<4, 2, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            case 3: gm::ser_chain_bwd_thread_kernel<4, 3, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            default: gm::ser_chain_bwd_thread_kernel<4, 4, W><<<tgrid, W * 32, 0, stream>>>(b); break;
+            }
+        }
+        return launched();
+    }
     const unsigned grid = blocks_for(a.rows, WPB_SER);
     switch (nlegs) {
     case 1: gm::ser_chain_bwd_kernel<1, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(b); break;

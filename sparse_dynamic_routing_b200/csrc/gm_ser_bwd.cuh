@@ -96,40 +96,29 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
     }
 }
 
-// The same backward, one thread per edge row, for small exact budgets (S2, S3; s1 <= S1M):
-// the referral is recomputed in registers exactly as the fused forward's per-thread referral
-// (same products, pairwise merge in ascending candidate order, arg-max selection), each
-// candidate finds the kept slot of its target, the first-leg gradient of slot a is summed
-// in ascending e, and the second-leg gradients are scatter-added with fp32 atomics. It
-// spends a fraction of the warp-per-row kernel's instructions when the budgets are 2 or 4.
-//
-// The dispatch picks this kernel or ser_bwd_kernel by shape and alignment alone, so the two
-// must agree bit for bit: the candidate products (__fmul_rn), the merge in ascending candidate
-// order (merge_pairs here and refer_thread in gm_fused_tile.cuh; __match_any_sync groups
-// summed from their first lane in refer_merge), the selection (weight descending, then target
-// ascending, zero weights never kept), g / W for a log-weight gradient, and the first-leg sums
-// (g * w2 rounded, then added in ascending e). Only dw2, summed by atomics, varies in order.
-template <int S2, int S3, int S1M, int WPB, int SF = 0>
-__global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
+// Backward of one referral step of one row by one thread. The step's candidates are
+// recomputed from the first leg (j, w1) [S_IN] and the second-leg rows at (leg_idx, leg_w)
+// [S3 each] (then the row's SF refresh slots when SF > 0), merged and selected exactly as
+// refer_thread does (the kept set, s_keep <= S_OUT slots); with g[r] the upstream gradient of
+// kept slot r (of ln W_r when is_log), each candidate reaching a kept target passes it on:
+// d1[a] = sum over e of g * w2 (ascending e, each product and add rounded once), g * w1 is
+// added to the second-leg weight (fp32 atomics into dleg), and refresh slot f gets gf[f] = g.
+template <int S_IN, int S3, int S_OUT, int SF = 0>
+__device__ __forceinline__ void refer_thread_backward(const SerArgs &a, uint32_t row, uint32_t seq_base,
+                                                      uint32_t h, const int32_t (&j)[S_IN],
+                                                      const float (&w1)[S_IN], const int32_t *leg_idx,
+                                                      const float *leg_w, int s_keep,
+                                                      const float (&g)[S_OUT], bool is_log, float *dleg,
+                                                      float (&d1)[S_IN], float (&gf)[SF > 0 ? SF : 1])
 {
-    constexpr int NP2 = S2 * S3, NC = NP2 + SF;  // SF refresh slots after the paths
-    const SerArgs &a = b.f;
-    const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
-    if (row >= a.rows) return;  // no warp-wide operation below
-    uint32_t seq_base, h;
-    a.map.split(row, seq_base, h);
-    int32_t j[S2];
-    float w1[S2];
-    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
-    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
-
+    constexpr int NP2 = S_IN * S3, NC = NP2 + SF;  // SF refresh slots after the paths
     int32_t ct[NC];
     float cu[NC], w2c[NC];
-    size_t r2[S2];
+    size_t r2[S_IN];
 #pragma unroll
-    for (int x = 0; x < S2; ++x) {
+    for (int x = 0; x < S_IN; ++x) {
         bool act = w1[x] > 0.0f;
-        if (act && (j[x] < 0 || j[x] >= a.n)) {
+        if (act && (uint32_t)j[x] >= (uint32_t)a.n) {
             raise_index_error();
             act = false;
         }
@@ -142,13 +131,13 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
         }
         r2[x] = act ? ((size_t)(seq_base + (uint32_t)j[x]) * a.k + h) * S3 : 0;
         if (act) {
-            ld_vec<S3>(a.a2_idx + r2[x], t2);
-            ld_vec<S3>(a.a2_w + r2[x], w2);
+            ld_vec<S3>(leg_idx + r2[x], t2);
+            ld_vec<S3>(leg_w + r2[x], w2);
         }
 #pragma unroll
         for (int e = 0; e < S3; ++e) {
             bool v = w2[e] > 0.0f;
-            if (v && (t2[e] < 0 || t2[e] >= a.n)) {
+            if (v && (uint32_t)t2[e] >= (uint32_t)a.n) {
                 raise_index_error();
                 v = false;
             }
@@ -166,7 +155,7 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 #pragma unroll
         for (int f = 0; f < SF; ++f) {
             bool v = wf[f] > 0.0f;
-            if (v && (tf[f] < 0 || tf[f] >= a.n)) {
+            if (v && (uint32_t)tf[f] >= (uint32_t)a.n) {
                 raise_index_error();
                 v = false;
             }
@@ -179,10 +168,10 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
     for (int c = 0; c < NC; ++c) cand[c] = cu[c] != 0.0f;
     merge_pairs<0, NC>(ct, cu);
     // selection (weight desc, target asc) and the upstream gradient of each kept slot
-    int32_t kt[S1M];
-    float kg[S1M];
+    int32_t kt[S_OUT];
+    float kg[S_OUT];
 #pragma unroll
-    for (int r = 0; r < S1M; ++r) {
+    for (int r = 0; r < S_OUT; ++r) {
         float bw = 0.0f;
         int32_t bt = 0;
 #pragma unroll
@@ -193,37 +182,78 @@ __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
         }
 #pragma unroll
         for (int c = 0; c < NC; ++c) cu[c] = (cu[c] == bw && ct[c] == bt) ? 0.0f : cu[c];
-        const bool keep = r < a.s1 && bw > 0.0f;
-        float g = keep ? __ldg(b.gout + (size_t)row * a.s1 + r) : 0.0f;
-        if (b.grad_is_log) g = keep ? g / bw : 0.0f;
+        const bool keep = r < s_keep && bw > 0.0f;
+        float gr = keep ? g[r] : 0.0f;
+        if (is_log) gr = keep ? gr / bw : 0.0f;
         kt[r] = keep ? bt : -1;  // -1 never equals a valid target
-        kg[r] = g;
+        kg[r] = gr;
     }
     // per candidate: the gradient of its kept target (0 if cut)
     float gc[NC];
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-        float g = 0.0f;
+        float gg = 0.0f;
 #pragma unroll
-        for (int r = 0; r < S1M; ++r) g = (cand[c] && ct[c] == kt[r]) ? kg[r] : g;
-        gc[c] = g;
+        for (int r = 0; r < S_OUT; ++r) gg = (cand[c] && ct[c] == kt[r]) ? kg[r] : gg;
+        gc[c] = gg;
     }
 #pragma unroll
-    for (int x = 0; x < S2; ++x) {
-        float d1 = 0.0f;
+    for (int x = 0; x < S_IN; ++x) {
+        float acc = 0.0f;
 #pragma unroll
-        for (int e = 0; e < S3; ++e) d1 = __fadd_rn(d1, __fmul_rn(gc[x * S3 + e], w2c[x * S3 + e]));
-        float *p = b.dw1 + (size_t)row * S2 + x;
-        *p = b.accumulate ? *p + d1 : d1;
+        for (int e = 0; e < S3; ++e) acc = __fadd_rn(acc, __fmul_rn(gc[x * S3 + e], w2c[x * S3 + e]));
+        d1[x] = acc;
 #pragma unroll
         for (int e = 0; e < S3; ++e)
-            if (gc[x * S3 + e] != 0.0f) atomicAdd(b.dw2 + r2[x] + e, __fmul_rn(gc[x * S3 + e], w1[x]));
+            if (gc[x * S3 + e] != 0.0f) atomicAdd(dleg + r2[x] + e, __fmul_rn(gc[x * S3 + e], w1[x]));
+    }
+    if constexpr (SF > 0) {
+#pragma unroll
+        for (int f = 0; f < SF; ++f) gf[f] = gc[NP2 + f];
+    }
+}
+
+// The same backward as ser_bwd_kernel, one thread per edge row, for small exact budgets (S2,
+// S3; s1 <= S1M), through refer_thread_backward: the referral is recomputed in registers
+// exactly as the fused forward's per-thread referral (same products, pairwise merge in
+// ascending candidate order, selection by weight then target), and the gradients flow as in
+// the warp kernel. It spends a fraction of the warp-per-row kernel's instructions when the
+// budgets are 2 or 4.
+//
+// The dispatch picks this kernel or ser_bwd_kernel by shape and alignment alone, so the two
+// must agree bit for bit: the candidate products (__fmul_rn), the merge in ascending candidate
+// order (merge_pairs here and refer_thread in gm_fused_tile.cuh; __match_any_sync groups
+// summed from their first lane in refer_merge), the selection (weight descending, then target
+// ascending, zero weights never kept), g / W for a log-weight gradient, and the first-leg sums
+// (g * w2 rounded, then added in ascending e). Only dw2, summed by atomics, varies in order.
+template <int S2, int S3, int S1M, int WPB, int SF = 0>
+__global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
+{
+    const SerArgs &a = b.f;
+    const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
+    if (row >= a.rows) return;  // no warp-wide operation below
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    int32_t j[S2];
+    float w1[S2];
+    ld_vec<S2>(a.a1_idx + (size_t)row * S2, j);
+    ld_vec<S2>(a.a1_w + (size_t)row * S2, w1);
+    float g[S1M];
+#pragma unroll
+    for (int r = 0; r < S1M; ++r) g[r] = r < a.s1 ? __ldg(b.gout + (size_t)row * a.s1 + r) : 0.0f;
+    float d1[S2], gf[SF > 0 ? SF : 1];
+    refer_thread_backward<S2, S3, S1M, SF>(a, row, seq_base, h, j, w1, a.a2_idx, a.a2_w, a.s1, g,
+                                           b.grad_is_log != 0, b.dw2, d1, gf);
+#pragma unroll
+    for (int x = 0; x < S2; ++x) {
+        float *p = b.dw1 + (size_t)row * S2 + x;
+        *p = b.accumulate ? *p + d1[x] : d1[x];
     }
     if constexpr (SF > 0) {  // refresh slots: d W / d w_f = 1
 #pragma unroll
         for (int f = 0; f < SF; ++f) {
             float *p = b.dfw + (size_t)row * SF + f;
-            *p = b.accumulate ? *p + gc[NP2 + f] : gc[NP2 + f];
+            *p = b.accumulate ? *p + gf[f] : gf[f];
         }
     }
 }

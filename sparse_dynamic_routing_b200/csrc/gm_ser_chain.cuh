@@ -12,7 +12,9 @@
 // One warp per edge row. The backward recomputes the chain, keeping each step's first leg in
 // registers, then runs the steps in reverse: each step's first-leg gradient (summed in a
 // fixed order) is the upstream gradient of the previous step's kept weights, and each leg's
-// gradient is scatter-added with fp32 atomics.
+// gradient is scatter-added with fp32 atomics. For budgets s2 = s3 = s_mid of 2 or 4 the
+// backward also runs one thread per row (ser_chain_bwd_thread_kernel), with the same results
+// (the per-thread referral steps agree bit for bit with the warp ones).
 #pragma once
 
 #include "gm_common.cuh"
@@ -122,6 +124,49 @@ __global__ void __launch_bounds__(WPB * 32) ser_chain_bwd_kernel(ChainBwdArgs b)
     if (lane < a.s2) {
         float *p = b.dw1 + (size_t)row * a.s2 + lane;
         *p = b.accumulate ? *p + g_l : g_l;
+    }
+}
+
+// The chain backward one thread per edge row, for budgets S = s2 = s3 = s_mid in {2, 4} and
+// s1 <= 4: the chain is recomputed step by step with refer_thread (each step's first leg kept
+// in registers), then refer_thread_backward runs the steps in reverse, the first-leg gradient
+// of step m being the upstream gradient of step m - 1's kept weights.
+template <int S, int NL, int WPB>
+__global__ void __launch_bounds__(WPB * 32) ser_chain_bwd_thread_kernel(ChainBwdArgs b)
+{
+    constexpr int S1M = 4;
+    const SerArgs &a = b.f;
+    const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
+    if (row >= a.rows) return;  // no warp-wide operation below
+    uint32_t seq_base, h;
+    a.map.split(row, seq_base, h);
+    int32_t jm[NL][S];
+    float wm[NL][S];
+    ld_vec<S>(a.a1_idx + (size_t)row * S, jm[0]);
+    ld_vec<S>(a.a1_w + (size_t)row * S, wm[0]);
+#pragma unroll
+    for (int m = 0; m + 1 < NL; ++m)
+        refer_thread<S, S, S>(a, row, seq_base, h, jm[m], wm[m], chain_leg_idx(a, m), chain_leg_w(a, m), S,
+                              jm[m + 1], wm[m + 1]);
+    float g1[S1M];
+#pragma unroll
+    for (int r = 0; r < S1M; ++r) g1[r] = r < a.s1 ? __ldg(b.gout + (size_t)row * a.s1 + r) : 0.0f;
+    float d1[S], unused[1];
+    refer_thread_backward<S, S, S1M>(a, row, seq_base, h, jm[NL - 1], wm[NL - 1], chain_leg_idx(a, NL - 1),
+                                     chain_leg_w(a, NL - 1), a.s1, g1, b.grad_is_log != 0, b.dleg[NL - 1],
+                                     d1, unused);
+#pragma unroll
+    for (int m = NL - 2; m >= 0; --m) {
+        float g[S];
+#pragma unroll
+        for (int x = 0; x < S; ++x) g[x] = d1[x];
+        refer_thread_backward<S, S, S>(a, row, seq_base, h, jm[m], wm[m], chain_leg_idx(a, m), chain_leg_w(a, m),
+                                       S, g, false, b.dleg[m], d1, unused);
+    }
+#pragma unroll
+    for (int x = 0; x < S; ++x) {
+        float *p = b.dw1 + (size_t)row * S + x;
+        *p = b.accumulate ? *p + d1[x] : d1[x];
     }
 }
 

@@ -62,9 +62,11 @@ def edges(rng, B, n, k, s, zero_frac=0.1):
     return idx, w
 
 
+# budgets s2 = s3 = s_mid in {2, 4} with s1 <= 4 and up to 4 legs run the per-thread backward
 @pytest.mark.parametrize("s2,s3,s_mid,s1,nlegs,n", [(2, 2, 2, 2, 2, 128), (4, 4, 4, 4, 3, 300),
                                                     (4, 4, 4, 2, 2, 97), (2, 3, 5, 4, 4, 61),
-                                                    (1, 2, 2, 3, 7, 45), (3, 3, 3, 3, 1, 40)])
+                                                    (1, 2, 2, 3, 7, 45), (3, 3, 3, 3, 1, 40),
+                                                    (2, 2, 2, 3, 4, 150), (4, 4, 4, 1, 1, 70)])
 def test_chain_forward_and_backward(s2, s3, s_mid, s1, nlegs, n):
     rng = np.random.default_rng(s2 * 1000 + s3 * 100 + s_mid * 10 + nlegs)
     B, k = 2, 3
@@ -163,4 +165,35 @@ def test_fused_chain_full_size_layer():
     assert_close(lse.reshape(wl.B * wl.n, wl.hq)[sel], lse_ref, 2e-2, "lse")
     ci, cw = gm.gm_ser_chain_forward(g["a1_idx"], g["a1_w"], g_legs, wl.s2, wl.s1)
     assert torch.equal(ci, ai) and torch.equal(cw, aw)
+    gm.gm_check_device_errors()
+
+
+def misaligned(a):
+    """`a` on the GPU at a data pointer 4 bytes past a 16-byte boundary (forces the warp kernels)."""
+    src = torch.from_numpy(np.ascontiguousarray(a))
+    flat = torch.empty(src.numel() + 4, dtype=src.dtype, device="cuda")
+    view = flat[1:1 + src.numel()].view(src.shape)
+    view.copy_(src)
+    assert view.data_ptr() % 16 == 4
+    return view
+
+
+@pytest.mark.parametrize("s,nlegs", [(2, 2), (4, 2), (4, 3)])
+def test_chain_backward_thread_and_warp_agree(s, nlegs):
+    """The per-thread and warp-per-row chain backwards are picked by shape and alignment
+    alone: the first-leg gradient must match bit for bit (leg gradients: fp32 atomics)."""
+    rng = np.random.default_rng(40 + s * 10 + nlegs)
+    B, n, k = 1, 160, 2
+    a1 = edges(rng, B, n, k, s)
+    legs = [edges(rng, B, n, k, s) for _ in range(nlegs)]
+    g = rng.standard_normal((B, n, k, 4)).astype(np.float32)
+    thread = gm.gm_ser_chain_backward(t(a1[0]), t(a1[1]), [(t(i), t(w)) for i, w in legs], s, t(g))
+    warp = gm.gm_ser_chain_backward(misaligned(a1[0]), misaligned(a1[1]),
+                                    [(misaligned(i), misaligned(w)) for i, w in legs], s, t(g))
+    np.testing.assert_array_equal(thread[0].cpu().numpy().view(np.uint32),
+                                  warp[0].cpu().numpy().view(np.uint32))
+    for a, b in zip(thread[1], warp[1]):
+        ref = b.cpu().double().numpy()
+        err = np.abs(a.cpu().double().numpy() - ref).max()
+        assert err <= 1e-5 * max(np.abs(ref).max(), 1e-30)
     gm.gm_check_device_errors()
