@@ -459,7 +459,7 @@ template <typename T, int D, int G> struct SeaBwdGather {
                 rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
             if (rs != GM_OK) return rs;
             auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
-            const size_t smem = (size_t)WPB_GATHER * gm::gather_warp_bytes<G>(GATHER_U, GATHER_P);
+            const size_t smem = (size_t)WPB_GATHER * GATHER_P * GATHER_U * G * 32 * 16;
             if (smem > 48 * 1024 &&
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return GM_ERR_CUDA;

@@ -46,6 +46,23 @@ __device__ __forceinline__ void write_record(int32_t *srec, int32_t pos, uint32_
     for (int x = 0; x < Rec<G>::WORDS / 4; ++x) dst[x] = make_int4(w[4 * x], w[4 * x + 1], w[4 * x + 2], w[4 * x + 3]);
 }
 
+template <int G>
+__device__ __forceinline__ void read_record(const int32_t *srec, int64_t pos, int32_t &key, int32_t &row,
+                                            float (&cf)[2 * G])
+{
+    int32_t w[Rec<G>::WORDS];
+    const int4 *src = reinterpret_cast<const int4 *>(srec + pos * Rec<G>::WORDS);
+#pragma unroll
+    for (int x = 0; x < Rec<G>::WORDS / 4; ++x) {
+        const int4 v = __ldg(src + x);
+        w[4 * x] = v.x; w[4 * x + 1] = v.y; w[4 * x + 2] = v.z; w[4 * x + 3] = v.w;
+    }
+    key = w[0];
+    row = w[1];
+#pragma unroll
+    for (int x = 0; x < 2 * G; ++x) cf[x] = __int_as_float(w[2 + x]);
+}
+
 // Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges).
 struct GatherWs {
     int32_t *cnt;     // [R]      edges per target row (counted, then consumed by the row pass)
@@ -158,32 +175,21 @@ __global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, Row
 
 // Gather: one warp per chunk of 32 sorted records. Lanes [0, C) own dK chunk c, lanes
 // [C, 2C) dV chunk c (16 bytes of every feature row). Each lane stages exactly the q (or
-// dO) chunks it will read with cp.async, U records per group, P groups ahead. The window of
-// 32 records sits in shared memory, so every lane reads a record's target, source and
-// coefficients with two broadcast loads.
-template <int G> __host__ __device__ constexpr int gather_warp_bytes(int U, int P)
-{
-    return P * U * G * 32 * 16 + 32 * Rec<G>::WORDS * 4;
-}
-
+// dO) chunks it will read with cp.async, U records per group, P groups ahead.
 template <typename T, int D, int G, int WPB, int U, int P>
 __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q, const void *dout, float *dk, float *dv,
                                                                  GatherWs ws, uint32_t R, int accumulate)
 {
     constexpr int VEC = Vec<T>::N, C = D / VEC, NP = VEC / 2, ROW = D * (int)sizeof(T);
     constexpr int GROUP = U * G * 32 * 16;  // bytes of one group of records, all lanes
-    constexpr int WORDS = Rec<G>::WORDS;
     static_assert(2 * C <= 32, "dK and dV halves fit one warp");
-    constexpr int NW = WORDS / 4;  // 16-byte words per record
-    static_assert(2 * G <= 8, "coefficients of one record fit two 16-byte words");
+    static_assert(2 * G <= 8, "coefficients of one record fit two 16-byte loads");
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    char *ring = smem + (size_t)wid * gather_warp_bytes<G>(U, P);
-    const int4 *win = reinterpret_cast<const int4 *>(ring + P * GROUP);  // [32][NW] records
+    char *ring = smem + (size_t)wid * P * GROUP;
     const int role = lane / C, c = lane % C;
     const bool working = role < 2;
-    // this lane's chunk of source row 0 (head 0)
-    const char *src = static_cast<const char *>(role == 0 ? q : dout) + (size_t)c * 16;
+    const char *src = static_cast<const char *>(role == 0 ? q : dout);
     float *dst_base = (role == 0 ? dk : dv) + c * VEC;
 
     const int total = ws.off[R];
@@ -223,22 +229,17 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
     }
     if (p0 >= total) return;  // warp-uniform
 
-    // the chunk's records (window [wbase, wbase + 32) of the sorted list, one per lane, then
-    // staged in shared memory for broadcast reads)
+    // the chunk's records (window [wbase, wbase + 32) of the sorted list, one per lane)
     int64_t wbase = p0;
     int wlen = (int)min((int64_t)32, (int64_t)total - wbase);
-    int32_t mkey = -1;
+    int32_t mkey = -1, mrow = 0;
+    float mcf[2 * G];
     auto load_window = [&]() {
-        __syncwarp();  // the previous window's broadcast reads are done
-        int4 *dw = const_cast<int4 *>(win) + NW * lane;
-        const int4 *srcw = reinterpret_cast<const int4 *>(ws.srec + (wbase + lane) * WORDS);
+        mkey = -1;
+        mrow = 0;
 #pragma unroll
-        for (int x = 0; x < NW; ++x) {
-            const int4 w = lane < wlen ? __ldg(srcw + x) : make_int4(x == 0 ? -1 : 0, 0, 0, 0);
-            dw[x] = w;
-            if (x == 0) mkey = w.x;
-        }
-        __syncwarp();
+        for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
+        if (lane < wlen) read_record<G>(ws.srec, wbase + lane, mkey, mrow, mcf);
     };
     load_window();
     const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
@@ -257,12 +258,12 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int k = lo + grp * U + u;
+                const int32_t row = __shfl_sync(FULL, mrow, k & 31);
                 if (k < hi && working) {
-                    const uint32_t row = (uint32_t)win[NW * k].y;
                     char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
-                    const char *rsrc = src + (size_t)row * (G * ROW);
 #pragma unroll
-                    for (int g = 0; g < G; ++g) cp_async16(slot + g * 32 * 16, rsrc + g * ROW);
+                    for (int g = 0; g < G; ++g)
+                        cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
                 }
             }
             cp_async_commit();
@@ -275,18 +276,11 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const int k = lo + grp * U + u;
-                if (k >= hi) break;  // warp-uniform
-                int32_t w[WORDS];
-#pragma unroll
-                for (int x = 0; x < NW; ++x) {
-                    const int4 v = win[NW * k + x];
-                    w[4 * x] = v.x; w[4 * x + 1] = v.y; w[4 * x + 2] = v.z; w[4 * x + 3] = v.w;
-                }
-                const uint32_t key = (uint32_t)w[0];
-                // coefficients: scale dz_g (g < G) then p_g, from word 2 of the record
+                const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
                 float cf[2 * G];
 #pragma unroll
-                for (int x = 0; x < 2 * G; ++x) cf[x] = __int_as_float(w[2 + x]);
+                for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
+                if (k >= hi) break;  // warp-uniform
                 if (key != cur) {    // warp-uniform: a new target starts here
                     write_row(cur);
 #pragma unroll
