@@ -398,7 +398,7 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
  * gm_sea_backward_workspace_size - bytes of workspace gm_sea_backward needs for its gather
  * path on this shape, or 0 when the gather path does not cover it (then pass NULL). Covered:
  * s <= 4, head_dim 64 or 128 with hq/hkv <= 2 for GM_BF16, head_dim 64 with hq/hkv <= 4 for
- * GM_F32. The size grows as 8*(B*n*hkv) + 32*(B*n*hkv*s) bytes (hq/hkv <= 2) plus padding.
+ * GM_F32. The size grows as 8*(B*n*hkv) + 36*(B*n*hkv*s) bytes (hq/hkv <= 2) plus padding.
  * Pure host function; no CUDA call.
  */
 size_t gm_sea_backward_workspace_size(gm_dtype dtype, int s, int B, int n, int hq, int hkv, int d);
@@ -424,8 +424,8 @@ size_t gm_sea_backward_workspace_size(gm_dtype dtype, int s, int B, int n, int h
  *     two streams without ordering) race on it and give wrong results: serialise them.
  *   - Shapes the gather path does not cover (see gm_sea_backward_workspace_size) return
  *     GM_ERR_UNSUPPORTED; a covered shape whose scratch need exceeds the array returns
- *     GM_ERR_SCRATCH_TOO_SMALL (about 136 bytes per edge row at s = 4, hq/hkv = 2: up to
- *     ~240k rows B*n*hkv). Both are checked before anything is launched.
+ *     GM_ERR_SCRATCH_TOO_SMALL (about 152 bytes per edge row at s = 4, hq/hkv = 2: up to
+ *     ~220k rows B*n*hkv). Both are checked before anything is launched.
  * Results: as gm_sea_backward with a workspace.
  */
 gm_status gm_sea_backward_noalloc(const void *q, const void *k, const void *v, const void *dout,

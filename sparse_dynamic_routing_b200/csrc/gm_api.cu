@@ -366,7 +366,7 @@ gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
 {
     using TG = gm::BwdTileGeom<T, D, G, S1M>;
     auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE, GATHER, SB>;
-    const size_t smem = (size_t)WPB_BWD_TILE * (gm::bwd_tile_bytes<S1M, SB>() + BWD_TILE_P * TG::STAGE);
+    const size_t smem = (size_t)WPB_BWD_TILE * (gm::bwd_tile_bytes<S1M, SB, GATHER>() + BWD_TILE_P * TG::STAGE);
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return GM_ERR_CUDA;
@@ -412,7 +412,7 @@ bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
 }
 
 struct WsLayout {
-    size_t cnt, off, bsum, srec, total;
+    size_t cnt, off, bsum, rank, srec, total;
     uint32_t nblk;
 };
 
@@ -425,7 +425,8 @@ WsLayout ws_layout(int64_t R, int64_t E, int G)
     L.cnt = 0;
     L.off = L.cnt + up((size_t)R * 4);
     L.bsum = L.off + up((size_t)(R + 1) * 4);
-    L.srec = L.bsum + up((size_t)L.nblk * 4);
+    L.rank = L.bsum + up((size_t)L.nblk * 4);
+    L.srec = L.rank + up((size_t)E * 4);
     L.total = L.srec + up((size_t)E * words * 4);
     return L;
 }
@@ -442,12 +443,12 @@ template <typename T, int D, int G> struct SeaBwdGather {
             gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, R);
             const int64_t want = (E + 255) / 256;
             gm::edge_count_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
-                idx, w, a.n, a.map, sdiv, E, a.hkv, ws.cnt);
+                idx, w, a.n, a.map, sdiv, E, a.hkv, ws.cnt, ws.rank);
             gm::scan_block_sums_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum);
             gm::scan_block_offsets_kernel<<<1, gm::SCAN_THREADS, 0, st>>>(ws.bsum, ws.nblk, ws.off + R);
             gm::scan_apply_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum, ws.off);
             if (launched() != GM_OK) return GM_ERR_CUDA;
-            a.cnt = ws.cnt;
+            a.rank = ws.rank;
             a.off = ws.off;
             a.srec = ws.srec;
             gm_status rs;
@@ -1005,8 +1006,8 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
         const WsLayout L = ws_layout(rows, rows * s, hq / hkv);
         char *base = static_cast<char *>(workspace);
         const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.srec),
-                              L.nblk};
+                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.rank),
+                              reinterpret_cast<int32_t *>(base + L.srec), L.nblk};
         return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream);
     }
 
@@ -1086,8 +1087,8 @@ gm_status gm_ser_sea_backward(const void *q, const void *k, const void *v, const
     const WsLayout L = ws_layout(rows, rows * s1, hq / hkv);
     char *base = static_cast<char *>(workspace);
     const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                          reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.srec),
-                          L.nblk};
+                          reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.rank),
+                          reinterpret_cast<int32_t *>(base + L.srec), L.nblk};
     return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream, s2);
 }
 

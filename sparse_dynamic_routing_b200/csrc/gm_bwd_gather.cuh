@@ -4,18 +4,19 @@
 // of the attention in "Graph Machine: Towards Better Pretraining via Edges", ai.info summary,
 // "Key Contributions" item 3) is done as a gather over edges sorted by target instead of as
 // fp32 read-modify-write atomics on the gradient rows:
-//   1. a count pass counts the active edges of every target row (b, t, h) (integer atomics);
+//   1. a count pass counts the active edges of every target row (b, t, h) with integer
+//      atomics, and keeps each edge's rank inside its target (the value its atomic returned);
 //   2. an exclusive scan of the counts gives each target row its bucket [off[r], off[r+1]);
 //   3. the row pass (sea_bwd_tile_kernel with GATHER = true) stores dq and d ln w as usual and
 //      writes, for every active edge, a record (target row, source row, scale dz_g and p_g
-//      over the group's query heads g) straight into its target's bucket;
+//      over the group's query heads g) straight to off[target] + rank of its edge;
 //   4. the gather pass walks the sorted records in chunks of 32, one warp per chunk: a warp
 //      owns every target whose first record lies in its chunk (following it past the chunk
 //      end if needed), sums scale dz_g q_g into dK and p_g dO_g into dV, and writes each owned
 //      row once; the target rows nothing points at are written as zeros by the owner of the
 //      next non-empty target (or of the last one).
-// The order of records inside a bucket comes from integer atomics and varies run to run, so
-// dK/dV sums vary in rounding order (not in the set of terms). There are no spin-waits: the
+// The order of records inside a bucket comes from the count pass's integer atomics and
+// varies run to run, so dK/dV sums vary in rounding order (not in the set of terms). There are no spin-waits: the
 // scan is reduce -> scan of block totals -> rescan, three launches.
 #pragma once
 
@@ -65,9 +66,10 @@ __device__ __forceinline__ void read_record(const int32_t *srec, int64_t pos, in
 
 // Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges).
 struct GatherWs {
-    int32_t *cnt;     // [R]      edges per target row (counted, then consumed by the row pass)
+    int32_t *cnt;     // [R]      edges per target row
     int32_t *off;     // [R + 1]  bucket offsets; off[R] = number of active edges
     int32_t *bsum;    // [nblk]   scan block totals, then their offsets
+    int32_t *rank;    // [E]      an active edge's place inside its target's bucket
     int32_t *srec;    // [E * Rec<G>::WORDS] records sorted by target row
     uint32_t nblk;    // scan blocks of SCAN_TILE rows
 };
@@ -158,9 +160,10 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_apply_kernel(const int32_t 
     }
 }
 
-// Count: active edges per target row (range errors are reported by the row pass).
+// Count: active edges per target row, and each active edge's rank among them (range errors
+// are reported by the row pass, which applies the same activity test).
 __global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, RowMap map, FastDiv sdiv,
-                                  int64_t E, int hkv, int32_t *cnt)
+                                  int64_t E, int hkv, int32_t *cnt, int32_t *rank)
 {
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < E; e += (int64_t)gridDim.x * blockDim.x) {
         const float we = w[e];
@@ -169,7 +172,7 @@ __global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, Row
         const uint32_t row = sdiv.div((uint32_t)e);
         uint32_t seq_base, h;
         map.split(row, seq_base, h);
-        atomicAdd(cnt + (seq_base + (uint32_t)t) * (uint32_t)hkv + h, 1);
+        rank[e] = atomicAdd(cnt + (seq_base + (uint32_t)t) * (uint32_t)hkv + h, 1);
     }
 }
 

@@ -45,11 +45,11 @@ template <typename T, int D, int G, int S1M> struct BwdTileGeom {
 #endif
 
 // Shared memory per warp of the tile row pass: the edge tile (K/V row, log2 w per slot), with
-// the fused referral backward (SB > 0) also each slot's target, weight and d ln w, then the
-// P stages.
-template <int S1M, int SB> __host__ __device__ constexpr int bwd_tile_bytes()
+// the fused referral backward (SB > 0) also each slot's target, weight and d ln w, in gather
+// mode each slot's record position; then the P stages.
+template <int S1M, int SB, bool GATHER> __host__ __device__ constexpr int bwd_tile_bytes()
 {
-    return 32 * S1M * (SB > 0 ? 20 : 8);
+    return 32 * S1M * ((SB > 0 ? 20 : 8) + (GATHER ? 4 : 0));
 }
 
 // Referral backward of one edge row by one thread, fused after the attention backward of its
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    constexpr int TILE_BYTES = bwd_tile_bytes<S1M, SB>();
+    constexpr int TILE_BYTES = bwd_tile_bytes<S1M, SB, GATHER>();
     char *wbase = smem + (size_t)wid * (TILE_BYTES + P * TG::STAGE);
     int32_t *tile_t = reinterpret_cast<int32_t *>(wbase);
     float *tile_lw = reinterpret_cast<float *>(wbase + 32 * S1M * 4);
@@ -124,6 +124,8 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
     int32_t *tile_tt = reinterpret_cast<int32_t *>(wbase + 32 * S1M * 8);
     float *tile_w = reinterpret_cast<float *>(wbase + 32 * S1M * 12);
     float *tile_g = reinterpret_cast<float *>(wbase + 32 * S1M * 16);
+    // gather mode: where each active slot's record goes (off[target] + the edge's rank)
+    int32_t *tile_pos = reinterpret_cast<int32_t *>(wbase + 32 * S1M * (SB > 0 ? 20 : 8));
     char *stages = wbase + TILE_BYTES;
 
     const uint32_t rows = a.rows;
@@ -161,8 +163,12 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                         }
                     }
                 }
-                tile_t[lane * S1M + r] = (int32_t)((seq_base + (uint32_t)t) * (uint32_t)a.hkv + h);
+                const uint32_t key = (seq_base + (uint32_t)t) * (uint32_t)a.hkv + h;
+                tile_t[lane * S1M + r] = (int32_t)key;
                 tile_lw[lane * S1M + r] = lw;
+                if constexpr (GATHER)  // the count pass applied the same activity test
+                    tile_pos[lane * S1M + r] =
+                        lw != -INFINITY ? __ldg(a.off + key) + __ldg(a.rank + (size_t)row * a.s + r) : -1;
                 if constexpr (SB > 0) {
                     tile_tt[lane * S1M + r] = t;
                     tile_w[lane * S1M + r] = lw == -INFINITY ? 0.0f : __ldg(a.w + (size_t)row * a.s + r);
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 }
                 if (c < S1M && mine) {
                     const uint32_t key = (uint32_t)tile_t[lr * S1M + c];
-                    const int32_t pos = a.off[key] + atomicSub(a.cnt + key, 1) - 1;
+                    const int32_t pos = tile_pos[lr * S1M + c];
                     // the count pass applies the same activity test, so pos stays inside the
                     // bucket; the bound only keeps a broken invariant from writing outside
                     if ((uint32_t)pos < a.rows * (uint32_t)a.s) write_record<G>(a.srec, pos, key, row, rc);

@@ -30,9 +30,9 @@ struct SeaBwdArgs {
     const int32_t *idx;
     const float *w;
     float *dq, *dk, *dv, *dlogw;
-    // gather mode only (see gm_bwd_gather.cuh): target counts (consumed), bucket offsets, and
-    // the sorted record arrays; unused by the atomic path
-    int32_t *cnt;
+    // gather mode only (see gm_bwd_gather.cuh): each edge's rank inside its target's bucket,
+    // the bucket offsets, and the sorted record array; unused by the atomic path
+    const int32_t *rank;
     const int32_t *off;
     int32_t *srec;
     int s, n, hkv;
