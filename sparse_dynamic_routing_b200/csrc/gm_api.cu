@@ -412,10 +412,11 @@ bool gather_supported(gm_dtype dtype, int d, int G, int s, int64_t E)
 }
 
 struct WsLayout {
-    size_t cnt, off, bsum, rank, srec, total;
+    size_t cnt, state, ticket, off, rank, srec, total;
     uint32_t nblk;
 };
 
+// [cnt | scan tile words | ticket] (cleared at every call) [off] [rank] [records]
 WsLayout ws_layout(int64_t R, int64_t E, int G)
 {
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -423,12 +424,26 @@ WsLayout ws_layout(int64_t R, int64_t E, int G)
     WsLayout L;
     L.nblk = (uint32_t)((R + gm::SCAN_TILE - 1) / gm::SCAN_TILE);
     L.cnt = 0;
-    L.off = L.cnt + up((size_t)R * 4);
-    L.bsum = L.off + up((size_t)(R + 1) * 4);
-    L.rank = L.bsum + up((size_t)L.nblk * 4);
+    L.state = L.cnt + up((size_t)R * 4);
+    L.ticket = L.state + (size_t)L.nblk * 8;
+    L.off = L.state + up((size_t)L.nblk * 8 + 8);
+    L.rank = L.off + up((size_t)(R + 1) * 4);
     L.srec = L.rank + up((size_t)E * 4);
     L.total = L.srec + up((size_t)E * words * 4);
     return L;
+}
+
+gm::GatherWs gather_ws(void *workspace, const WsLayout &L)
+{
+    char *base = static_cast<char *>(workspace);
+    return gm::GatherWs{reinterpret_cast<int32_t *>(base + L.cnt),
+                        reinterpret_cast<unsigned long long *>(base + L.state),
+                        reinterpret_cast<uint32_t *>(base + L.ticket),
+                        reinterpret_cast<int32_t *>(base + L.off),
+                        reinterpret_cast<int32_t *>(base + L.rank),
+                        reinterpret_cast<int32_t *>(base + L.srec),
+                        L.nblk,
+                        (int64_t)(L.off / 4)};
 }
 
 template <typename T, int D, int G> struct SeaBwdGather {
@@ -439,14 +454,13 @@ template <typename T, int D, int G> struct SeaBwdGather {
     {
         if constexpr (TileOK<T, D, G>::value && 2 * (D / gm::Vec<T>::N) <= 32 && 2 * G <= 8) {
             const int64_t R = a.rows, E = R * a.s;
-            const gm::FastDiv sdiv((uint32_t)a.s);
-            gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, R);
-            const int64_t want = (E + 255) / 256;
-            gm::edge_count_kernel<<<(unsigned)(want < 148 * 16 ? want : 148 * 16), 256, 0, st>>>(
-                idx, w, a.n, a.map, sdiv, E, a.hkv, ws.cnt, ws.rank);
-            gm::scan_block_sums_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum);
-            gm::scan_block_offsets_kernel<<<1, gm::SCAN_THREADS, 0, st>>>(ws.bsum, ws.nblk, ws.off + R);
-            gm::scan_apply_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.bsum, ws.off);
+            gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, ws.zero_words);
+            const unsigned cgrid = (unsigned)((R + 255) / 256);
+            if (a.s <= 2)
+                gm::edge_count_kernel<2><<<cgrid, 256, 0, st>>>(idx, w, a.n, a.map, a.s, a.rows, a.hkv, ws.cnt, ws.rank);
+            else
+                gm::edge_count_kernel<4><<<cgrid, 256, 0, st>>>(idx, w, a.n, a.map, a.s, a.rows, a.hkv, ws.cnt, ws.rank);
+            gm::scan_lookback_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.state, ws.ticket, ws.off);
             if (launched() != GM_OK) return GM_ERR_CUDA;
             a.rank = ws.rank;
             a.off = ws.off;
@@ -1004,10 +1018,7 @@ gm_status gm_sea_backward(const void *q, const void *k, const void *v, const voi
     if (workspace != nullptr && need > 0) {
         if (workspace_bytes < need || !aligned16(workspace)) return GM_ERR_INVALID_ARG;
         const WsLayout L = ws_layout(rows, rows * s, hq / hkv);
-        char *base = static_cast<char *>(workspace);
-        const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                              reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.rank),
-                              reinterpret_cast<int32_t *>(base + L.srec), L.nblk};
+        const gm::GatherWs ws = gather_ws(workspace, L);
         return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream);
     }
 
@@ -1085,10 +1096,7 @@ gm_status gm_ser_sea_backward(const void *q, const void *k, const void *v, const
                  s1, n, hkv, scale, accumulate, (uint32_t)rows, row_map(hkv, n),
                  a1_idx, a2_idx, a1_w, a2_w, dw1, dw2};
     const WsLayout L = ws_layout(rows, rows * s1, hq / hkv);
-    char *base = static_cast<char *>(workspace);
-    const gm::GatherWs ws{reinterpret_cast<int32_t *>(base + L.cnt), reinterpret_cast<int32_t *>(base + L.off),
-                          reinterpret_cast<int32_t *>(base + L.bsum), reinterpret_cast<int32_t *>(base + L.rank),
-                          reinterpret_cast<int32_t *>(base + L.srec), L.nblk};
+    const gm::GatherWs ws = gather_ws(workspace, L);
     return dispatch<SeaBwdGather>(dtype, d, hq / hkv, a, ws, idx, w, stream, s2);
 }
 

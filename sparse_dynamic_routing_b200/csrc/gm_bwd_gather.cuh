@@ -16,8 +16,8 @@
 //      row once; the target rows nothing points at are written as zeros by the owner of the
 //      next non-empty target (or of the last one).
 // The order of records inside a bucket comes from the count pass's integer atomics and
-// varies run to run, so dK/dV sums vary in rounding order (not in the set of terms). There are no spin-waits: the
-// scan is reduce -> scan of block totals -> rescan, three launches.
+// varies run to run, so dK/dV sums vary in rounding order (not in the set of terms). The scan
+// is one launch with a decoupled look-back between its blocks; its waits are bounded.
 #pragma once
 
 #include "gm_common.cuh"
@@ -64,14 +64,17 @@ __device__ __forceinline__ void read_record(const int32_t *srec, int64_t pos, in
     for (int x = 0; x < 2 * G; ++x) cf[x] = __int_as_float(w[2 + x]);
 }
 
-// Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges).
+// Caller-provided scratch (sizes in elements; R = B*n*hkv target rows, E = R*s edges). cnt,
+// state and ticket are contiguous, the first zero_words int32 words, cleared at every call.
 struct GatherWs {
-    int32_t *cnt;     // [R]      edges per target row
-    int32_t *off;     // [R + 1]  bucket offsets; off[R] = number of active edges
-    int32_t *bsum;    // [nblk]   scan block totals, then their offsets
-    int32_t *rank;    // [E]      an active edge's place inside its target's bucket
-    int32_t *srec;    // [E * Rec<G>::WORDS] records sorted by target row
-    uint32_t nblk;    // scan blocks of SCAN_TILE rows
+    int32_t *cnt;               // [R]      edges per target row
+    unsigned long long *state;  // [nblk]   scan tile words: status << 32 | value
+    uint32_t *ticket;           //          scan tiles taken so far
+    int32_t *off;               // [R + 1]  bucket offsets; off[R] = number of active edges
+    int32_t *rank;              // [E]      an active edge's place inside its target's bucket
+    int32_t *srec;              // [E * Rec<G>::WORDS] records sorted by target row
+    uint32_t nblk;              // scan tiles of SCAN_TILE rows
+    int64_t zero_words;
 };
 
 constexpr int SCAN_THREADS = 1024;
@@ -113,66 +116,111 @@ __device__ __forceinline__ int32_t block_exclusive_scan(int32_t v, int32_t &tota
     return before + incl - v;
 }
 
-// Scan step 1: totals of SCAN_TILE-row blocks of the counts.
-__global__ void __launch_bounds__(SCAN_THREADS) scan_block_sums_kernel(const int32_t *cnt, int64_t R, int32_t *bsum)
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v)
 {
-    const int64_t base = (int64_t)blockIdx.x * SCAN_TILE + (int64_t)threadIdx.x * SCAN_PER_THREAD;
-    int32_t s = 0;
-#pragma unroll
-    for (int k = 0; k < SCAN_PER_THREAD; ++k)
-        if (base + k < R) s += cnt[base + k];
-    int32_t total;
-    block_exclusive_scan(s, total);
-    if (threadIdx.x == 0) bsum[blockIdx.x] = total;
+    asm volatile("st.release.gpu.global.b64 [%0], %1;\n" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];\n" : "=l"(v) : "l"(p) : "memory");
+    return v;
 }
 
-// Scan step 2 (one block): exclusive scan of the block totals in place; off[R] = grand total.
-__global__ void __launch_bounds__(SCAN_THREADS) scan_block_offsets_kernel(int32_t *bsum, uint32_t nblk, int32_t *off_end)
-{
-    int32_t carry = 0;
-    for (uint32_t base = 0; base < nblk; base += SCAN_THREADS) {
-        const uint32_t i = base + threadIdx.x;
-        const int32_t v = i < nblk ? bsum[i] : 0;
-        int32_t total;
-        const int32_t ex = block_exclusive_scan(v, total);
-        if (i < nblk) bsum[i] = carry + ex;
-        carry += total;
-    }
-    if (threadIdx.x == 0) *off_end = carry;
-}
+constexpr unsigned long long SCAN_AGGREGATE = 1ull << 32, SCAN_PREFIX = 2ull << 32;
 
-// Scan step 3: off[r] = block offset + exclusive prefix inside the block.
-__global__ void __launch_bounds__(SCAN_THREADS) scan_apply_kernel(const int32_t *cnt, int64_t R, const int32_t *bsum, int32_t *off)
+// Exclusive scan of the counts into off, in one launch (single-pass scan with decoupled
+// look-back; Merrill and Garland, "Single-pass Parallel Prefix Scan with Decoupled Look-back",
+// 2016). A block takes the next tile from a ticket, scans its SCAN_TILE counts, publishes the
+// tile total at once and the inclusive prefix when it knows it; its prefix is the sum of the
+// totals of the tiles before it back to the nearest published prefix. A tile only waits on
+// tiles with earlier tickets, whose blocks are running or done, so the wait ends; it is still
+// bounded (WAIT_LIMIT_NS, then ERR_WAIT_TIMEOUT and a wrong prefix instead of a hang).
+__global__ void __launch_bounds__(SCAN_THREADS) scan_lookback_kernel(const int32_t *cnt, int64_t R,
+                                                                     unsigned long long *state, uint32_t *ticket,
+                                                                     int32_t *off)
 {
-    const int64_t base = (int64_t)blockIdx.x * SCAN_TILE + (int64_t)threadIdx.x * SCAN_PER_THREAD;
-    int32_t c[SCAN_PER_THREAD], s = 0;
+    __shared__ uint32_t s_tile;
+    __shared__ int32_t s_prefix;
+    if (threadIdx.x == 0) s_tile = atomicAdd(ticket, 1u);
+    __syncthreads();
+    const uint32_t tile = s_tile;
+    const int64_t base = (int64_t)tile * SCAN_TILE + (int64_t)threadIdx.x * SCAN_PER_THREAD;
+    int32_t c[SCAN_PER_THREAD], sum = 0;
 #pragma unroll
     for (int k = 0; k < SCAN_PER_THREAD; ++k) {
         c[k] = base + k < R ? cnt[base + k] : 0;
-        s += c[k];
+        sum += c[k];
     }
     int32_t total;
-    int32_t run = bsum[blockIdx.x] + block_exclusive_scan(s, total);
+    const int32_t ex = block_exclusive_scan(sum, total);
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int32_t prefix = 0;
+        if (tile == 0) {
+            if (lane == 0) st_release_u64(state, SCAN_PREFIX | (uint32_t)total);
+        } else {
+            if (lane == 0) st_release_u64(state + tile, SCAN_AGGREGATE | (uint32_t)total);
+            const unsigned long long t0 = globaltimer_ns();
+            bool late = false;
+            for (int64_t j = (int64_t)tile - 1;; j -= 32) {
+                // lane L reads tile j - L; tiles before 0 count as a zero prefix
+                const int64_t mine = j - lane;
+                unsigned long long st = mine >= 0 ? ld_acquire_u64(state + mine) : SCAN_PREFIX;
+                while (true) {  // every exit is warp-uniform
+                    const bool pending = (st >> 32) == 0;
+                    if (!__any_sync(FULL, pending)) break;
+                    if (__any_sync(FULL, globaltimer_ns() - t0 > WAIT_LIMIT_NS)) {
+                        late = true;
+                        break;
+                    }
+                    if (pending) st = ld_acquire_u64(state + mine);
+                }
+                if (late) break;
+                const unsigned pre = __ballot_sync(FULL, st >= SCAN_PREFIX);
+                const int stop = pre ? __ffs(pre) - 1 : 31;  // nearest published prefix
+                int32_t v = lane <= stop ? (int32_t)(uint32_t)st : 0;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(FULL, v, o);
+                prefix += v;
+                if (pre) break;
+            }
+            if (late && lane == 0) atomicOr(&g_error_flag, ERR_WAIT_TIMEOUT);
+            if (lane == 0) st_release_u64(state + tile, SCAN_PREFIX | (uint32_t)(prefix + total));
+        }
+        if (lane == 0) s_prefix = prefix;
+    }
+    __syncthreads();
+    int32_t run = s_prefix + ex;
 #pragma unroll
     for (int k = 0; k < SCAN_PER_THREAD; ++k) {
         if (base + k < R) off[base + k] = run;
         run += c[k];
     }
+    if (tile == gridDim.x - 1 && threadIdx.x == 0) off[R] = s_prefix + total;
 }
 
 // Count: active edges per target row, and each active edge's rank among them (range errors
-// are reported by the row pass, which applies the same activity test).
-__global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, RowMap map, FastDiv sdiv,
-                                  int64_t E, int hkv, int32_t *cnt, int32_t *rank)
+// are reported by the row pass, which applies the same activity test). One thread per edge
+// row: its slots' atomics are independent and in flight together.
+template <int S1M>
+__global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, RowMap map, int s, uint32_t rows,
+                                 int hkv, int32_t *cnt, int32_t *rank)
 {
-    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < E; e += (int64_t)gridDim.x * blockDim.x) {
-        const float we = w[e];
-        const int32_t t = idx[e];
-        if (!(we > 0.0f) || t < 0 || t >= n) continue;
-        const uint32_t row = sdiv.div((uint32_t)e);
+    for (uint32_t row = blockIdx.x * blockDim.x + threadIdx.x; row < rows; row += gridDim.x * blockDim.x) {
         uint32_t seq_base, h;
         map.split(row, seq_base, h);
-        rank[e] = atomicAdd(cnt + (seq_base + (uint32_t)t) * (uint32_t)hkv + h, 1);
+        int32_t t[S1M];
+        float we[S1M];
+#pragma unroll
+        for (int r = 0; r < S1M; ++r) {
+            we[r] = r < s ? __ldg(w + (size_t)row * s + r) : 0.0f;
+            t[r] = r < s ? __ldg(idx + (size_t)row * s + r) : 0;
+        }
+#pragma unroll
+        for (int r = 0; r < S1M; ++r)
+            if (we[r] > 0.0f && (uint32_t)t[r] < (uint32_t)n)
+                rank[(size_t)row * s + r] = atomicAdd(cnt + (seq_base + (uint32_t)t[r]) * (uint32_t)hkv + h, 1);
     }
 }
 
