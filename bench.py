@@ -3,8 +3,8 @@
 
 One step = one pass of the whole hot path over one batch of synthetic input:
   1. gm_ser_sea_forward  - SER (two-hop referral, merge, top-s1) fused with SEA forward,
-  2. gm_sea_backward     - zero-fill of dK/dV, then the SEA backward (dq, dK/dV scatter-add,
-                           d ln w) on the refreshed edges with upstream gradient dO.
+  2. gm_sea_backward     - the SEA backward (dq, dK/dV, d ln w) on the refreshed edges with
+                           upstream gradient dO: edge count, scan, row pass, per-target gather.
 Metric: tokens/s per sparse layer (B*n tokens per step / step time), summed over ranks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
@@ -67,6 +67,13 @@ def parse_args(argv=None):
                    help="skip the other workloads (s = 2 layer, 21-layer stack, n = 32768 step)")
     p.add_argument("--profile-call", default=None, choices=["dense_refresh"],
                    help="run only this call, warmup + steps times, for a profiler; print nothing")
+    p.add_argument("--write-traffic", default=None, metavar="CSV",
+                   help="write profiles/dram_traffic.txt from an ncu --csv log of dram__bytes_read.sum "
+                        "and dram__bytes_write.sum over a bench run (no GPU needed), then exit")
+    p.add_argument("--traffic-batch", type=int, default=None,
+                   help="batch size the --write-traffic capture ran at (traffic is scaled to the workload's)")
+    p.add_argument("--traffic-command", default="",
+                   help="the command line of the capture, recorded in the table")
     return p.parse_args(argv)
 
 
@@ -248,6 +255,62 @@ def ncu_traffic(kernel: str, workload: str):
                 return None
             return float(f["dram_bytes_per_launch"])
     return None
+
+
+# The kernels of each timed call, as ncu names them (one launch of each per call).
+TRAFFIC_CALLS = {
+    "sea_fwd_tile_kernel (fused SER->SEA)": ("sea_fwd_tile_kernel",),
+    "gm_sea_backward (count + scan + row pass + gather)": (
+        "zero_i32_kernel", "edge_count_kernel", "scan_lookback_kernel", "sea_bwd_tile_kernel",
+        "sea_bwd_gather_kernel"),
+}
+
+
+def write_traffic_table(csv_path: str, workload: str, capture_batch: int, command: str) -> str:
+    """profiles/dram_traffic.txt from ncu's per-launch DRAM byte counters: per kernel the median
+    over its launches, summed over the call's kernels, scaled from the captured batch to the
+    workload's (every kernel processes the B*n*hkv edge rows independently)."""
+    import csv
+    per = {}  # (launch id, kernel) -> bytes
+    with open(csv_path) as fh:
+        rows = [ln for ln in fh if ln.startswith('"')]
+    for r in csv.DictReader(rows):
+        if r["Metric Name"] not in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            continue
+        name = r["Kernel Name"].replace("void ", "").split("<")[0].split("(")[0].strip()
+        scale_unit = {"byte": 1, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}[r["Metric Unit"]]
+        key = (r["ID"], name)
+        per[key] = per.get(key, 0.0) + float(r["Metric Value"].replace(",", "")) * scale_unit
+    by_kernel = {}
+    for (_, name), b in per.items():
+        by_kernel.setdefault(name, []).append(b)
+    wl = I.WORKLOADS[workload]
+    scale = wl.B / capture_batch
+    lines = [
+        "# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the bench's timed",
+        f"# calls on {workload} (B={wl.B}), read by bench.py for the roofline's \"traffic\" field.",
+        f"# Written by `python bench.py --write-traffic <csv> --traffic-batch {capture_batch}` from one ncu",
+        f"# capture at B={capture_batch}, scaled by {scale:g}: every kernel processes the B*n*hkv edge rows",
+        "# independently. Per kernel the median over its launches; a call sums its kernels. DRAM write",
+        "# bytes count lines written back during the kernel: results still dirty in L2 at its end are",
+        "# not counted, so writes can read below the bytes a kernel stores.",
+        f"# Capture: {command}",
+        "# `source` is bench.py's hash of the kernel sources; when they change bench.py reports null.",
+    ]
+    src = source_hash()
+    for call, kernels in TRAFFIC_CALLS.items():
+        parts = {}
+        for k in kernels:
+            if k not in by_kernel:
+                raise SystemExit(f"{csv_path}: no DRAM counters for {k}")
+            parts[k] = statistics.median(by_kernel[k]) * scale
+        detail = ",".join(f"{k}:{int(v)}" for k, v in parts.items())
+        lines.append(f"kernel={call.replace(' ', '_')} workload={workload} "
+                     f"dram_bytes_per_launch={int(sum(parts.values()))} source={src} kernels={detail}")
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    with open(path, "w") as fh:
+        fh.write("\n".join(lines) + "\n")
+    return path
 
 
 def peak_hbm():
@@ -942,6 +1005,11 @@ def run_reference(args):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.write_traffic:
+        if not args.traffic_batch:
+            raise SystemExit("--write-traffic needs --traffic-batch")
+        print(write_traffic_table(args.write_traffic, args.workload, args.traffic_batch, args.traffic_command))
+        return
     if args.impl == "reference":
         res = run_reference(args)
     else:
