@@ -13,8 +13,8 @@
 //   4. the gather pass walks the sorted records in chunks of 32, one warp per chunk: a warp
 //      owns every target whose first record lies in its chunk (following it past the chunk
 //      end if needed), sums scale dz_g q_g into dK and p_g dO_g into dV, and writes each owned
-//      row once; the target rows nothing points at are written as zeros by the owner of the
-//      next non-empty target (or of the last one).
+//      row once; the target rows nothing points at (count 0) are written as zeros, each
+//      warp of the grid taking an equal slice of all target rows.
 // The order of records inside a bucket comes from the count pass's integer atomics and
 // varies run to run, so dK/dV sums vary in rounding order (not in the set of terms). The scan
 // is one launch with a decoupled look-back between its blocks; its waits are bounded.
@@ -264,115 +264,127 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
             *reinterpret_cast<float4 *>(dst + 2 * x) = o;
         }
     };
-    auto zero_rows = [&](int64_t from, int64_t to) {  // rows nothing points at: [from, to)
-        if (accumulate || !working) return;
+    // The rows nothing points at (count 0) are zeroed by slices, every warp of the grid taking
+    // an equal share of the rows whatever its chunk holds: long runs of empty targets (the late
+    // positions of a sequence under uniform causal edges) never fall on one warp.
+    auto zero_slice = [&]() {
+        if (accumulate) return;
+        const uint32_t nwarps = gridDim.x * WPB;
+        const uint32_t per = (R + nwarps - 1) / nwarps;
+        const uint32_t z0 = (uint32_t)chunk * per, z1 = min(z0 + per, R);
         const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int64_t t = from; t < to; ++t) {
-            float *dst = dst_base + (size_t)t * D;
+        for (uint32_t b0 = z0; b0 < z1; b0 += 32) {
+            const uint32_t t = b0 + lane;
+            unsigned empty = __ballot_sync(FULL, t < z1 && __ldg(ws.cnt + t) == 0);
+            while (empty) {  // warp-uniform
+                const uint32_t te = b0 + (uint32_t)(__ffs(empty) - 1);
+                empty &= empty - 1;
+                if (working) {
+                    float *dst = dst_base + (size_t)te * D;
 #pragma unroll
-            for (int x = 0; x < VEC; x += 4) *reinterpret_cast<float4 *>(dst + x) = z;
+                    for (int x = 0; x < VEC; x += 4) *reinterpret_cast<float4 *>(dst + x) = z;
+                }
+            }
         }
     };
 
-    if (total == 0) {  // no active edge anywhere: every row is zero, 32 rows per chunk
-        zero_rows(min(p0, (int64_t)R), min(p0 + 32, (int64_t)R));
-        return;
-    }
-    if (p0 >= total) return;  // warp-uniform
+    // the record walk; its early exits leave the zero slice to run after it
+    auto walk = [&]() {
+        if (p0 >= total) return;  // warp-uniform
 
-    // the chunk's records (window [wbase, wbase + 32) of the sorted list, one per lane)
-    int64_t wbase = p0;
-    int wlen = (int)min((int64_t)32, (int64_t)total - wbase);
-    int32_t mkey = -1, mrow = 0;
-    float mcf[2 * G];
-    auto load_window = [&]() {
-        mkey = -1;
-        mrow = 0;
-#pragma unroll
-        for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
-        if (lane < wlen) read_record<G>(ws.srec, wbase + lane, mkey, mrow, mcf);
-    };
-    load_window();
-    const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
-
-    // a leading run that continues the previous chunk's last target belongs to that chunk
-    const int start = __popc(__ballot_sync(FULL, lane < wlen && mkey == prev_key));
-    if (start == wlen) return;  // warp-uniform
-
-    uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, start);
-    zero_rows((int64_t)prev_key + 1, cur);
-
-    // Accumulate records [lo, hi) of the current window, U per copy group, P groups in
-    // flight; a change of key writes the finished target (and zeroes any empty rows between).
-    auto process = [&](int lo, int hi) {
-        auto issue = [&](int grp) {
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = lo + grp * U + u;
-                const int32_t row = __shfl_sync(FULL, mrow, k & 31);
-                if (k < hi && working) {
-                    char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-                        cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
-                }
-            }
-            cp_async_commit();
+        // the chunk's records (window [wbase, wbase + 32) of the sorted list, one per lane)
+        int64_t wbase = p0;
+        int wlen = (int)min((int64_t)32, (int64_t)total - wbase);
+        int32_t mkey = -1, mrow = 0;
+        float mcf[2 * G];
+        auto load_window = [&]() {
+            mkey = -1;
+            mrow = 0;
+    #pragma unroll
+            for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
+            if (lane < wlen) read_record<G>(ws.srec, wbase + lane, mkey, mrow, mcf);
         };
-        const int ngroups = (hi - lo + U - 1) / U;
-#pragma unroll
-        for (int grp = 0; grp < P; ++grp) issue(grp);
-        for (int grp = 0; grp < ngroups; ++grp) {
-            cp_async_wait<P - 1>();
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = lo + grp * U + u;
-                const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
-                float cf[2 * G];
-#pragma unroll
-                for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
-                if (k >= hi) break;  // warp-uniform
-                if (key != cur) {    // warp-uniform: a new target starts here
-                    write_row(cur);
-#pragma unroll
-                    for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
-                    zero_rows((int64_t)cur + 1, key);
-                    cur = key;
-                }
-                if (working) {
-                    const char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        float f[VEC];
-                        unpack<T>(*reinterpret_cast<const uint4 *>(slot + g * 32 * 16), f);
-                        const float k2 = role == 0 ? cf[g] : cf[G + g];
-                        const float2 kk = make_float2(k2, k2);
-#pragma unroll
-                        for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+        load_window();
+        const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
+
+        // a leading run that continues the previous chunk's last target belongs to that chunk
+        const int start = __popc(__ballot_sync(FULL, lane < wlen && mkey == prev_key));
+        if (start == wlen) return;  // warp-uniform
+
+        uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, start);
+
+        // Accumulate records [lo, hi) of the current window, U per copy group, P groups in
+        // flight; a change of key writes the finished target (and zeroes any empty rows between).
+        auto process = [&](int lo, int hi) {
+            auto issue = [&](int grp) {
+    #pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int k = lo + grp * U + u;
+                    const int32_t row = __shfl_sync(FULL, mrow, k & 31);
+                    if (k < hi && working) {
+                        char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
+    #pragma unroll
+                        for (int g = 0; g < G; ++g)
+                            cp_async16(slot + g * 32 * 16, src + ((size_t)row * G + g) * ROW + c * 16);
                     }
                 }
+                cp_async_commit();
+            };
+            const int ngroups = (hi - lo + U - 1) / U;
+    #pragma unroll
+            for (int grp = 0; grp < P; ++grp) issue(grp);
+            for (int grp = 0; grp < ngroups; ++grp) {
+                cp_async_wait<P - 1>();
+    #pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int k = lo + grp * U + u;
+                    const uint32_t key = (uint32_t)__shfl_sync(FULL, mkey, k & 31);
+                    float cf[2 * G];
+    #pragma unroll
+                    for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
+                    if (k >= hi) break;  // warp-uniform
+                    if (key != cur) {    // warp-uniform: a new target starts here
+                        write_row(cur);
+    #pragma unroll
+                        for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
+                        cur = key;
+                    }
+                    if (working) {
+                        const char *slot = ring + (grp % P) * GROUP + ((u * G) * 32 + lane) * 16;
+    #pragma unroll
+                        for (int g = 0; g < G; ++g) {
+                            float f[VEC];
+                            unpack<T>(*reinterpret_cast<const uint4 *>(slot + g * 32 * 16), f);
+                            const float k2 = role == 0 ? cf[g] : cf[G + g];
+                            const float2 kk = make_float2(k2, k2);
+    #pragma unroll
+                            for (int x = 0; x < NP; ++x) acc[x] = __ffma2_rn(kk, make_float2(f[2 * x], f[2 * x + 1]), acc[x]);
+                        }
+                    }
+                }
+                issue(grp + P);
             }
-            issue(grp + P);
-        }
-        cp_async_wait<0>();
-    };
+            cp_async_wait<0>();
+        };
 
-    process(start, wlen);
-    // the last owned target may continue past the chunk (hot rows): follow it window by
-    // window with the same pipeline
-    int64_t pos = wbase + wlen;
-    while (wlen == 32 && pos < total) {
-        wbase = pos;
-        wlen = (int)min((int64_t)32, (int64_t)total - wbase);
-        load_window();
-        const int run = __popc(__ballot_sync(FULL, lane < wlen && (uint32_t)mkey == cur));
-        if (run == 0) break;  // warp-uniform
-        process(0, run);
-        pos = wbase + run;
-        if (run < wlen) break;  // the target ended inside this window
-    }
-    write_row(cur);
-    if (pos >= total) zero_rows((int64_t)cur + 1, R);  // owner of the last target: trailing rows
+        process(start, wlen);
+        // the last owned target may continue past the chunk (hot rows): follow it window by
+        // window with the same pipeline
+        int64_t pos = wbase + wlen;
+        while (wlen == 32 && pos < total) {
+            wbase = pos;
+            wlen = (int)min((int64_t)32, (int64_t)total - wbase);
+            load_window();
+            const int run = __popc(__ballot_sync(FULL, lane < wlen && (uint32_t)mkey == cur));
+            if (run == 0) break;  // warp-uniform
+            process(0, run);
+            pos = wbase + run;
+            if (run < wlen) break;  // the target ended inside this window
+        }
+        write_row(cur);
+    };
+    walk();
+    zero_slice();
 }
 
 }  // namespace gm
