@@ -31,8 +31,9 @@
  * dereferenced. An active slot whose index lies outside [0, n) is treated as inactive and
  * raises the device error flag (see gm_check_device_errors); kernels never trap. Weights are
  * expected finite and >= 0; indices are expected causal (<= the row's own position); the
- * regular build does not check this, the checked build does (gm_checked_build). Position 0 of each sequence is the padding token: SER pads missing
- * output slots with (index 0, weight 0.0f).
+ * regular build does not check this, the checked build does (gm_checked_build). Position 0
+ * of each sequence is the padding token: SER pads missing output slots with (index 0,
+ * weight 0.0f).
  *
  * Ownership and synchrony. The caller allocates and owns every buffer. Entry points allocate
  * no device memory, enqueue their kernels on `stream` (0 = the legacy default stream) and
@@ -505,9 +506,10 @@ gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, c
  * flag. Returns GM_ERR_INDEX_RANGE if any kernel of this library on the current device met
  * an active slot whose index lay outside [0, n) since the last check, GM_ERR_EDGE_INVALID if
  * (checked build) an input edge broke the edge invariants (see gm_checked_build),
- * GM_ERR_WAIT_TIMEOUT if a
- * kernel gave up on a bounded wait for an asynchronous copy or tensor-core operation (its
- * outputs are then incomplete), GM_ERR_CUDA if the synchronisation failed, else GM_OK.
+ * GM_ERR_WAIT_TIMEOUT if a kernel gave up on a bounded wait (an asynchronous copy, a
+ * tensor-core operation, or the backward scan's look-back at earlier blocks; its outputs are
+ * then incomplete), GM_ERR_CUDA if the synchronisation failed, else GM_OK. When several
+ * occurred, the first of GM_ERR_WAIT_TIMEOUT, GM_ERR_EDGE_INVALID, GM_ERR_INDEX_RANGE.
  */
 gm_status gm_check_device_errors(cudaStream_t stream);
 

@@ -632,6 +632,19 @@ gm_status gm_ser_forward(const int32_t *a1_idx, const float *a1_w, int s2,
               (uint32_t)((int64_t)B * n * k), row_map(k, n)};
     check_edges(a1_idx, a1_w, s2, B, n, k, stream);
     check_edges(a2_idx, a2_w, s3, B, n, k, stream);
+    // one thread per row for budgets 2 or 4 (vector loads and stores need 16-byte alignment)
+    const bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w) &&
+                         aligned16(out_idx) && aligned16(out_w);
+    const unsigned tgrid = (unsigned)((a.rows + 127) / 128);
+    if (aligned && s2 == s3 && (s2 == 2 || s2 == 4) && s1 <= 4) {
+        if (s2 == 2)
+            s1 <= 2 ? gm::ser_thread_kernel<2, 2, 2><<<tgrid, 128, 0, stream>>>(a)
+                    : gm::ser_thread_kernel<2, 2, 4><<<tgrid, 128, 0, stream>>>(a);
+        else
+            s1 <= 2 ? gm::ser_thread_kernel<4, 4, 2><<<tgrid, 128, 0, stream>>>(a)
+                    : gm::ser_thread_kernel<4, 4, 4><<<tgrid, 128, 0, stream>>>(a);
+        return launched();
+    }
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
     return launched();
 }
@@ -754,6 +767,18 @@ gm_status gm_ser_refresh_forward(const int32_t *a1_idx, const float *a1_w, int s
     check_edges(a1_idx, a1_w, s2, B, n, k, stream);
     check_edges(a2_idx, a2_w, s3, B, n, k, stream);
     check_edges(f_idx, f_w, sf, B, n, k, stream);
+    const bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w) &&
+                         aligned16(f_idx) && aligned16(f_w) && aligned16(out_idx) && aligned16(out_w);
+    const unsigned tgrid = (unsigned)((a.rows + 127) / 128);
+    if (aligned && s2 == s3 && (s2 == 2 || s2 == 4) && s1 <= 4 && (sf == 2 || sf == 4)) {
+        if (s2 == 2)
+            sf == 2 ? gm::ser_thread_kernel<2, 2, 4, 2><<<tgrid, 128, 0, stream>>>(a)
+                    : gm::ser_thread_kernel<2, 2, 4, 4><<<tgrid, 128, 0, stream>>>(a);
+        else
+            sf == 2 ? gm::ser_thread_kernel<4, 4, 4, 2><<<tgrid, 128, 0, stream>>>(a)
+                    : gm::ser_thread_kernel<4, 4, 4, 4><<<tgrid, 128, 0, stream>>>(a);
+        return launched();
+    }
     gm::ser_kernel<WPB_SER><<<blocks_for(a.rows, WPB_SER), WPB_SER * 32, 0, stream>>>(a);
     return launched();
 }
@@ -839,6 +864,22 @@ gm_status gm_ser_chain_forward(const int32_t *a1_idx, const float *a1_w, int s2,
     a.out_idx = out_idx;
     check_chain_edges(a, stream);
     a.out_w = out_w;
+    // one thread per row for budgets s2 = s3 = s_mid of 2 or 4 and up to 4 legs
+    bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(out_idx) && aligned16(out_w);
+    for (int m = 0; m < nlegs; ++m) aligned = aligned && aligned16(leg_idx[m]) && aligned16(leg_w[m]);
+    if (aligned && s2 == s3 && s_mid == s2 && (s2 == 2 || s2 == 4) && s1 <= 4 && nlegs >= 2 && nlegs <= 4) {
+        const unsigned tgrid = (unsigned)((a.rows + 127) / 128);
+        if (s2 == 2) {
+            if (nlegs == 2) gm::ser_thread_kernel<2, 2, 4, 0, 2><<<tgrid, 128, 0, stream>>>(a);
+            else if (nlegs == 3) gm::ser_thread_kernel<2, 2, 4, 0, 3><<<tgrid, 128, 0, stream>>>(a);
+            else gm::ser_thread_kernel<2, 2, 4, 0, 4><<<tgrid, 128, 0, stream>>>(a);
+        } else {
+            if (nlegs == 2) gm::ser_thread_kernel<4, 4, 4, 0, 2><<<tgrid, 128, 0, stream>>>(a);
+            else if (nlegs == 3) gm::ser_thread_kernel<4, 4, 4, 0, 3><<<tgrid, 128, 0, stream>>>(a);
+            else gm::ser_thread_kernel<4, 4, 4, 0, 4><<<tgrid, 128, 0, stream>>>(a);
+        }
+        return launched();
+    }
     const unsigned grid = blocks_for(a.rows, WPB_SER);
     switch (nlegs) {
     case 1: gm::ser_chain_kernel<1, WPB_SER><<<grid, WPB_SER * 32, 0, stream>>>(a); break;

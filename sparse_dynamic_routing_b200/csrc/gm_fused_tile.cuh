@@ -208,6 +208,32 @@ __device__ __forceinline__ void ser_thread(const SerArgs &a, uint32_t row, int32
     }
 }
 
+// The referral alone, one thread per edge row (the tiled forward's phase 1 without the
+// attention): exact budgets S2, S3, s1 <= S1M, with SF refresh slots or a chain of NL steps.
+// Same arithmetic and order as ser_kernel (a warp per row), so the two give the same bits.
+// A' is written with 16-byte stores when s1 = S1M = 4 (16-byte aligned outputs).
+template <int S2, int S3, int S1M, int SF = 0, int NL = 1>
+__global__ void __launch_bounds__(128) ser_thread_kernel(SerArgs sa)
+{
+    const uint32_t row = blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= sa.rows) return;
+    int32_t to[S1M];
+    float wo[S1M];
+    ser_thread<S2, S3, S1M, SF, NL>(sa, row, to, wo);
+    if (sa.s1 == S1M && S1M == 4) {
+        *reinterpret_cast<int4 *>(sa.out_idx + (size_t)row * 4) = make_int4(to[0], to[1], to[2], to[3]);
+        *reinterpret_cast<float4 *>(sa.out_w + (size_t)row * 4) = make_float4(wo[0], wo[1], wo[2], wo[3]);
+    } else {
+#pragma unroll
+        for (int r = 0; r < S1M; ++r) {
+            if (r < sa.s1) {
+                sa.out_idx[(size_t)row * sa.s1 + r] = to[r];
+                sa.out_w[(size_t)row * sa.s1 + r] = wo[r];
+            }
+        }
+    }
+}
+
 // The S entries of one row of a warp's shared-memory edge tile (16-byte aligned for S = 4,
 // 8-byte for S = 2), read as one vector.
 template <int S, typename V> __device__ __forceinline__ void ld_tile(const V *p, V (&o)[S])
