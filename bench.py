@@ -527,6 +527,8 @@ def run_ours(args):
 def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     """The calls around the step, each timed alone with CUDA events, L2 flushed between reps.
 
+    ser_forward and sea_forward are the fused forward's two halves as separate calls, and
+    ser_forward_then_sea_forward the pair in sequence (A' written, then read back);
     leg_sparsify builds the step's two legs from the workload's stored edges; ser_backward
     takes the step's d ln w back to the legs; leg_backward takes those leg gradients back to
     the stored weights and the mixing coefficients; ser_sea_refresh_forward is the fused
@@ -596,7 +598,30 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     f_dw2 = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
     f_ws = torch.empty(gm.gm_sea_backward_workspace_size(g["q"].dtype, wl.s1, B, n, wl.hq, k, wl.d),
                        dtype=torch.uint8, device=dev)
+    # the two halves of the fused forward as separate calls (the survey's gm_ser_forward and
+    # gm_sea_forward), and the two in sequence: A' makes one round trip through HBM
+    fd = compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ap_i.cpu().numpy(),
+                          ap_w.cpu().numpy())["detail"]["fused_forward"]
+    ser_b = fd["a1"] + fd["a2_rows"] + fd["a_prime"]
+    sea_b = fd["q"] + fd["o"] + fd["lse"] + fd["a_prime"] + fd["kv_rows"]
+    so_i = torch.empty_like(ap_i)
+    so_w = torch.empty_like(ap_w)
+    so_o = torch.empty_like(g["q"])
+    so_lse = torch.empty((B, n, wl.hq), dtype=f32, device=dev)
     calls = {
+        "ser_forward": ("ser_thread_kernel", ser_b,
+                        lambda: gm.gm_ser_forward(g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"], wl.s1,
+                                                  out_idx=so_i, out_w=so_w, stream=stream)),
+        "sea_forward": ("sea_fwd_tile_kernel (SEA alone, edges read)", sea_b,
+                        lambda: gm.gm_sea_forward(g["q"], g["k"], g["v"], ap_i, ap_w, wl.scale, o=so_o,
+                                                  lse=so_lse, stream=stream)),
+        "ser_forward_then_sea_forward": ("the unfused pair of the step's fused forward", ser_b + sea_b,
+                                         lambda: (gm.gm_ser_forward(g["a1_idx"], g["a1_w"], g["a2_idx"],
+                                                                    g["a2_w"], wl.s1, out_idx=so_i,
+                                                                    out_w=so_w, stream=stream),
+                                                  gm.gm_sea_forward(g["q"], g["k"], g["v"], so_i, so_w,
+                                                                    wl.scale, o=so_o, lse=so_lse,
+                                                                    stream=stream))),
         "leg_sparsify": ("leg_fwd_tile_kernel", e_b + mix_b + leg_b,
                          lambda: gm.gm_leg_sparsify(le["e_idx"], le["e_w"], le["mix1"], le["mix2"],
                                                     wl.s2, wl.s3, a1i, a1w, a2i, a2w, stream=stream)),
@@ -616,14 +641,14 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
                                       g["q"], g["k"], g["v"], g["a1_idx"], g["a1_w"], ch_legs,
                                       wl.s2, wl.s1, wl.scale, out_idx=ch_i, out_w=ch_w, o=ch_o,
                                       lse=ch_lse, stream=stream)),
-        "ser_refresh_backward": ("zero_i32_kernel + ser_bwd_kernel (warp per row, refresh lanes)",
+        "ser_refresh_backward": ("zero_i32_kernel + ser_bwd_thread_kernel (refresh slots)",
                                  leg_b + e_b + tok * k * wl.s1 * 4 + grad_b + tok * k * wl.s1 * 4
                                  + tok * k * wl.s3 * 4,
                                  lambda: gm.gm_ser_refresh_backward(
                                      g["a1_idx"], g["a1_w"], g["a2_idx"], g["a2_w"], le["e_idx"],
                                      le["e_w"], dlw, grad_is_log=True, dw1=rf_dw1, dw2=rf_dw2,
                                      dfw=rf_dfw, stream=stream)),
-        "ser_chain_backward": ("zero_i32_kernel x2 + ser_chain_bwd_kernel (3 legs)",
+        "ser_chain_backward": ("zero_i32_kernel x2 + ser_chain_bwd_thread_kernel (3 legs)",
                                leg_b + tok * k * wl.s3 * 8 + tok * k * wl.s1 * 4
                                + tok * k * (wl.s2 + 2 * wl.s3) * 4 + 2 * tok * k * wl.s3 * 4,
                                lambda: gm.gm_ser_chain_backward(

@@ -538,7 +538,7 @@ gm_status launch_dense_refresh(const void *q, const void *k, int64_t tokens, con
     auto kern = gm::dense_refresh_kernel<D, G, BN, SFM>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Geo::SMEM_BYTES) != cudaSuccess)
         return GM_ERR_CUDA;
-    kern<<<(unsigned)((int64_t)a.BH * a.nblk), 320, Geo::SMEM_BYTES, st>>>(tq, tk, a);
+    kern<<<(unsigned)((int64_t)a.BH * a.nblk), Geo::THREADS, Geo::SMEM_BYTES, st>>>(tq, tk, a);
     return launched();
 }
 

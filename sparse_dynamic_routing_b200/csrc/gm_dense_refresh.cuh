@@ -13,9 +13,9 @@
 // prefix run on the tensor cores: tcgen05.mma with bf16 operands staged by TMA in the
 // 128-byte swizzle layout and fp32 accumulators in tensor memory (TMEM), two key stages and
 // two accumulator sets, so the MMAs of key block j + 1 overlap the selection over block j.
-// Warp roles: warps 0-7 select (two threads per query row = TMEM lane, each taking every other
-// 32-column chunk of a key block), warp 8 loads (TMA), warp 9 issues the MMAs. Every wait is
-// bounded (gm_common.cuh, mbar_wait).
+// Warp roles: warps 0 .. 4 NPART - 1 select (NPART threads per query row = TMEM lane, thread
+// p taking the 32-column chunks p, p + NPART, ... of a key block), warp 4 NPART loads (TMA),
+// warp 4 NPART + 1 issues the MMAs. Every wait is bounded (gm_common.cuh, mbar_wait).
 //
 // Selection per thread, streaming over ascending t: a sorted register list of the SFM heaviest
 // (mass, t) so far (SFM = sf rounded up to 2, 4 or 8; the first sf of the top SFM are the top
@@ -24,14 +24,18 @@
 // is branch-free: per column G FMAs, a max, a compare that sets a bit of a candidate mask, and
 // a store of the x_g to a per-thread shared-memory slot; then each lane walks its own mask
 // (computing the few candidates' masses with G exponentials and inserting those that beat the
-// list), so the lanes of a warp never diverge per column. At the end the two threads of a row
-// merge their lists.
+// list), so the lanes of a warp never diverge per column. At the end the NPART threads of a
+// row merge their lists.
 #pragma once
 
 #include <cuda.h>
 
 #include "gm_common.cuh"
 #include "gm_umma.cuh"
+
+#ifndef GM_DENSE_NPART
+#define GM_DENSE_NPART 4
+#endif
 
 namespace gm {
 
@@ -53,7 +57,11 @@ template <int D, int G, int BN> struct DenseGeom {
     static constexpr int K_ATOM = BN * 128;
     static constexpr int QBYTES = G * NA * Q_ATOM;
     static constexpr int KBYTES = NST * NA * K_ATOM;
-    static constexpr int NSEL = 2 * BM;             // selection threads (two per row)
+    // selection threads per query row: one per 32-column chunk of a key block, at most
+    // GM_DENSE_NPART (more threads hide more of the scan's latency)
+    static constexpr int NPART = (BN / 32) < GM_DENSE_NPART ? (BN / 32) : GM_DENSE_NPART;
+    static constexpr int NSEL = NPART * BM;         // selection threads
+    static constexpr int THREADS = NSEL + 64;       // + the load warp and the MMA warp
     static constexpr int SUB = G == 4 ? 8 : 16;     // columns scanned per candidate mask
     static constexpr int OFF_K = QBYTES;
     static constexpr int OFF_LIST = QBYTES + KBYTES;  // x values [SUB][NSEL][G]
@@ -67,6 +75,7 @@ template <int D, int G, int BN> struct DenseGeom {
     static constexpr int SMEM_BYTES = TMEM_COLS > 256 && NEED < 120 * 1024 ? 120 * 1024 : NEED;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     static_assert(BN == 64 || BN == 128, "key block of 64 or 128");
+    static_assert((NPART - 1) * 2 * BM * 8 <= SUB * NSEL * G, "the parts' lists (SFM <= 8) fit the x slots");
     static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512 && (TMEM_COLS & (TMEM_COLS - 1)) == 0,
                   "accumulators fit the 512 TMEM columns");
 };
@@ -101,7 +110,7 @@ template <int SFM> __device__ __forceinline__ float skip_bound(const float (&kw)
 }
 
 template <int D, int G, int BN, int SFM>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(DenseGeom<D, G, BN>::THREADS, 1)
 dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                      DenseRefreshArgs a)
 {
@@ -149,7 +158,8 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     umma::fence_after_sync();
     const uint32_t tmem = *tslot_p;
 
-    if (warp == 8) {
+    constexpr int LOAD_WARP = Geo::NSEL / 32, MMA_WARP = LOAD_WARP + 1;
+    if (warp == LOAD_WARP) {
         // ---- loads: the query tile once, then the key blocks through NST stages ----------
         if (lane == 0) {
             mbar_arrive_expect(q_full, Geo::QBYTES);
@@ -173,7 +183,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
                 for (int j = max(0, issued - NST); j < issued; ++j) mbar_wait(k_full + 8 * (j % NST), (j / NST) & 1);
             }
         }
-    } else if (warp == 9) {
+    } else if (warp == MMA_WARP) {
         // ---- MMAs: S_g = Q_g K^T into accumulator set j % NACC ------------------------------
         if (lane == 0) {
             constexpr uint32_t idesc = umma::idesc_bf16_f32(Geo::BM, BN);
@@ -201,9 +211,9 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
             mbar_wait(mma_done, 0);
         }
     } else {
-        // ---- selection: two threads per query row i = TMEM lane (warp w reads lane quarter
-        // w % 4), the thread of half w / 4 scanning the chunks cc with cc % 2 == w / 4 ---------
-        const int quarter = warp & 3, half = warp >> 2;
+        // ---- selection: NPART threads per query row i = TMEM lane (warp w reads lane quarter
+        // w % 4), the thread of part w / 4 scanning the chunks cc with cc % NPART == w / 4 -----
+        const int quarter = warp & 3, part = warp >> 2;
         const int r = quarter * 32 + lane;
         const int tid = threadIdx.x;  // 0 .. NSEL-1
         const int i = i0 + r;
@@ -230,7 +240,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
             if (!ok) break;
             umma::fence_after_sync();
 #pragma unroll 1
-            for (int cc = half; cc < BN / 32; cc += 2) {
+            for (int cc = part; cc < BN / 32; cc += Geo::NPART) {
                 uint32_t sv[G][32];
 #pragma unroll
                 for (int g = 0; g < G; ++g) umma::tmem_ld32(tlane + (as * G + g) * BN + cc * 32, sv[g]);
@@ -272,24 +282,29 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
             umma::fence_before_sync();
             mbar_arrive(acc_empty + 8 * as);
         }
-        // the two threads of a row merge their lists: the second half hands its list over in
-        // shared memory (the x-value slots, free now), the first inserts it and writes the row
-        float *hand = listx;  // [BM][SFM] masses, then [BM][SFM] positions
+        // the NPART threads of a row merge their lists: parts 1.. hand theirs over in shared
+        // memory (the x-value slots, free now), part 0 inserts them and writes the row
+        float *hand = listx;  // per part p >= 1: [BM][SFM] masses, then [BM][SFM] positions
         named_barrier_sync(1, Geo::NSEL);  // every scan is done with the slots
-        if (half == 1) {
+        if (part > 0) {
+            float *mine = hand + (size_t)(part - 1) * 2 * Geo::BM * SFM;
 #pragma unroll
             for (int x = 0; x < SFM; ++x) {
-                hand[r * SFM + x] = kw[x];
-                hand[Geo::BM * SFM + r * SFM + x] = __int_as_float(kt[x]);
+                mine[r * SFM + x] = kw[x];
+                mine[Geo::BM * SFM + r * SFM + x] = __int_as_float(kt[x]);
             }
         }
         named_barrier_sync(1, Geo::NSEL);
-        if (half == 0 && ok) {
+        if (part == 0 && ok) {
 #pragma unroll
-            for (int x = 0; x < SFM; ++x) {
-                const float m = hand[r * SFM + x];
-                if (m > kw[SFM - 1] || (m == kw[SFM - 1] && m >= 0.0f))
-                    list_insert<SFM>(kw, kt, m, __float_as_int(hand[Geo::BM * SFM + r * SFM + x]));
+            for (int p = 1; p < Geo::NPART; ++p) {
+                const float *theirs = hand + (size_t)(p - 1) * 2 * Geo::BM * SFM;
+#pragma unroll
+                for (int x = 0; x < SFM; ++x) {
+                    const float m = theirs[r * SFM + x];
+                    if (m > kw[SFM - 1] || (m == kw[SFM - 1] && m >= 0.0f))
+                        list_insert<SFM>(kw, kt, m, __float_as_int(theirs[Geo::BM * SFM + r * SFM + x]));
+                }
             }
             if (valid) {
                 const size_t o = ((size_t)(row0 + i) * a.hkv + h) * a.sf;
