@@ -65,7 +65,8 @@ template <int D, int G, int BN> struct DenseGeom {
     static constexpr int SUB = G == 4 ? 8 : 16;     // columns scanned per candidate mask
     static constexpr int OFF_K = QBYTES;
     static constexpr int OFF_LIST = QBYTES + KBYTES;  // x values [SUB][NSEL][G]
-    static constexpr int OFF_BAR = OFF_LIST + SUB * NSEL * G * 4;
+    static constexpr int OFF_BOUND = OFF_LIST + SUB * NSEL * G * 4;  // skip bounds [BM][NPART]
+    static constexpr int OFF_BAR = OFF_BOUND + BM * NPART * 4;
     static constexpr int NBAR = 2 + 2 * NST + 2 * NACC;  // q_full, k_full/empty, acc_full/empty, mma_done
     static constexpr int TMEM_COLS = NACC * G * BN;
     // + TMEM slot and 1 KB of alignment; a CTA that takes more than half of the 512 TMEM columns
@@ -127,6 +128,11 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
     const uint32_t mma_done = acc_empty + 8 * NACC, tslot = mma_done + 8;
     const uint32_t *tslot_p = reinterpret_cast<const uint32_t *>(sm + Geo::OFF_BAR + Geo::NBAR * 8);
     float *listx = reinterpret_cast<float *>(sm + Geo::OFF_LIST);  // [SUB][NSEL][G] x values
+    // each selection thread's current skip bound, [row][part]: a position whose mass lies
+    // below any part's smallest kept mass cannot enter the row's top list, so every part
+    // filters by the largest of the row's bounds (they only grow; a stale read is still valid)
+    volatile float *sbound = reinterpret_cast<float *>(sm + Geo::OFF_BOUND);
+    if (threadIdx.x < Geo::NSEL) sbound[threadIdx.x] = -INFINITY;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ib = a.nblk - 1 - (int)(blockIdx.x / (unsigned)a.BH);  // longest prefixes first
@@ -277,6 +283,11 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
                         if (m > kw[SFM - 1]) list_insert<SFM>(kw, kt, m, t0 + c);
                     }
                     L = skip_bound<SFM>(kw);
+                    if constexpr (Geo::NPART > 1) {
+                        sbound[r * Geo::NPART + part] = L;
+#pragma unroll
+                        for (int p = 0; p < Geo::NPART; ++p) L = fmaxf(L, sbound[r * Geo::NPART + p]);
+                    }
                 }
             }
             umma::fence_before_sync();
