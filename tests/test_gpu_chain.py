@@ -196,4 +196,10 @@ def test_chain_backward_thread_and_warp_agree(s, nlegs):
         ref = b.cpu().double().numpy()
         err = np.abs(a.cpu().double().numpy() - ref).max()
         assert err <= 1e-5 * max(np.abs(ref).max(), 1e-30)
+    # the forward: one thread per row (aligned legs) against one warp per row, bit for bit
+    ft = gm.gm_ser_chain_forward(t(a1[0]), t(a1[1]), [(t(i), t(w)) for i, w in legs], s, 4)
+    fw = gm.gm_ser_chain_forward(misaligned(a1[0]), misaligned(a1[1]),
+                                 [(misaligned(i), misaligned(w)) for i, w in legs], s, 4)
+    for a, b in zip(ft, fw):
+        np.testing.assert_array_equal(a.cpu().numpy().view(np.uint32), b.cpu().numpy().view(np.uint32))
     gm.gm_check_device_errors()

@@ -221,4 +221,10 @@ def test_thread_and_warp_backward_agree_bit_for_bit_on_ties(s, sf):
         oi, ow, _ = oracle.ser(*args, s1)
     assert_bits(wi, ww, oi, ow)
     assert_bits(fi_, fw_, oi, ow)
+    # the standalone referral on misaligned legs takes the warp-per-row kernel
+    if sf:
+        mi, mw = gm.gm_ser_refresh_forward(*[misaligned(a) for a in args], s1)
+    else:
+        mi, mw = gm.gm_ser_forward(*[misaligned(a) for a in args], s1)
+    assert_bits(mi, mw, oi, ow)
     gm.gm_check_device_errors()
