@@ -17,6 +17,7 @@
 // Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
 #pragma once
 
+
 #include "gm_bwd_gather.cuh"
 #include "gm_common.cuh"
 #include "gm_fused_tile.cuh"
@@ -113,7 +114,7 @@ template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER, int SB
 __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
     using TG = BwdTileGeom<T, D, G, S1M>;
-    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
+    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NP = VEC / 2;
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     constexpr int TILE_BYTES = bwd_tile_bytes<S1M, SB, GATHER>();
@@ -129,7 +130,6 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
     char *stages = wbase + TILE_BYTES;
 
     const uint32_t rows = a.rows;
-    const uint32_t ntiles = (rows + 31) / 32;
     const uint32_t W = gridDim.x * WPB;
     const int rr = lane / C, c = lane % C;
     const float sl2 = a.scale * LOG2E;
@@ -137,8 +137,24 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
     const char *kbase = static_cast<const char *>(a.k) + (size_t)c * 16;
     const char *vbase = static_cast<const char *>(a.v) + (size_t)c * 16;
 
-    for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
-        const uint32_t r0 = tile * 32;
+    // rounds of one 32-row tile per warp, the remainder split evenly over the warps (as in
+    // the forward tile kernel)
+    const uint32_t gw = blockIdx.x * WPB + wid;
+    const uint32_t full = rows / (W * 32);
+    const uint32_t rem = rows - full * W * 32;
+    const uint32_t per = (rem + W - 1) / W;
+    const uint32_t nround = full + (rem > 0 ? 1u : 0u);
+    for (uint32_t round = 0; round < nround; ++round) {
+        uint32_t r0, rend;
+        if (round < full) {
+            r0 = (round * W + gw) * 32;
+            rend = r0 + 32;
+        } else {
+            r0 = full * W * 32 + gw * per;
+            if (r0 >= rows) break;  // warp-uniform
+            rend = min(r0 + per, rows);
+        }
+        const int npass = (int)((rend - r0 + RPW - 1) / RPW);  // warp-uniform, <= 32 / RPW
 
         // ---- phase 1: the tile's edges, one thread per row ----------------------------------
         {
@@ -146,12 +162,12 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
             // slots are stored as K/V rows ((b*n + t)*hkv + h): phase 2 issues its copies and
             // keys its records without decomposing the row again
             uint32_t seq_base = 0, h = 0;
-            if (row < rows) a.map.split(row, seq_base, h);
+            if (row < rend) a.map.split(row, seq_base, h);
 #pragma unroll
             for (int r = 0; r < S1M; ++r) {
                 int32_t t = 0;
                 float lw = -INFINITY;
-                if (row < rows && r < a.s) {
+                if (row < rend && r < a.s) {
                     const float w = __ldg(a.w + (size_t)row * a.s + r);
                     const int32_t ti = __ldg(a.idx + (size_t)row * a.s + r);
                     if (w > 0.0f) {
@@ -180,7 +196,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
 
         // ---- phase 2 ----------------------------------------------------------------------------
         auto issue = [&](int pass) {
-            if (pass < NPASS) {
+            if (pass < npass) {
                 const int lr = pass * RPW + rr;
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
@@ -192,7 +208,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 ld_tile<S1M>(tile_t + lr * S1M, tv);
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj) {
-                    const bool live = row < rows && lwv[jj] != -INFINITY;
+                    const bool live = row < rend && lwv[jj] != -INFINITY;
                     const size_t off = (size_t)(live ? (uint32_t)tv[jj] : 0u) * TG::ROW;
                     cp_async16_zfill(st + TG::RK + jj * TG::ROW + c * 16, kbase + off, live);
                     cp_async16_zfill(st + TG::RV + jj * TG::ROW + c * 16, vbase + off, live);
@@ -204,7 +220,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
         // the loads; without them in shared memory more warps are resident)
         auto load_qg = [&](int pass, uint4 (&qv)[G], uint4 (&gv)[G]) {
             const uint32_t row = r0 + pass * RPW + rr;
-            const bool ok = pass < NPASS && row < rows;
+            const bool ok = pass < npass && row < rend;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const size_t off = (size_t)row * (G * TG::ROW) + g * TG::ROW + c * 16;
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
 #pragma unroll
         for (int pass = 0; pass < P; ++pass) issue(pass);
 
-        for (int pass = 0; pass < NPASS; ++pass) {
+        for (int pass = 0; pass < npass; ++pass) {
             uint4 qc[G], gc[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) {
@@ -228,7 +244,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
             cp_async_wait<P - 1>();
             const int lr = pass * RPW + rr;
             const uint32_t row = r0 + lr;
-            const bool valid = row < rows;
+            const bool valid = row < rend;
             const char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
 
             float lw[S1M];
@@ -459,7 +475,7 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
         if constexpr (SB > 0) {
             // ---- phase 3: the referral backward of the tile's rows, one thread per row ------
             const uint32_t row = r0 + lane;
-            if (row < rows) {
+            if (row < rend) {
                 uint32_t seq_base, h;
                 a.map.split(row, seq_base, h);
                 int32_t kt[S1M];

@@ -25,6 +25,7 @@
 // the reduction, so rows at a ragged tail simply compute on zeros and store nothing.
 #pragma once
 
+
 #include "gm_common.cuh"
 #include "gm_sea.cuh"
 #include "gm_ser.cuh"
@@ -284,7 +285,7 @@ template <typename T, int D, int G, bool REFER, int S2, int S3, int S1M, int P, 
 __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel(SerArgs sa, SeaArgs a)
 {
     using TG = TileGeom<T, D, G, S1M, CPL>;
-    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NPASS = TG::NPASS, NP = VEC / 2;
+    constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NP = VEC / 2;
     static_assert(VEC % 2 == 0, "packed fp32x2 math");
     extern __shared__ __align__(16) char smem[];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -296,8 +297,16 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
     char *stages = wbase + TILE_BYTES;
 
     const uint32_t rows = a.rows;
-    const uint32_t ntiles = (rows + 31) / 32;
     const uint32_t W = gridDim.x * WPB;
+    const uint32_t gw = blockIdx.x * WPB + wid;
+    // Rows are dealt in rounds: every warp takes a 32-row tile per round, the grid sweeping
+    // the rows in order (one sequence's K/V stays in L2); the rows left after the full rounds
+    // are split evenly, so every warp's last tile holds the same number of rows (at most 32)
+    // and no round runs with part of the warps idle.
+    const uint32_t full = rows / (W * 32);
+    const uint32_t rem = rows - full * W * 32;
+    const uint32_t per = (rem + W - 1) / W;
+    const uint32_t nround = full + (rem > 0 ? 1u : 0u);
     const int rr = lane / C, c = lane % C;  // phase-2 row within the pass, chunk
     const float sl2 = a.scale * LOG2E;
     const T *Qg = static_cast<const T *>(a.q);
@@ -306,8 +315,17 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
     const char *kbase = static_cast<const char *>(a.k) + (size_t)(c * CPL) * 16;
     const char *vbase = static_cast<const char *>(a.v) + (size_t)(c * CPL) * 16;
 
-    for (uint32_t tile = blockIdx.x * WPB + wid; tile < ntiles; tile += W) {
-        const uint32_t r0 = tile * 32;
+    for (uint32_t round = 0; round < nround; ++round) {
+        uint32_t r0, rend;
+        if (round < full) {
+            r0 = (round * W + gw) * 32;
+            rend = r0 + 32;
+        } else {
+            r0 = full * W * 32 + gw * per;
+            if (r0 >= rows) break;  // warp-uniform
+            rend = min(r0 + per, rows);
+        }
+        const int npass = (int)((rend - r0 + RPW - 1) / RPW);  // warp-uniform, <= NPASS
 
         // ---- phase 1: the tile's edges, one thread per row ------------------------------
         {
@@ -320,7 +338,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                 wo[r] = 0.0f;
             }
             if constexpr (!REFER) {
-                if (row < rows) {
+                if (row < rend) {
 #pragma unroll
                     for (int r = 0; r < S1M; ++r) {
                         if (r < a.s) {
@@ -337,7 +355,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                         }
                     }
                 }
-            } else if (row < rows) {
+            } else if (row < rend) {
                 ser_thread<S2, S3, S1M, SF, NL>(sa, row, to, wo);
                 if (sa.out_idx != nullptr) {
                     if (sa.s1 == S1M && S1M == 4) {
@@ -357,7 +375,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
             // K/V row of each slot ((b*n + t)*hkv + h), so phase 2 issues its copies without
             // decomposing the row again
             uint32_t seq_base = 0, h = 0;
-            if (row < rows) a.map.split(row, seq_base, h);
+            if (row < rend) a.map.split(row, seq_base, h);
 #pragma unroll
             for (int r = 0; r < S1M; ++r) {
                 tile_t[lane * S1M + r] = (int32_t)((seq_base + (uint32_t)to[r]) * (uint32_t)a.hkv + h);
@@ -368,7 +386,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
 
         // ---- phase 2: attention, RPW rows per pass, P passes of copies in flight -----------
         auto issue = [&](int pass) {
-            if (pass < NPASS) {
+            if (pass < npass) {
                 const int lr = pass * RPW + rr;  // row within the tile
                 const uint32_t row = r0 + lr;
                 char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
@@ -380,7 +398,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
                 ld_tile<S1M>(tile_t + lr * S1M, tv);
 #pragma unroll
                 for (int jj = 0; jj < S1M; ++jj) {
-                    const bool live = row < rows && lwv[jj] != -INFINITY;
+                    const bool live = row < rend && lwv[jj] != -INFINITY;
                     const uint32_t kvrow = live ? (uint32_t)tv[jj] : 0u;
 #pragma unroll
                     for (int cc = 0; cc < CPL; ++cc) {
@@ -400,7 +418,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
             for (int g = 0; g < G; ++g)
 #pragma unroll
                 for (int cc = 0; cc < CPL; ++cc)
-                    qv[g][cc] = (pass < NPASS && row < rows)
+                    qv[g][cc] = (pass < npass && row < rend)
                                     ? ld16(reinterpret_cast<const char *>(Qg) + (size_t)row * (G * TG::ROW) +
                                            g * TG::ROW + (c * CPL + cc) * 16)
                                     : make_uint4(0u, 0u, 0u, 0u);
@@ -410,7 +428,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
 #pragma unroll
         for (int pass = 0; pass < P; ++pass) issue(pass);
 
-        for (int pass = 0; pass < NPASS; ++pass) {
+        for (int pass = 0; pass < npass; ++pass) {
             uint4 qcur[G][CPL];
 #pragma unroll
             for (int g = 0; g < G; ++g)
@@ -420,7 +438,7 @@ __global__ void __launch_bounds__(WPB * 32, GM_TILE_MINB(P)) sea_fwd_tile_kernel
             cp_async_wait<P - 1>();
             const int lr = pass * RPW + rr;
             const uint32_t row = r0 + lr;
-            const bool valid = row < rows;
+            const bool valid = row < rend;
             const char *st = stages + (pass % P) * TG::STAGE + rr * TG::RBYTES;
 
             float lw[S1M];
