@@ -513,6 +513,16 @@ gm_status gm_dense_refresh_edges(const void *q, const void *k, gm_dtype dtype, c
  */
 gm_status gm_check_device_errors(cudaStream_t stream);
 
+/*
+ * gm_selftest_wait_timeout - diagnostic for the bounded waits: launches one kernel whose
+ * single wait (on a shared-memory barrier that nothing arrives at) runs out after about one
+ * second; the kernel then sets the device error flag and returns, so the following
+ * gm_check_device_errors returns GM_ERR_WAIT_TIMEOUT and the device stays usable. The
+ * library's real waits (asynchronous copies and tensor-core operations of
+ * gm_dense_refresh_edges, the look-back of the backward's scan) give up the same way.
+ */
+gm_status gm_selftest_wait_timeout(cudaStream_t stream);
+
 /* Static, human-readable name of a status code. Never NULL. */
 const char *gm_status_string(gm_status status);
 

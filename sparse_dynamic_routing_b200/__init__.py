@@ -17,6 +17,8 @@ its Python binding plus the seeded synthetic-input generators (`inputs`).
     gm_ser_sea_backward both backward passes in one call (the referral's inside the attention's)
     gm_dense_refresh_edges
                         refresh edges from a dense attention layer (its top positions)
+    gm_selftest_wait_timeout
+                        diagnostic: one bounded wait that runs out (GM_ERR_WAIT_TIMEOUT)
 """
 from ._binding import (  # noqa: F401
     GM_BF16,
@@ -44,6 +46,7 @@ from ._binding import (  # noqa: F401
     gm_ser_sea_refresh_forward,
     gm_ser_sea_backward,
     gm_ser_sea_forward,
+    gm_selftest_wait_timeout,
     gm_version,
     load_library,
     status_string,

@@ -61,6 +61,7 @@ SIGNATURES = {
     "gm_status_string": [_ci],
     "gm_version": [],
     "gm_checked_build": [],
+    "gm_selftest_wait_timeout": [_vp],
 }
 
 
@@ -610,6 +611,12 @@ def gm_check_device_errors(stream=None):
     """Synchronise the stream; raise GMIndexRangeError if a kernel met a bad index, GMError if a
     kernel gave up on a bounded wait (GM_ERR_WAIT_TIMEOUT)."""
     _check(load_library().gm_check_device_errors(_stream(stream)), "gm_check_device_errors")
+
+
+def gm_selftest_wait_timeout(stream=None):
+    """Launch the bounded-wait diagnostic (about one second); gm_check_device_errors then
+    raises GMError with status GM_ERR_WAIT_TIMEOUT."""
+    _check(load_library().gm_selftest_wait_timeout(_stream(stream)), "gm_selftest_wait_timeout")
 
 
 def gm_version() -> int:

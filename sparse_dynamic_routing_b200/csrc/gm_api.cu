@@ -591,11 +591,30 @@ gm_status noalloc_scratch(void **out)
     return GM_OK;
 }
 
+// One bounded wait that nothing completes: the thread waits on a shared-memory barrier with
+// no arrivals, gives up after WAIT_LIMIT_NS, sets ERR_WAIT_TIMEOUT and returns.
+__global__ void wait_timeout_selftest_kernel()
+{
+    __shared__ __align__(8) unsigned long long bar;
+    if (threadIdx.x == 0) {
+        const uint32_t b = gm::smem_u32(&bar);
+        gm::mbar_init(b, 1);
+        gm::mbar_init_fence();
+        (void)gm::mbar_wait(b, 0);
+    }
+}
+
 }  // namespace
 
 extern "C" {
 
 int gm_version(void) { return 100; }
+
+gm_status gm_selftest_wait_timeout(cudaStream_t stream)
+{
+    wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>();
+    return launched();
+}
 
 int gm_checked_build(void) { return GM_CHECKED ? 1 : 0; }
 
