@@ -96,6 +96,24 @@ template <int SFM> __device__ __forceinline__ void list_insert(float (&kw)[SFM],
     }
 }
 
+// The same insertion for a thread's own stream of positions, which arrive in ascending t: an
+// equal mass already in the list has the smaller position and stays first, so the strict
+// comparison alone gives the (mass desc, position asc) order.
+template <int SFM>
+__device__ __forceinline__ void list_insert_ascending(float (&kw)[SFM], int (&kt)[SFM], float m, int t)
+{
+#pragma unroll
+    for (int r = 0; r < SFM; ++r) {
+        const bool before = m > kw[r];
+        const float w0 = kw[r];
+        const int t0 = kt[r];
+        kw[r] = before ? m : w0;
+        kt[r] = before ? t : t0;
+        m = before ? w0 : m;
+        t = before ? t0 : t;
+    }
+}
+
 // Barrier over the first `count` threads of the CTA (the selection warps), id 1 (id 0 is the
 // CTA-wide __syncthreads).
 __device__ __forceinline__ void named_barrier_sync(int id, int count)
@@ -280,7 +298,7 @@ dense_refresh_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_const
 #pragma unroll
                         for (int g = 0; g < G; ++g) sum += ex2(myx[c * Geo::NSEL * G + g]);
                         const float m = sum * (1.0f / G);
-                        if (m > kw[SFM - 1]) list_insert<SFM>(kw, kt, m, t0 + c);
+                        if (m > kw[SFM - 1]) list_insert_ascending<SFM>(kw, kt, m, t0 + c);
                     }
                     L = skip_bound<SFM>(kw);
                     if constexpr (Geo::NPART > 1) {
