@@ -239,6 +239,26 @@ gm_status dispatch(gm_dtype dtype, int d, int G, Args &&...args)
 #undef GM_CASE_G
 }
 
+// Launch with programmatic stream serialization: the kernel may start while the previous one
+// on the stream drains, and waits for it (pdl_wait) before touching its outputs. Used for the
+// chain of kernels inside one backward call, whose first kernel is launched the ordinary way.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t st,
+                Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    (void)cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // Persistent grid for a kernel with `smem` bytes of dynamic shared memory per block:
 // as many blocks as fit on the device at once, but no more than the rows need.
 template <typename K>
@@ -362,7 +382,7 @@ constexpr int BWD_TILE_P = GM_BWD_TILE_P;
 constexpr int WPB_BWD_TILE = GM_WPB_BWD_TILE;
 
 template <typename T, int D, int G, int S1M, bool GATHER, int SB = 0>
-gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
+gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st, bool pdl = false)
 {
     using TG = gm::BwdTileGeom<T, D, G, S1M>;
     auto kern = gm::sea_bwd_tile_kernel<T, D, G, S1M, BWD_TILE_P, WPB_BWD_TILE, GATHER, SB>;
@@ -372,7 +392,10 @@ gm_status launch_bwd_tile(const SeaBwdArgs &a, cudaStream_t st)
         return GM_ERR_CUDA;
     const int64_t tiles = ((int64_t)a.rows + 31) / 32;
     const unsigned grid = persistent_blocks(kern, WPB_BWD_TILE * 32, smem, tiles, WPB_BWD_TILE);
-    kern<<<grid, WPB_BWD_TILE * 32, smem, st>>>(a);
+    if (pdl)
+        launch_pdl(kern, grid, WPB_BWD_TILE * 32, smem, st, a);
+    else
+        kern<<<grid, WPB_BWD_TILE * 32, smem, st>>>(a);
     return launched();
 }
 
@@ -457,21 +480,27 @@ template <typename T, int D, int G> struct SeaBwdGather {
             gm::zero_i32_kernel<<<148 * 4, 256, 0, st>>>(ws.cnt, ws.zero_words);
             const unsigned cgrid = (unsigned)((R + 255) / 256);
             if (a.s <= 2)
-                gm::edge_count_kernel<2><<<cgrid, 256, 0, st>>>(idx, w, a.n, a.map, a.s, a.rows, a.hkv, ws.cnt, ws.rank);
+                launch_pdl(gm::edge_count_kernel<2>, cgrid, 256, 0, st, idx, w, a.n, a.map, a.s, a.rows, a.hkv,
+                           ws.cnt, ws.rank);
             else
-                gm::edge_count_kernel<4><<<cgrid, 256, 0, st>>>(idx, w, a.n, a.map, a.s, a.rows, a.hkv, ws.cnt, ws.rank);
-            gm::scan_lookback_kernel<<<ws.nblk, gm::SCAN_THREADS, 0, st>>>(ws.cnt, R, ws.state, ws.ticket, ws.off);
+                launch_pdl(gm::edge_count_kernel<4>, cgrid, 256, 0, st, idx, w, a.n, a.map, a.s, a.rows, a.hkv,
+                           ws.cnt, ws.rank);
+            launch_pdl(gm::scan_lookback_kernel, ws.nblk, gm::SCAN_THREADS, 0, st, ws.cnt, R, ws.state, ws.ticket,
+                       ws.off);
             if (launched() != GM_OK) return GM_ERR_CUDA;
             a.rank = ws.rank;
             a.off = ws.off;
             a.srec = ws.srec;
             gm_status rs;
             if (sb == 2)
-                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 2>(a, st) : launch_bwd_tile<T, D, G, 4, true, 2>(a, st);
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 2>(a, st, true)
+                              : launch_bwd_tile<T, D, G, 4, true, 2>(a, st, true);
             else if (sb == 4)
-                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 4>(a, st) : launch_bwd_tile<T, D, G, 4, true, 4>(a, st);
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true, 4>(a, st, true)
+                              : launch_bwd_tile<T, D, G, 4, true, 4>(a, st, true);
             else
-                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st) : launch_bwd_tile<T, D, G, 4, true>(a, st);
+                rs = a.s <= 2 ? launch_bwd_tile<T, D, G, 2, true>(a, st, true)
+                              : launch_bwd_tile<T, D, G, 4, true>(a, st, true);
             if (rs != GM_OK) return rs;
             auto kern = gm::sea_bwd_gather_kernel<T, D, G, WPB_GATHER, GATHER_U, GATHER_P>;
             const size_t smem = (size_t)WPB_GATHER * GATHER_P * GATHER_U * G * 32 * 16;
@@ -479,8 +508,8 @@ template <typename T, int D, int G> struct SeaBwdGather {
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
                 return GM_ERR_CUDA;
             const int64_t chunks = (E + 31) / 32;  // upper bound: the active count is on the device
-            kern<<<blocks_for(chunks, WPB_GATHER), WPB_GATHER * 32, smem, st>>>(a.q, a.dout, a.dk, a.dv, ws,
-                                                                               (uint32_t)R, a.accumulate);
+            launch_pdl(kern, blocks_for(chunks, WPB_GATHER), WPB_GATHER * 32, smem, st, a.q, a.dout, a.dk, a.dv, ws,
+                       (uint32_t)R, a.accumulate);
             return launched();
         } else {
             return GM_ERR_UNSUPPORTED;

@@ -83,6 +83,7 @@ constexpr int SCAN_TILE = SCAN_THREADS * SCAN_PER_THREAD;
 
 __global__ void zero_i32_kernel(int32_t *p, int64_t count)
 {
+    pdl_trigger();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x)
         p[i] = 0;
 }
@@ -142,6 +143,8 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_lookback_kernel(const int32
 {
     __shared__ uint32_t s_tile;
     __shared__ int32_t s_prefix;
+    pdl_wait();  // the counts
+    pdl_trigger();
     if (threadIdx.x == 0) s_tile = atomicAdd(ticket, 1u);
     __syncthreads();
     const uint32_t tile = s_tile;
@@ -207,6 +210,8 @@ template <int S1M>
 __global__ void edge_count_kernel(const int32_t *idx, const float *w, int n, RowMap map, int s, uint32_t rows,
                                  int hkv, int32_t *cnt, int32_t *rank)
 {
+    pdl_wait();  // the zeroed counters
+    pdl_trigger();
     for (uint32_t row = blockIdx.x * blockDim.x + threadIdx.x; row < rows; row += gridDim.x * blockDim.x) {
         uint32_t seq_base, h;
         map.split(row, seq_base, h);
@@ -231,6 +236,7 @@ template <typename T, int D, int G, int WPB, int U, int P>
 __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q, const void *dout, float *dk, float *dv,
                                                                  GatherWs ws, uint32_t R, int accumulate)
 {
+    pdl_wait();  // the records of the row pass
     constexpr int VEC = Vec<T>::N, C = D / VEC, NP = VEC / 2, ROW = D * (int)sizeof(T);
     constexpr int GROUP = U * G * 32 * 16;  // bytes of one group of records, all lanes
     static_assert(2 * C <= 32, "dK and dV halves fit one warp");

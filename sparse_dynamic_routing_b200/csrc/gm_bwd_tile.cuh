@@ -113,6 +113,8 @@ __device__ __forceinline__ void ser_backward_row(const SeaBwdArgs &a, uint32_t r
 template <typename T, int D, int G, int S1M, int P, int WPB, bool GATHER, int SB = 0>
 __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_bwd_tile_kernel(SeaBwdArgs a)
 {
+    pdl_wait();  // the bucket offsets and ranks (gather mode), when launched after the scan
+    pdl_trigger();
     using TG = BwdTileGeom<T, D, G, S1M>;
     constexpr int VEC = TG::VEC, C = TG::C, RPW = TG::RPW, NP = VEC / 2;
     extern __shared__ __align__(16) char smem[];

@@ -182,6 +182,14 @@ template <int N> __device__ __forceinline__ void cp_async_wait()
     asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while the kernel before it on the stream is still running; pdl_wait() blocks
+// until that kernel has completed and its memory is visible (a no-op for a kernel launched
+// the ordinary way). pdl_trigger() lets the next such kernel launch early. Both are hardware
+// waits, not spin loops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- shared-memory barriers (mbarrier) with bounded waits --------------------------------
 //
 // Completion of asynchronous copies (TMA) and tensor-core operations is counted on 64-bit
