@@ -1,22 +1,24 @@
 // gm_bwd_tile.cuh - SEA backward, tiled for small edge budgets (s <= 4, head_dim 64/128).
 //
 // Same mathematics as sea_bwd_kernel (gm_sea_bwd.cuh); the work division of the tiled
-// forward (gm_fused_tile.cuh): a warp owns tiles of 32 consecutive edge rows; phase 1 loads
-// the tile's edges one thread per row into shared memory; phase 2 processes RPW rows per
-// pass with C lanes per row, each lane owning one 16-byte chunk of every feature row for all
-// G query heads, with its K and V chunks staged by the lane itself via cp.async P passes
-// ahead and its q and dO chunks read into registers one pass ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
+// forward (gm_fused_tile.cuh): a warp owns tiles of 32 consecutive edge rows (the last
+// round's shorter); phase 1 loads the tile's edges one thread per row into shared memory;
+// phase 2 processes RPW rows per pass with C lanes per row, each lane owning one 16-byte
+// chunk of every feature row for all G query heads, with its K and V chunks staged by the
+// lane itself via cp.async P passes ahead and its q and dO chunks read into registers one
+// pass ahead. Per row and query head, with z_j = scale q.k_j + ln w_j, p = softmax(z),
 // dp_j = dO.v_j, D = sum_j p_j dp_j and dz_j = p_j (dp_j - D):
 //   dq          = scale sum_j dz_j k_j                       (stored)
 //   dK[t_j]    += scale sum_heads dz_j q                     (GATHER = false: 16-byte fp32
 //   dV[t_j]    += sum_heads p_j dO                            vector atomics)
 //   dlogw[j]    = sum_heads dz_j                             (stored)
 // With GATHER = true the two scatter-adds are not done here: the kernel writes each active
-// edge's record (target row, source row, scale dz_g, p_g) into its target's bucket, and the
-// gather pass of gm_bwd_gather.cuh forms dK and dV.
+// edge's record (target row, source row, scale dz_g, p_g) at its place in its target's
+// bucket (the bucket offset plus the rank the count pass gave the edge), and the gather pass
+// of gm_bwd_gather.cuh forms dK and dV. With SB > 0 a third phase runs the referral backward
+// of the tile's rows (ser_backward_row).
 // Every shuffle runs on all 32 lanes (slots padded to S1M and masked after the reduction).
 #pragma once
-
 
 #include "gm_bwd_gather.cuh"
 #include "gm_common.cuh"

@@ -5,7 +5,8 @@
 // ("Graph Machine: Towards Better Pretraining via Edges", ai.info summary, "Main Findings":
 // 2 or 4 positions per KV head).
 //
-// A warp owns tiles of 32 consecutive edge rows (b, i, h).
+// A warp owns tiles of 32 consecutive edge rows (b, i, h), dealt in rounds over the whole
+// grid; the rows left after the full rounds are split evenly, so the last tiles are shorter.
 //  Phase 1 - referral, one thread per row. Lane L gathers its row's s2 first-leg slots and
 //    the s3 second-leg slots behind each (vector loads), forms the s2*s3 candidates in
 //    registers, merges duplicates in ascending candidate order (the first occurrence
@@ -24,7 +25,6 @@
 // All shuffles run on all 32 lanes: slots are padded to S1M and inactive ones masked after
 // the reduction, so rows at a ragged tail simply compute on zeros and store nothing.
 #pragma once
-
 
 #include "gm_common.cuh"
 #include "gm_sea.cuh"
