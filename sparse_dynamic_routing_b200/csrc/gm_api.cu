@@ -721,11 +721,11 @@ gm_status gm_ser_backward(const int32_t *a1_idx, const float *a1_w, int s2,
     const bool aligned = aligned16(a1_idx) && aligned16(a1_w) && aligned16(a2_idx) && aligned16(a2_w);
     const unsigned tblocks = blocks_for(rows, 32 * WPB_SER_THREAD);
     if (aligned && s2 == 4 && s3 == 4 && s1 <= 4) {
-        gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        launch_pdl(gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD>, tblocks, WPB_SER_THREAD * 32, 0, stream, b);
         return launched();
     }
     if (aligned && s2 == 2 && s3 == 2 && s1 <= 4) {
-        gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+        launch_pdl(gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD>, tblocks, WPB_SER_THREAD * 32, 0, stream, b);
         return launched();
     }
     gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);
@@ -861,11 +861,11 @@ gm_status gm_ser_refresh_backward(const int32_t *a1_idx, const float *a1_w, int 
     const unsigned tblocks = blocks_for(rows, 32 * WPB_SER_THREAD);
     if (aligned && s2 == s3 && (s2 == 2 || s2 == 4) && s1 <= 4 && (sf == 2 || sf == 4)) {
         if (s2 == 4)
-            sf == 4 ? gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 4><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b)
-                    : gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 2><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+            sf == 4 ? launch_pdl(gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 4>, tblocks, WPB_SER_THREAD * 32, 0, stream, b)
+                    : launch_pdl(gm::ser_bwd_thread_kernel<4, 4, 4, WPB_SER_THREAD, 2>, tblocks, WPB_SER_THREAD * 32, 0, stream, b);
         else
-            sf == 4 ? gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 4><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b)
-                    : gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 2><<<tblocks, WPB_SER_THREAD * 32, 0, stream>>>(b);
+            sf == 4 ? launch_pdl(gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 4>, tblocks, WPB_SER_THREAD * 32, 0, stream, b)
+                    : launch_pdl(gm::ser_bwd_thread_kernel<2, 2, 4, WPB_SER_THREAD, 2>, tblocks, WPB_SER_THREAD * 32, 0, stream, b);
         return launched();
     }
     gm::ser_bwd_kernel<WPB_SER><<<blocks_for(rows, WPB_SER), WPB_SER * 32, 0, stream>>>(b);

@@ -65,6 +65,7 @@ __device__ __forceinline__ float refer_step_backward(const ReferCand &c, unsigne
 template <int WPB>
 __global__ void __launch_bounds__(WPB * 32) ser_bwd_kernel(SerBwdArgs b)
 {
+    pdl_wait();  // the zeroed leg gradients (launched after the zero-fill)
     const SerArgs &a = b.f;
     const int lane = threadIdx.x & 31;
     const uint32_t row = blockIdx.x * WPB + (threadIdx.x >> 5);
@@ -229,6 +230,7 @@ __device__ __forceinline__ void refer_thread_backward(const SerArgs &a, uint32_t
 template <int S2, int S3, int S1M, int WPB, int SF = 0>
 __global__ void __launch_bounds__(WPB * 32) ser_bwd_thread_kernel(SerBwdArgs b)
 {
+    pdl_wait();  // the zeroed leg gradients (launched after the zero-fill)
     const SerArgs &a = b.f;
     const uint32_t row = blockIdx.x * (WPB * 32) + threadIdx.x;
     if (row >= a.rows) return;  // no warp-wide operation below
