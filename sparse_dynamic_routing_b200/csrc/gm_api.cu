@@ -486,7 +486,7 @@ template <typename T, int D, int G> struct SeaBwdGather {
                 launch_pdl(gm::edge_count_kernel<4>, cgrid, 256, 0, st, idx, w, a.n, a.map, a.s, a.rows, a.hkv,
                            ws.cnt, ws.rank);
             launch_pdl(gm::scan_lookback_kernel, ws.nblk, gm::SCAN_THREADS, 0, st, ws.cnt, R, ws.state, ws.ticket,
-                       ws.off);
+                       ws.off, a.dk, a.dv, D, a.accumulate);
             if (launched() != GM_OK) return GM_ERR_CUDA;
             a.rank = ws.rank;
             a.off = ws.off;

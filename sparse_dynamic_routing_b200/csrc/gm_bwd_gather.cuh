@@ -13,8 +13,10 @@
 //   4. the gather pass walks the sorted records in chunks of 32, one warp per chunk: a warp
 //      owns every target whose first record lies in its chunk (following it past the chunk
 //      end if needed), sums scale dz_g q_g into dK and p_g dO_g into dV, and writes each owned
-//      row once; the target rows nothing points at (count 0) are written as zeros, each
-//      warp of the grid taking an equal slice of all target rows.
+//      row once; a hot target (more than GATHER_HOT records, edges collapsed onto a few
+//      positions) is instead summed by every chunk it spans, each adding its part with fp32
+//      atomics into the row the scan zeroed; the target rows nothing points at (count 0) are
+//      written as zeros, each warp of the grid taking an equal slice of all target rows.
 // The order of records inside a bucket comes from the count pass's integer atomics and
 // varies run to run, so dK/dV sums vary in rounding order (not in the set of terms). The scan
 // is one launch with a decoupled look-back between its blocks; its waits are bounded.
@@ -24,9 +26,10 @@
 
 namespace gm {
 
-// A sorted record: target row, source edge row (b*n + i)*hkv + h, then scale dz_g and p_g
-// for the G query heads (fp32 bits), padded to whole 16-byte words (32 bytes for G = 2), so
-// the row pass writes and the gather pass reads it in full sectors.
+// A sorted record: target row, source edge row (b*n + i)*hkv + h with the target's hot bit in
+// bit 31, then scale dz_g and p_g for the G query heads (fp32 bits), padded to whole 16-byte
+// words (32 bytes for G = 2), so the row pass writes and the gather pass reads it in full
+// sectors.
 template <int G> struct Rec {
     static constexpr int WORDS = (2 + 2 * G + 3) / 4 * 4;
 };
@@ -76,6 +79,11 @@ struct GatherWs {
     uint32_t nblk;              // scan tiles of SCAN_TILE rows
     int64_t zero_words;
 };
+
+// A target row with more records than this is "hot" (edges collapsed onto a few positions):
+// instead of one warp walking all of its records, every chunk sums its own part and adds it
+// with fp32 atomics into the row, which the scan zeroes beforehand.
+constexpr int GATHER_HOT = 256;
 
 constexpr int SCAN_THREADS = 1024;
 constexpr int SCAN_PER_THREAD = 4;
@@ -139,7 +147,8 @@ constexpr unsigned long long SCAN_AGGREGATE = 1ull << 32, SCAN_PREFIX = 2ull << 
 // bounded (WAIT_LIMIT_NS, then ERR_WAIT_TIMEOUT and a wrong prefix instead of a hang).
 __global__ void __launch_bounds__(SCAN_THREADS) scan_lookback_kernel(const int32_t *cnt, int64_t R,
                                                                      unsigned long long *state, uint32_t *ticket,
-                                                                     int32_t *off)
+                                                                     int32_t *off, float *dk, float *dv, int D,
+                                                                     int accumulate)
 {
     __shared__ uint32_t s_tile;
     __shared__ int32_t s_prefix;
@@ -201,6 +210,20 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_lookback_kernel(const int32
         run += c[k];
     }
     if (tile == gridDim.x - 1 && threadIdx.x == 0) off[R] = s_prefix + total;
+    // hot rows receive atomic additions in the gather pass: start them at zero
+    if (!accumulate) {
+#pragma unroll
+        for (int k = 0; k < SCAN_PER_THREAD; ++k) {
+            if (base + k < R && c[k] > GATHER_HOT) {
+                float4 *pk = reinterpret_cast<float4 *>(dk + (size_t)(base + k) * D);
+                float4 *pv = reinterpret_cast<float4 *>(dv + (size_t)(base + k) * D);
+                for (int x = 0; x < D / 4; ++x) {
+                    pk[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    pv[x] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+        }
+    }
 }
 
 // Count: active edges per target row, and each active edge's rank among them (range errors
@@ -257,12 +280,18 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
 #pragma unroll
     for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
 
-    auto write_row = [&](uint32_t t) {  // acc -> row t (added to it when accumulating)
+    // acc -> row t: stored (added to it when accumulating), or for a hot row added with fp32
+    // atomics (the row was zeroed by the scan unless accumulating)
+    auto write_row = [&](uint32_t t, bool hot) {
         if (!working) return;
         float *dst = dst_base + (size_t)t * D;
 #pragma unroll
         for (int x = 0; x < NP; x += 2) {
             float4 o = make_float4(acc[x].x, acc[x].y, acc[x + 1].x, acc[x + 1].y);
+            if (hot) {
+                atomicAdd(reinterpret_cast<float4 *>(dst + 2 * x), o);
+                continue;
+            }
             if (accumulate) {
                 const float4 old = *reinterpret_cast<const float4 *>(dst + 2 * x);
                 o.x += old.x; o.y += old.y; o.z += old.z; o.w += old.w;
@@ -302,6 +331,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
         int64_t wbase = p0;
         int wlen = (int)min((int64_t)32, (int64_t)total - wbase);
         int32_t mkey = -1, mrow = 0;
+        bool mhot = false;
         float mcf[2 * G];
         auto load_window = [&]() {
             mkey = -1;
@@ -309,15 +339,21 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
     #pragma unroll
             for (int x = 0; x < 2 * G; ++x) mcf[x] = 0.0f;
             if (lane < wlen) read_record<G>(ws.srec, wbase + lane, mkey, mrow, mcf);
+            mhot = mrow < 0;  // bit 31: the target is hot
+            mrow &= 0x7fffffff;
         };
         load_window();
         const int32_t prev_key = p0 > 0 ? __ldg(ws.srec + (p0 - 1) * Rec<G>::WORDS) : -1;
 
-        // a leading run that continues the previous chunk's last target belongs to that chunk
+        // a leading run that continues the previous chunk's last target belongs to that chunk,
+        // unless the target is hot: then every chunk sums its own part of it
         const int start = __popc(__ballot_sync(FULL, lane < wlen && mkey == prev_key));
-        if (start == wlen) return;  // warp-uniform
+        const bool lead_hot = start > 0 && __shfl_sync(FULL, mhot, 0);  // warp-uniform
+        const int first = lead_hot ? 0 : start;
+        if (first == wlen) return;  // warp-uniform
 
-        uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, start);
+        uint32_t cur = (uint32_t)__shfl_sync(FULL, mkey, first);
+        bool cur_hot = lead_hot;  // a target starting inside the chunk is settled at its end
 
         // Accumulate records [lo, hi) of the current window, U per copy group, P groups in
         // flight; a change of key writes the finished target (and zeroes any empty rows between).
@@ -350,7 +386,8 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
                     for (int x = 0; x < 2 * G; ++x) cf[x] = __shfl_sync(FULL, mcf[x], k & 31);
                     if (k >= hi) break;  // warp-uniform
                     if (key != cur) {    // warp-uniform: a new target starts here
-                        write_row(cur);
+                        write_row(cur, cur_hot);
+                        cur_hot = false;  // it starts inside the window
     #pragma unroll
                         for (int x = 0; x < NP; ++x) acc[x] = make_float2(0.0f, 0.0f);
                         cur = key;
@@ -373,11 +410,13 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
             cp_async_wait<0>();
         };
 
-        process(start, wlen);
-        // the last owned target may continue past the chunk (hot rows): follow it window by
-        // window with the same pipeline
+        process(first, wlen);
+        // the last target may continue past the chunk: a hot one is left to the chunks it
+        // spans (each adds its part), any other is followed window by window with the same
+        // pipeline
         int64_t pos = wbase + wlen;
-        while (wlen == 32 && pos < total) {
+        if (!cur_hot) cur_hot = __shfl_sync(FULL, mhot, wlen - 1);  // the last record is cur's
+        while (!cur_hot && wlen == 32 && pos < total) {
             wbase = pos;
             wlen = (int)min((int64_t)32, (int64_t)total - wbase);
             load_window();
@@ -387,7 +426,7 @@ __global__ void __launch_bounds__(WPB * 32) sea_bwd_gather_kernel(const void *q,
             pos = wbase + run;
             if (run < wlen) break;  // the target ended inside this window
         }
-        write_row(cur);
+        write_row(cur, cur_hot);
     };
     walk();
     zero_slice();

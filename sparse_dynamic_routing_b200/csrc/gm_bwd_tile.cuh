@@ -186,9 +186,17 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 const uint32_t key = (seq_base + (uint32_t)t) * (uint32_t)a.hkv + h;
                 tile_t[lane * S1M + r] = (int32_t)key;
                 tile_lw[lane * S1M + r] = lw;
-                if constexpr (GATHER)  // the count pass applied the same activity test
-                    tile_pos[lane * S1M + r] =
-                        lw != -INFINITY ? __ldg(a.off + key) + __ldg(a.rank + (size_t)row * a.s + r) : -1;
+                if constexpr (GATHER) {  // the count pass applied the same activity test
+                    // the record's place, and in bit 31 whether its target is hot (its bucket
+                    // holds more than GATHER_HOT records; the gather pass splits those)
+                    int32_t pos = -1;
+                    if (lw != -INFINITY) {
+                        const int32_t o0 = __ldg(a.off + key), o1 = __ldg(a.off + key + 1);
+                        pos = o0 + __ldg(a.rank + (size_t)row * a.s + r);
+                        if (o1 - o0 > GATHER_HOT) pos |= (int32_t)0x80000000u;
+                    }
+                    tile_pos[lane * S1M + r] = pos;
+                }
                 if constexpr (SB > 0) {
                     tile_tt[lane * S1M + r] = t;
                     tile_w[lane * S1M + r] = lw == -INFINITY ? 0.0f : __ldg(a.w + (size_t)row * a.s + r);
@@ -438,10 +446,13 @@ __global__ void __launch_bounds__(WPB * 32, GATHER ? GM_BWD_TILE_MINB : 4) sea_b
                 }
                 if (c < S1M && mine) {
                     const uint32_t key = (uint32_t)tile_t[lr * S1M + c];
-                    const int32_t pos = tile_pos[lr * S1M + c];
+                    const uint32_t tp = (uint32_t)tile_pos[lr * S1M + c];
+                    const uint32_t pos = tp & 0x7fffffffu;
                     // the count pass applies the same activity test, so pos stays inside the
-                    // bucket; the bound only keeps a broken invariant from writing outside
-                    if ((uint32_t)pos < a.rows * (uint32_t)a.s) write_record<G>(a.srec, pos, key, row, rc);
+                    // bucket; the bound only keeps a broken invariant from writing outside.
+                    // The hot bit travels in bit 31 of the source row (rows < 2^31).
+                    if (pos < a.rows * (uint32_t)a.s)
+                        write_record<G>(a.srec, (int32_t)pos, key, row | (tp & 0x80000000u), rc);
                 }
             }
             if (valid) {

@@ -173,6 +173,13 @@ def test_backward_paths_on_hot_rows():
                                  workspace=ws)
         for name, a_, b_ in zip(("dq", "dk", "dv", "dlogw"), got, ref[:4]):
             assert_close(a_, b_, TOL["bf16"], f"{name} ({ws})")
+        # accumulating onto the first result: the hot rows (more than a few hundred records
+        # each here) take the gather pass's atomic route without the zero-fill
+        again = gm.gm_sea_backward(g["q"], g["k"], g["v"], g["dout"], g["idx"], g["w"], scale,
+                                   dq=got[0], dk=got[1], dv=got[2], dlogw=got[3], workspace=ws,
+                                   accumulate=True)
+        for name, a_, b_ in zip(("dq", "dk", "dv", "dlogw"), again, ref[:4]):
+            assert_close(a_, 2.0 * b_, 2 * TOL["bf16"], f"{name} accumulated ({ws})")
     gm.gm_check_device_errors()
 
 
