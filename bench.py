@@ -598,8 +598,9 @@ def measure_extra(gm, wl, g, x, ap_i, ap_w, dlw, dev, stream, peak, reps=20):
     f_dw2 = torch.empty((B, n, k, wl.s3), dtype=f32, device=dev)
     f_ws = torch.empty(gm.gm_sea_backward_workspace_size(g["q"].dtype, wl.s1, B, n, wl.hq, k, wl.d),
                        dtype=torch.uint8, device=dev)
-    # the two halves of the fused forward as separate calls (the unfused entry points gm_ser_forward and
-    # gm_sea_forward), and the two in sequence: A' makes one round trip through HBM
+    # the two halves of the fused forward as separate calls (the unfused entry points
+    # gm_ser_forward and gm_sea_forward), and the two in sequence: A' makes one round trip
+    # through HBM
     fd = compulsory_bytes(wl, x["a1_idx"].numpy(), x["a1_w"].numpy(), ap_i.cpu().numpy(),
                           ap_w.cpu().numpy())["detail"]["fused_forward"]
     ser_b = fd["a1"] + fd["a2_rows"] + fd["a_prime"]
