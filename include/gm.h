@@ -371,7 +371,9 @@ gm_status gm_ser_sea_forward(const int32_t *a1_idx, const float *a1_w, int s2,
  * Two execution paths:
  *   - with a workspace (workspace != NULL and the shape is covered, see
  *     gm_sea_backward_workspace_size): dk/dv are gathered per target row from a reverse
- *     edge index built in the workspace; each dk/dv row is written once, no atomics on them;
+ *     edge index built in the workspace; each dk/dv row is written once, without atomics,
+ *     except the rows more than 256 slots point at, which are zeroed and then summed by
+ *     several warps with 16-byte fp32 atomics;
  *   - without one: dk/dv are zeroed by a library kernel (unless accumulating) and
  *     scatter-added with 16-byte fp32 atomics.
  *
