@@ -420,8 +420,11 @@ template <typename T, int D, int G> struct SeaBwd {
 #define GM_GATHER_P 2
 #endif
 #ifndef GM_WPB_GATHER
-#define GM_WPB_GATHER 2
+#define GM_WPB_GATHER 1
 #endif
+// One warp per block: a block's resources are freed as soon as its one chunk is done, so
+// chunks that follow a long target past their end hold back no other warp (at B = 8, n = 4096:
+// 294 -> 284 us for the backward, against two warps per block).
 constexpr int WPB_GATHER = GM_WPB_GATHER;
 constexpr int GATHER_U = GM_GATHER_U;  // records per copy group
 constexpr int GATHER_P = GM_GATHER_P;  // copy groups in flight per warp
