@@ -256,11 +256,11 @@ template <int S, typename V> __device__ __forceinline__ void ld_tile(const V *p,
     }
 }
 
-// Resident 4-warp blocks per SM the forward tile kernel is compiled for: caps registers at
+// Resident one-warp blocks per SM the forward tile kernel is compiled for: caps registers at
 // 65536 / (32 * WPB * MINB) without spills. With two stages in flight shared memory admits
-// six; with one, registers (73 at seven blocks) are the limit.
+// 24 warps; with one, registers (73 at 28 warps) are the limit.
 #ifndef GM_TILE_MINB
-#define GM_TILE_MINB(P) ((P) == 1 ? 7 : 6)
+#define GM_TILE_MINB(P) ((P) == 1 ? 28 : 24)
 #endif
 
 template <typename T, int D, int G, int S1M, int CPL = 1> struct TileGeom {

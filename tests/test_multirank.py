@@ -19,13 +19,16 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, store_path, out):
+    # the variables torchrun sets (read by bench.dist_env); the rendezvous itself goes through
+    # a file store and the loopback interface, so no port can be taken in between
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
-                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank), GLOO_SOCKET_IFNAME="lo")
     import bench
     from sparse_dynamic_routing_b200 import inputs as I
 
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+    dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank,
+                            world_size=world)
     try:
         r, w, local = bench.dist_env()
         assert (r, w, local) == (rank, world, rank)
@@ -39,12 +42,13 @@ def _worker(rank, world, port, out):
         dist.destroy_process_group()
 
 
-def test_two_ranks_weak_scaling_and_max_timing():
+def test_two_ranks_weak_scaling_and_max_timing(tmp_path):
     ctx = mp.get_context("spawn")
     mgr = ctx.Manager()
     out = mgr.dict()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, out)) for r in range(2)]
+    store = str(tmp_path / "store")
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, store, out)) for r in range(2)]
     for p in procs:
         p.start()
     for p in procs:
